@@ -1,0 +1,189 @@
+/*
+ * pa.h -- C ABI of the B200 paged KV-cache decode library (libpa.so).
+ *
+ * The operation is PagedAttention decode as the pages describe it: each
+ * sequence's KV cache lives in fixed-size physical blocks (16 or 32 tokens;
+ * "vLLM Architecture, Memory and Benchmarks Deep Dive", section 2), a
+ * per-sequence block table maps logical blocks to physical ones so that the
+ * paged cache looks contiguous to attention ("Optimizing LLM Inference: A Deep
+ * Dive into vLLM's PagedAttention and Continuous Batching", section
+ * "PagedAttention: Borrowing a 50-Year-Old OS Masterpiece"), new tokens go into
+ * blocks handed out on demand (same page as the first, section 2, "On-Demand
+ * Allocation"), and query heads share KV heads (grouped-query attention, same
+ * page, section 1).
+ *
+ * Conventions shared by every call
+ *   - Pointers named as device pointers must point to memory of the current
+ *     CUDA device; the caller owns all memory.  The library never allocates,
+ *     frees or synchronises; each call enqueues its kernels on `stream` (a
+ *     cudaStream_t; NULL = the legacy default stream) and returns.
+ *   - Tensors are dense and row-major (C order).  Shapes use
+ *       B   = num_seqs (one new token per sequence),
+ *       Hq  = num_q_heads, Hkv = num_kv_heads (Hq / Hkv in {1, 2, 4, 8}),
+ *       d   = head_dim in {64, 128, 256},
+ *       bs  = block_size in {4, 8, 16, 32},
+ *       nb  = num_blocks (physical blocks in each pool).
+ *     K and V pools are [nb, bs, Hkv, d]; token t of sequence b lives in
+ *     physical block block_tables[b * max_blocks + t / bs], row t % bs.
+ *   - Query head hq attends with KV head hq / (Hq / Hkv).
+ *   - context_lens[b] counts every cached token of sequence b including the
+ *     one being decoded; a length of 0 gives a zero output.
+ *   - Element types: PA_DTYPE_F32 (binary32) or PA_DTYPE_BF16 (bfloat16).
+ *     Attention accumulates in fp32 and writes `out` in the input type.
+ *   - Base pointers of element arrays must be 16-byte aligned.
+ *   - Errors the host can see (null pointer, unsupported shape, workspace too
+ *     small) return a status and launch nothing.  Errors only the device can
+ *     see never trap: the kernel ORs a PA_DEV_* bit into *dev_status (if
+ *     dev_status is not NULL), skips the offending access, and the affected
+ *     output is zeros (attention) or left untouched (cache write).
+ *   - Inputs and outputs must not overlap.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, Hq % Hkv != 0, ... */
+    PA_ERR_UNSUPPORTED = 2,  /* head_dim / block_size / group / dtype not built */
+    PA_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed */
+    PA_ERR_WORKSPACE = 4     /* caller-provided workspace too small */
+} pa_status;
+
+typedef enum pa_dtype {
+    PA_DTYPE_F32 = 0,
+    PA_DTYPE_BF16 = 1
+} pa_dtype;
+
+/* Bits a kernel ORs into *dev_status. */
+#define PA_DEV_BAD_SLOT 0x1      /* cache write: slot >= nb * bs (row not written) */
+#define PA_DEV_BAD_BLOCK 0x2     /* a block-table entry read is outside [0, nb) */
+#define PA_DEV_BAD_CONTEXT 0x4   /* context_lens[b] < 0 or > max_blocks * bs */
+#define PA_DEV_WAIT_TIMEOUT 0x8  /* a bounded wait for an async copy ran out */
+
+/*
+ * pa_reshape_and_cache -- store each new token's K and V into its slot.
+ *
+ * Source: the new token's KV is kept in the block handed out for it
+ * ("vLLM Architecture, Memory and Benchmarks Deep Dive", section 2, "On-Demand
+ * Allocation"; section 1 for what the KV cache holds).
+ *
+ *   key, value    device, [num_tokens, Hkv, d], read only.
+ *   k_pool,v_pool device, [nb, bs, Hkv, d]; row (slot / bs, slot % bs) of
+ *                 every head is overwritten for each token with slot >= 0.
+ *   slot_mapping  device, [num_tokens] int64.  A negative slot means padding:
+ *                 the token is skipped.  A slot >= nb * bs sets
+ *                 PA_DEV_BAD_SLOT and the token is skipped.
+ *   The copy is bit-exact; nothing else in the pools changes.  Two tokens
+ *   with the same slot race (one of them wins).
+ */
+pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_pool, void *v_pool,
+                               const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
+                               int32_t *dev_status, void *stream);
+
+/*
+ * pa_decode_attention -- single-query GQA attention over the paged cache.
+ *
+ *   out[b, hq, :] = sum_t p_t V[t, hq / G, :] / sum_t p_t,
+ *   p_t = exp(s_t - max_t s_t),  s_t = scale * q[b, hq, :] . K[t, hq / G, :],
+ * over the tokens t < context_lens[b] of sequence b, gathered through its
+ * block table (the definition above is exact softmax attention; the library
+ * computes it with an online softmax in fp32 and, for long contexts, a
+ * flash-decoding split of the context into partitions merged by the
+ * log-sum-exp rule).
+ *
+ *   out            device, [B, Hq, d], written.
+ *   query          device, [B, Hq, d].
+ *   k_pool,v_pool  device, [nb, bs, Hkv, d].
+ *   block_tables   device, [B, max_blocks_per_seq] int32; entries at or past
+ *                  ceil(context_lens[b] / bs) are never read.
+ *   context_lens   device, [B] int32.
+ *   max_context_len host hint, >= every context_lens[b]; used to size the
+ *                  split.  Must be <= max_blocks_per_seq * bs.
+ *   scale          softmax scale (usually 1 / sqrt(d)).
+ *   workspace      device scratch of workspace_bytes bytes (may be NULL / 0).
+ *                  pa_decode_workspace_bytes() gives the size the library
+ *                  wants for its preferred split; with less (or none) it uses
+ *                  fewer, longer partitions, down to no split at all, so any
+ *                  size is correct.  Contents need no initialisation and are
+ *                  garbage afterwards.  Calls that share a workspace must not
+ *                  run concurrently.
+ *   dev_status     device int32 or NULL (see PA_DEV_*).
+ */
+pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
+                              const void *v_pool, const int32_t *block_tables,
+                              int max_blocks_per_seq, const int32_t *context_lens, int num_seqs,
+                              int max_context_len, int num_q_heads, int num_kv_heads,
+                              int head_dim, int block_size, int64_t num_blocks, float scale,
+                              pa_dtype dtype, void *workspace, size_t workspace_bytes,
+                              int32_t *dev_status, void *stream);
+
+/* Workspace bytes pa_decode_attention wants for these sizes (0 = it will not
+ * split).  Host only; touches no device. */
+size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
+                                 int max_context_len);
+
+/* ceil(max_context_len / partition_size), at least 1. Host only. */
+int pa_num_partitions(int max_context_len, int partition_size);
+
+/* Bytes of the three split-K buffers below for max_partitions partitions:
+ * tmp_out B*Hq*P*d floats, max_logits and exp_sums B*Hq*P floats each.
+ * Host only. */
+size_t pa_splitk_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
+                                 int max_partitions);
+
+/*
+ * pa_decode_splitk -- the partition pass of flash-decoding, made explicit.
+ *
+ * Partition p of sequence b covers tokens [p * P, min((p + 1) * P, ctx_b)),
+ * P = partition_size (a multiple of 16), for p < n_b = max(1, ceil(ctx_b/P)).
+ * For every (b, hq, p < n_b) it writes
+ *   max_logits[b, hq, p]      m_p = max logit s_t over the partition,
+ *   exp_sums[b, hq, p]        l_p = sum exp(s_t - m_p),
+ *   tmp_out[b, hq, p, :]      sum exp(s_t - m_p) V_t / l_p,
+ * with logits in natural-log units (s_t = scale * q . k).  An empty
+ * partition (ctx_b = 0) gives m = -inf, l = 0, tmp = 0.  Entries with
+ * p >= n_b are not touched.  For sequences with n_b == 1 it also writes the
+ * final out[b, :, :]; pa_splitk_reduce finishes the others.
+ *   max_partitions >= ceil(max_context_len / P); buffers as in
+ *   pa_splitk_workspace_bytes, device, fp32.  Other arguments as in
+ *   pa_decode_attention.
+ */
+pa_status pa_decode_splitk(void *out, const void *query, const void *k_pool, const void *v_pool,
+                           const int32_t *block_tables, int max_blocks_per_seq,
+                           const int32_t *context_lens, int num_seqs, int max_context_len,
+                           int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int64_t num_blocks, float scale, pa_dtype dtype, int partition_size,
+                           int max_partitions, float *tmp_out, float *max_logits,
+                           float *exp_sums, int32_t *dev_status, void *stream);
+
+/*
+ * pa_splitk_reduce -- merge the partitions of every sequence with n_b > 1:
+ *   M = max_p m_p,  w_p = l_p exp(m_p - M),
+ *   out[b, hq, :] = sum_p w_p tmp_out[b, hq, p, :] / sum_p w_p.
+ * Sequences with n_b == 1 are left alone (pa_decode_splitk wrote them).
+ * Arguments as in pa_decode_splitk; out is written in `dtype`.
+ */
+pa_status pa_splitk_reduce(void *out, const float *tmp_out, const float *max_logits,
+                           const float *exp_sums, const int32_t *context_lens, int num_seqs,
+                           int num_q_heads, int head_dim, int partition_size,
+                           int max_partitions, pa_dtype dtype, void *stream);
+
+/* Static description of a status code. */
+const char *pa_status_string(pa_status status);
+
+/* Number of kernels this library has launched in this process. */
+unsigned long long pa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,204 @@
+"""Python binding of libpa.so (argument marshalling only).
+
+Every function here takes torch tensors, checks that their shapes, dtypes and
+devices agree, derives the sizes the C ABI wants, and calls the C function of
+the same name on the current CUDA stream.  All computation happens in the
+library's CUDA kernels; there is no fallback.  If libpa.so is missing this
+module fails to import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} not found: build it with `python -m paged_kv_cache_455_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_F = ctypes.c_float
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE = range(5)
+PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
+PA_DEV_BAD_SLOT, PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_WAIT_TIMEOUT = 1, 2, 4, 8
+
+# Every symbol include/pa.h declares, with its C signature.
+SIGNATURES = {
+    "pa_reshape_and_cache": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _P, _P]),
+    "pa_decode_attention": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F,
+                                 _I, _P, _SZ, _P, _P]),
+    "pa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "pa_num_partitions": (_I, [_I, _I]),
+    "pa_splitk_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "pa_decode_splitk": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I,
+                              _I, _I, _P, _P, _P, _P, _P]),
+    "pa_splitk_reduce": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "pa_status_string": (ctypes.c_char_p, [_I]),
+    "pa_launch_count": (ctypes.c_ulonglong, []),
+}
+for _name, (_res, _args) in SIGNATURES.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.pa_status_string(status).decode()} (status {status})")
+
+
+def _check(status: int, where: str) -> None:
+    if status != PA_OK:
+        raise PaError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return PA_DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return PA_DTYPE_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _cuda(*tensors) -> None:
+    for t in tensors:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def launch_count() -> int:
+    return int(lib.pa_launch_count())
+
+
+def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
+                              max_context_len: int) -> int:
+    return int(lib.pa_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len))
+
+
+def pa_num_partitions(max_context_len: int, partition_size: int) -> int:
+    return int(lib.pa_num_partitions(max_context_len, partition_size))
+
+
+def pa_splitk_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
+                              max_partitions: int) -> int:
+    return int(lib.pa_splitk_workspace_bytes(num_seqs, num_q_heads, head_dim, max_partitions))
+
+
+def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_pool: torch.Tensor,
+                         v_pool: torch.Tensor, slot_mapping: torch.Tensor,
+                         dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """key/value [T, Hkv, d]; pools [nb, bs, Hkv, d]; slot_mapping [T] int64."""
+    _cuda(key, value, k_pool, v_pool, slot_mapping, dev_status)
+    T, hkv, d = key.shape
+    nb, bs = k_pool.shape[:2]
+    if value.shape != key.shape or v_pool.shape != k_pool.shape or k_pool.shape[2:] != (hkv, d):
+        raise ValueError("shape mismatch")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (T,):
+        raise ValueError("slot_mapping must be int64 [T]")
+    if not (key.dtype == value.dtype == k_pool.dtype == v_pool.dtype):
+        raise ValueError("dtype mismatch")
+    _check(lib.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_pool), _ptr(v_pool),
+                                    _ptr(slot_mapping), T, hkv, d, bs, nb, _dtype_code(key),
+                                    _ptr(dev_status), _stream(stream)), "pa_reshape_and_cache")
+
+
+def _attn_sizes(out, query, k_pool, v_pool, block_tables, context_lens):
+    _cuda(out, query, k_pool, v_pool, block_tables, context_lens)
+    B, hq, d = query.shape
+    nb, bs, hkv, d2 = k_pool.shape
+    if out.shape != query.shape or v_pool.shape != k_pool.shape or d2 != d:
+        raise ValueError("shape mismatch")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("block_tables must be int32 [B, max_blocks]")
+    if context_lens.dtype != torch.int32 or context_lens.shape != (B,):
+        raise ValueError("context_lens must be int32 [B]")
+    if not (out.dtype == query.dtype == k_pool.dtype == v_pool.dtype):
+        raise ValueError("dtype mismatch")
+    return B, hq, hkv, d, bs, nb, block_tables.shape[1]
+
+
+def pa_decode_attention(out: torch.Tensor, query: torch.Tensor, k_pool: torch.Tensor,
+                        v_pool: torch.Tensor, block_tables: torch.Tensor,
+                        context_lens: torch.Tensor, max_context_len: int, scale: float,
+                        workspace: Optional[torch.Tensor] = None,
+                        dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out, query [B, Hq, d]; pools [nb, bs, Hkv, d]; block_tables [B, max_blocks]
+    int32; context_lens [B] int32; workspace: any contiguous CUDA tensor (its
+    bytes are used) or None."""
+    B, hq, hkv, d, bs, nb, maxb = _attn_sizes(out, query, k_pool, v_pool, block_tables,
+                                              context_lens)
+    _cuda(workspace, dev_status)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_attention(_ptr(out), _ptr(query), _ptr(k_pool), _ptr(v_pool),
+                                   _ptr(block_tables), maxb, _ptr(context_lens), B,
+                                   int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+                                   _dtype_code(query), _ptr(workspace), ws_bytes,
+                                   _ptr(dev_status), _stream(stream)), "pa_decode_attention")
+
+
+def pa_decode_splitk(out: torch.Tensor, query: torch.Tensor, k_pool: torch.Tensor,
+                     v_pool: torch.Tensor, block_tables: torch.Tensor,
+                     context_lens: torch.Tensor, max_context_len: int, scale: float,
+                     partition_size: int, tmp_out: torch.Tensor, max_logits: torch.Tensor,
+                     exp_sums: torch.Tensor, dev_status: Optional[torch.Tensor] = None,
+                     stream=None) -> None:
+    """tmp_out [B, Hq, P, d] fp32; max_logits, exp_sums [B, Hq, P] fp32."""
+    B, hq, hkv, d, bs, nb, maxb = _attn_sizes(out, query, k_pool, v_pool, block_tables,
+                                              context_lens)
+    _cuda(tmp_out, max_logits, exp_sums, dev_status)
+    P = tmp_out.shape[2]
+    if tmp_out.shape != (B, hq, P, d) or max_logits.shape != (B, hq, P) or \
+            exp_sums.shape != (B, hq, P):
+        raise ValueError("split-K buffer shape mismatch")
+    if not (tmp_out.dtype == max_logits.dtype == exp_sums.dtype == torch.float32):
+        raise ValueError("split-K buffers must be float32")
+    _check(lib.pa_decode_splitk(_ptr(out), _ptr(query), _ptr(k_pool), _ptr(v_pool),
+                                _ptr(block_tables), maxb, _ptr(context_lens), B,
+                                int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+                                _dtype_code(query), int(partition_size), P, _ptr(tmp_out),
+                                _ptr(max_logits), _ptr(exp_sums), _ptr(dev_status),
+                                _stream(stream)), "pa_decode_splitk")
+
+
+def pa_splitk_reduce(out: torch.Tensor, tmp_out: torch.Tensor, max_logits: torch.Tensor,
+                     exp_sums: torch.Tensor, context_lens: torch.Tensor, partition_size: int,
+                     stream=None) -> None:
+    _cuda(out, tmp_out, max_logits, exp_sums, context_lens)
+    B, hq, P, d = tmp_out.shape
+    if out.shape != (B, hq, d):
+        raise ValueError("shape mismatch")
+    _check(lib.pa_splitk_reduce(_ptr(out), _ptr(tmp_out), _ptr(max_logits), _ptr(exp_sums),
+                                _ptr(context_lens), B, hq, d, int(partition_size), P,
+                                _dtype_code(out), _stream(stream)), "pa_splitk_reduce")
+
+
+__all__ = [
+    "lib", "LIB_PATH", "SIGNATURES", "PaError", "launch_count",
+    "pa_reshape_and_cache", "pa_decode_attention", "pa_decode_workspace_bytes",
+    "pa_num_partitions", "pa_splitk_workspace_bytes", "pa_decode_splitk", "pa_splitk_reduce",
+    "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA", "PA_ERR_WORKSPACE",
+    "PA_DTYPE_F32", "PA_DTYPE_BF16",
+    "PA_DEV_BAD_SLOT", "PA_DEV_BAD_BLOCK", "PA_DEV_BAD_CONTEXT", "PA_DEV_WAIT_TIMEOUT",
+]

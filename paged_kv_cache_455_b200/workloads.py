@@ -197,11 +197,16 @@ def _fragment_history(rng: np.random.Generator, alloc: FifoBlockAllocator, bs: i
     return done
 
 
-def make_layout(cfg: DecodeConfig, length_scale: float = 1.0) -> BatchLayout:
+def shard_seed(cfg: DecodeConfig, shard: int) -> int:
+    """Seed of data-parallel shard ``shard`` (shard 0 is the config's seed)."""
+    return cfg.seed + 7919 * shard
+
+
+def make_layout(cfg: DecodeConfig, length_scale: float = 1.0, shard: int = 0) -> BatchLayout:
     """Draws lengths and block tables for ``cfg`` from numpy's generator seeded
-    with ``cfg.seed``.  ``length_scale`` < 1 shrinks every length (used only to
-    fit the memory-pressure pool into free device memory)."""
-    rng = np.random.default_rng(cfg.seed)
+    with ``shard_seed(cfg, shard)``.  ``length_scale`` < 1 shrinks every length
+    (used only to fit the memory-pressure pool into free device memory)."""
+    rng = np.random.default_rng(shard_seed(cfg, shard))
     lens = draw_context_lens(cfg, rng)
     if length_scale != 1.0:
         lens = np.maximum(1, np.rint(lens * length_scale)).astype(np.int64)
@@ -239,6 +244,7 @@ def make_layout(cfg: DecodeConfig, length_scale: float = 1.0) -> BatchLayout:
         if ctx > 0:
             last = ctx - 1
             slots[b] = int(tables[b, last // bs]) * bs + last % bs
+    notes["shard"] = shard
     return BatchLayout(cfg, lens.astype(np.int32), tables, slots, nb, length_scale, notes)
 
 
@@ -298,12 +304,12 @@ def _fill_pool(pool_rows: torch.Tensor, slots: torch.Tensor, gen: torch.Generato
 def make_layers(layout: BatchLayout, device, layers: Optional[int] = None,
                 chunk_rows: int = 1 << 16) -> List[LayerTensors]:
     """Draws every layer's tensors with a torch generator on ``device`` seeded
-    with ``cfg.seed``.  Values are N(0,1) drawn in fp32 and cast to the
+    with the layout's shard seed.  Values are N(0,1) drawn in fp32 and cast to the
     config's dtype; pool slots outside ``valid_slots`` are NaN."""
     cfg = layout.config
     device = torch.device(device)
     gen = torch.Generator(device=device)
-    gen.manual_seed(cfg.seed)
+    gen.manual_seed(shard_seed(cfg, int(layout.notes.get("shard", 0))))
     nl = cfg.layers if layers is None else layers
     slots = torch.from_numpy(valid_slots(layout)).to(device)
     B, hq, hkv, d = cfg.num_seqs, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim

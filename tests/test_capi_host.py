@@ -1,0 +1,129 @@
+"""libpa.so loads on a CPU-only machine, exports every symbol include/pa.h
+declares, and rejects bad arguments on the host without touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from paged_kv_cache_455_b200 import build
+    build.build()
+    from paged_kv_cache_455_b200 import pa as mod
+    return mod
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(pa):
+    names = _declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(pa.lib, n), f"{n} declared in pa.h but not exported"
+        assert n in pa.SIGNATURES, f"{n} has no binding"
+
+
+def test_status_strings(pa):
+    assert pa.lib.pa_status_string(0) == b"ok"
+    for s in range(1, 5):
+        assert pa.lib.pa_status_string(s) not in (b"ok", b"unknown status")
+    assert pa.lib.pa_status_string(99) == b"unknown status"
+
+
+def test_size_helpers(pa):
+    assert pa.pa_num_partitions(8192, 256) == 32
+    assert pa.pa_num_partitions(8193, 256) == 33
+    assert pa.pa_num_partitions(0, 256) == 1
+    assert pa.pa_splitk_workspace_bytes(8, 16, 256, 32) == 8 * 16 * 32 * (256 + 2) * 4
+    assert pa.pa_decode_workspace_bytes(64, 16, 256, 256) == 0          # no split
+    assert pa.pa_decode_workspace_bytes(8, 16, 256, 8192) == 8 * 16 * 32 * 258 * 4
+
+
+# Fake device addresses: every call below fails validation before any CUDA
+# call, so none of them is dereferenced.
+A = 0x10000          # 16-byte aligned
+M = 0x10008          # misaligned
+
+
+def _attn(pa, **kw):
+    args = dict(out=A, query=A, k_pool=A, v_pool=A, block_tables=A, max_blocks=4,
+                context_lens=A, num_seqs=3, max_ctx=16, hq=8, hkv=2, d=64, bs=4, nb=16,
+                scale=0.125, dtype=0, ws=None, ws_bytes=0, status=None, stream=None)
+    args.update(kw)
+    a = args
+    return pa.lib.pa_decode_attention(a["out"], a["query"], a["k_pool"], a["v_pool"],
+                                      a["block_tables"], a["max_blocks"], a["context_lens"],
+                                      a["num_seqs"], a["max_ctx"], a["hq"], a["hkv"], a["d"],
+                                      a["bs"], a["nb"], a["scale"], a["dtype"], a["ws"],
+                                      a["ws_bytes"], a["status"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(out=None), 1), (dict(query=None), 1), (dict(block_tables=None), 1),
+    (dict(context_lens=None), 1), (dict(num_seqs=-1), 1), (dict(hq=6, hkv=4), 1),
+    (dict(hq=12, hkv=4), 2), (dict(hq=32, hkv=2), 2), (dict(d=96), 2), (dict(d=512), 2),
+    (dict(bs=24), 2), (dict(bs=64), 2), (dict(bs=2), 2), (dict(dtype=7), 2),
+    (dict(max_ctx=17), 1), (dict(nb=0), 1), (dict(max_blocks=0), 1),
+    (dict(out=M), 1), (dict(k_pool=M), 1), (dict(nb=1 << 40), 1),
+])
+def test_decode_attention_host_validation(pa, kw, want):
+    assert _attn(pa, **kw) == want
+
+
+def test_zero_sequences_is_a_no_op(pa):
+    assert _attn(pa, num_seqs=0, out=None, query=None) == 0
+
+
+def test_splitk_host_validation(pa):
+    L = pa.lib
+
+    def call(P=16, maxp=1, tmp=A, ml=A, es=A, max_ctx=16):
+        return L.pa_decode_splitk(A, A, A, A, A, 4, A, 3, max_ctx, 8, 2, 64, 4, 16, 0.125, 0,
+                                  P, maxp, tmp, ml, es, None, None)
+    assert call(P=24) == 1                      # not a multiple of 16
+    assert call(P=0) == 1
+    assert call(P=16, maxp=0) == 1
+    assert call(P=16, maxp=1, max_ctx=16) != 4  # enough partitions (fails later only on CUDA)
+    assert call(P=8 * 2, maxp=1, max_ctx=16) != 4
+    assert L.pa_decode_splitk(A, A, A, A, A, 8, A, 3, 32, 8, 2, 64, 4, 16, 0.125, 0,
+                              16, 1, A, A, A, None, None) == 4      # 32 tokens need 2 parts
+    assert call(tmp=None) == 1
+    assert L.pa_splitk_reduce(A, A, A, A, A, 3, 8, 64, 24, 2, 0, None) == 1
+    assert L.pa_splitk_reduce(A, A, A, A, A, 3, 8, 96, 16, 2, 0, None) == 2
+    assert L.pa_splitk_reduce(None, A, A, A, A, 3, 8, 64, 16, 2, 0, None) == 1
+
+
+def test_reshape_and_cache_host_validation(pa):
+    L = pa.lib
+
+    def call(**kw):
+        a = dict(key=A, value=A, kp=A, vp=A, slots=A, T=3, hkv=2, d=64, bs=4, nb=16, dt=0)
+        a.update(kw)
+        return L.pa_reshape_and_cache(a["key"], a["value"], a["kp"], a["vp"], a["slots"],
+                                      a["T"], a["hkv"], a["d"], a["bs"], a["nb"], a["dt"],
+                                      None, None)
+    assert call(key=None) == 1
+    assert call(slots=None) == 1
+    assert call(T=-1) == 1
+    assert call(bs=12) == 2
+    assert call(d=100) == 2
+    assert call(dt=5) == 2
+    assert call(value=M) == 1
+    assert call(T=0, key=None) == 0
+
+
+def test_binding_rejects_cpu_tensors(pa):
+    import torch
+    x = torch.zeros(3, 8, 64)
+    with pytest.raises(ValueError):
+        pa.pa_decode_attention(x, x, torch.zeros(16, 4, 2, 64), torch.zeros(16, 4, 2, 64),
+                               torch.zeros(3, 2, dtype=torch.int32),
+                               torch.zeros(3, dtype=torch.int32), 8, 0.125)
