@@ -158,7 +158,7 @@ class Workload:
         self.layers = W.make_layers(self.layout, device)
         self.tables, self.lens, self.slots = W.device_metadata(self.layout, device)
         L = self.layout
-        nbytes = pa.pa_decode_workspace_bytes(cfg.num_seqs, cfg.num_q_heads, cfg.head_dim,
+        nbytes = pa.pa_decode_workspace_bytes(cfg.num_seqs, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
                                               L.max_context_len)
         self.workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
         self.outs = [torch.empty_like(l.query) for l in self.layers]

@@ -95,9 +95,9 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_pool,
  *   p_t = exp(s_t - max_t s_t),  s_t = scale * q[b, hq, :] . K[t, hq / G, :],
  * over the tokens t < context_lens[b] of sequence b, gathered through its
  * block table (the definition above is exact softmax attention; the library
- * computes it with an online softmax in fp32 and, for long contexts, a
- * flash-decoding split of the context into partitions merged by the
- * log-sum-exp rule).
+ * computes it with an online softmax in fp32 over 16-token tiles and, where a
+ * sequence's tiles are spread over several warps, merges the pieces by the
+ * log-sum-exp rule, as in flash-decoding).
  *
  *   out            device, [B, Hq, d], written.
  *   query          device, [B, Hq, d].
@@ -106,15 +106,18 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_pool,
  *                  ceil(context_lens[b] / bs) are never read.
  *   context_lens   device, [B] int32.
  *   max_context_len host hint, >= every context_lens[b]; used to size the
- *                  split.  Must be <= max_blocks_per_seq * bs.
+ *                  grid.  Must be <= max_blocks_per_seq * bs.
  *   scale          softmax scale (usually 1 / sqrt(d)).
  *   workspace      device scratch of workspace_bytes bytes (may be NULL / 0).
- *                  pa_decode_workspace_bytes() gives the size the library
- *                  wants for its preferred split; with less (or none) it uses
- *                  fewer, longer partitions, down to no split at all, so any
- *                  size is correct.  Contents need no initialisation and are
- *                  garbage afterwards.  Calls that share a workspace must not
- *                  run concurrently.
+ *                  With at least pa_decode_workspace_bytes() bytes the work is
+ *                  split evenly over the GPU's warps (each warp owns an equal
+ *                  share of the batch's 16-token tiles, whatever the lengths)
+ *                  and the pieces of a sequence that straddles warps are
+ *                  merged by a second kernel; with less, every (sequence, KV
+ *                  head) is processed by one warp.  Both are exact to the
+ *                  same tolerance.  Contents need no initialisation and are
+ *                  garbage afterwards; calls sharing a workspace must not run
+ *                  concurrently.
  *   dev_status     device int32 or NULL (see PA_DEV_*).
  */
 pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
@@ -125,9 +128,10 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
                               pa_dtype dtype, void *workspace, size_t workspace_bytes,
                               int32_t *dev_status, void *stream);
 
-/* Workspace bytes pa_decode_attention wants for these sizes (0 = it will not
- * split).  Host only; touches no device. */
-size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
+/* Workspace bytes pa_decode_attention wants for these sizes (enough for GPUs
+ * of up to 256 SMs; about 8.5 MB for Hq/Hkv = 4, d = 256).  Host only;
+ * touches no device.  max_context_len is accepted for symmetry and unused. */
+size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int max_context_len);
 
 /* ceil(max_context_len / partition_size), at least 1. Host only. */

@@ -17,16 +17,16 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpa.so")
-SOURCES = [os.path.join(CSRC, "pa.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in
+           ("pa.cu", "pa_inst_f32.cu", "pa_inst_bf16.cu", "pa_inst_bf16_simt.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + \
     [os.path.join(INCLUDE, "pa.h")]
+OBJ_DIR = os.path.join(PKG, "_build")
 
-NVCC_FLAGS = [
-    "-gencode", "arch=compute_100a,code=sm_100a",
-    "-lineinfo", "-O3", "-std=c++17",
-    "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",
-    "--expt-relaxed-constexpr",
-]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+COMPILE_FLAGS = ARCH + ["-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC",
+                        "--expt-relaxed-constexpr"]
+LINK_FLAGS = ARCH + ["-shared", "-cudart", "static"]
 
 
 def nvcc() -> str:
@@ -43,17 +43,30 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-o", tmp, *SOURCES]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+def build(force: bool = False, verbose: bool = False, extra=(), out: str = LIB) -> str:
+    """Compiles every translation unit in parallel, then links libpa.so."""
+    if not force and out == LIB and up_to_date():
+        return out
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    tag = "%d" % os.getpid()
+    objs, procs = [], []
+    for src in SOURCES:
+        obj = os.path.join(OBJ_DIR, os.path.basename(src) + "." + tag + ".o")
+        cmd = [nvcc(), *COMPILE_FLAGS, *extra, "-I", INCLUDE, "-c", "-o", obj, src]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+            print(" ".join(cmd), file=sys.stderr)
+        procs.append(subprocess.Popen(cmd))
+        objs.append(obj)
+    failed = [p.args[-1] for p in procs if p.wait() != 0]
+    if failed:
+        raise RuntimeError("nvcc failed on " + ", ".join(failed))
+    tmp = out + ".tmp" + tag
+    subprocess.check_call([nvcc(), *LINK_FLAGS, "-o", tmp, *objs])
+    os.replace(tmp, out)
+    for o in objs:
+        os.remove(o)
+    return out
 
 
 def main(argv=None) -> None:

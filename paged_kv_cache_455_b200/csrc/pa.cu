@@ -1,31 +1,35 @@
 // pa.cu -- C ABI of the paged KV-cache decode library: argument checks,
-// launch geometry and kernel dispatch.  Kernels live in pa_kernels.cuh.
+// shared-memory geometry, TMA tensor maps, work-decomposition choice and
+// launches.  Device code lives in pa_kernels.cuh; the decode / merge kernels
+// are instantiated in pa_inst_*.cu.
 //
-// Split choice of pa_decode_attention: partitions of kPrefPartition tokens
-// when a sequence can be longer than that and the caller's workspace holds
-// the partials; with a smaller workspace the partitions grow until the
-// partials fit, down to one partition per sequence (no split).
+// pa_decode_attention uses the stream-K decomposition (mode 0) when the
+// caller's workspace holds the per-warp partials, and whole segments per warp
+// (mode 1) otherwise.  pa_decode_splitk runs mode 1 over fixed partitions.
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
-#include <type_traits>
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "pa.h"
-#include "pa_kernels.cuh"
+#include "pa_launch.cuh"
 
 namespace {
 
+using pa::DecodeLaunch;
 using pa::DecodeParams;
+using pa::TileGeo;
 
 std::atomic<unsigned long long> g_launches{0};
 
-constexpr int kPrefPartition = 256;   // tokens per split-K partition (multiple of 16)
+// Bound on decode warps used to size the stream-K workspace (256 SMs x 4).
+constexpr int kWorkspaceWarps = 1024;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -37,93 +41,186 @@ int ilog2_exact(int v)
     return (1 << s) == v ? s : -1;
 }
 
-int round_up(int v, int m) { return ((v + m - 1) / m) * m; }
+int64_t round_up(int64_t v, int64_t m) { return ((v + m - 1) / m) * m; }
 
-// ---------------------------------------------------------------------------
-// Per-device launch facts, computed once per (device, kernel).
-// ---------------------------------------------------------------------------
-struct KernelSlot {
-    const void *fn;
-    int device;
-    int grid;   // persistent grid: SMs * resident CTAs
+int elem_size(pa_dtype dt) { return dt == PA_DTYPE_F32 ? 4 : 2; }
+
+// =====================================================================
+// Cache write kernel: one warp per (token, KV head, K|V) row, 16-byte copies.
+// =====================================================================
+struct CacheParams {
+    const void *key;
+    const void *value;
+    void *k_pool;
+    void *v_pool;
+    const int64_t *slot_mapping;
+    int32_t *dev_status;
+    int64_t num_slots;      // nb * bs
+    int num_tokens;
+    int num_kv_heads;
+    int row_bytes;          // d * element size
 };
 
-std::mutex g_mu;
-KernelSlot g_slots[256];
-int g_nslots = 0;
-
-pa_status persistent_grid(const void *fn, int smem_bytes, int *grid_out)
+__global__ void __launch_bounds__(256) cache_write_kernel(const CacheParams p)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess)
-        return PA_ERR_CUDA;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t nrows = (int64_t)p.num_tokens * p.num_kv_heads * 2;
+    if (row >= nrows)
+        return;
+    const int kv = (int)(row & 1);
+    const int64_t th = row >> 1;
+    const int64_t t = th / p.num_kv_heads;
+    const int64_t h = th - t * p.num_kv_heads;
+    const int64_t slot = p.slot_mapping[t];
+    if (slot < 0)
+        return;
+    if (slot >= p.num_slots) {
+        if (lane == 0 && h == 0 && kv == 0)
+            pa::report(p.dev_status, PA_DEV_BAD_SLOT);
+        return;
+    }
+    const int4 *src = reinterpret_cast<const int4 *>(
+        static_cast<const uint8_t *>(kv ? p.value : p.key) + (t * p.num_kv_heads + h) * p.row_bytes);
+    int4 *dst = reinterpret_cast<int4 *>(static_cast<uint8_t *>(kv ? p.v_pool : p.k_pool) +
+                                         (slot * p.num_kv_heads + h) * p.row_bytes);
+    const int n16 = p.row_bytes >> 4;
+    for (int c = lane; c < n16; c += 32)
+        dst[c] = __ldg(src + c);
+}
+
+// =====================================================================
+// Tensor maps
+// =====================================================================
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 4-D maps (one TMA operation per box) unless the driver has refused one;
+// then 3-D maps with one operation per 128-byte column.
+std::atomic<int> g_four_d{1};
+
+struct MapKey {
+    const void *base;
+    int64_t rows;
+    int hkv, d, es, tr, four_d;
+    bool operator==(const MapKey &o) const
     {
-        std::lock_guard<std::mutex> lock(g_mu);
-        for (int i = 0; i < g_nslots; ++i)
-            if (g_slots[i].fn == fn && g_slots[i].device == dev) {
-                *grid_out = g_slots[i].grid;
-                return PA_OK;
+        return base == o.base && rows == o.rows && hkv == o.hkv && d == o.d && es == o.es &&
+               tr == o.tr && four_d == o.four_d;
+    }
+};
+
+struct MapEntry {
+    MapKey key;
+    alignas(64) CUtensorMap map;
+};
+
+std::mutex g_map_mu;
+MapEntry g_maps[128];
+int g_nmaps = 0, g_next_map = 0;
+
+// Tensor map over a pool [nb, bs, Hkv, d] whose box is `tr` token rows x d of
+// one head, 128-byte swizzled.  4-D: dims (128-byte column elements, token
+// row, column, head); 3-D: dims (d, head, token row).
+bool encode_pool_map(CUtensorMap *out, const void *base, int64_t nb, int bs, int hkv, int d,
+                     pa_dtype dt, int tr, int four_d)
+{
+    const int es = elem_size(dt);
+    const MapKey key{base, nb * bs, hkv, d, es, tr, four_d};
+    {
+        std::lock_guard<std::mutex> lock(g_map_mu);
+        for (int i = 0; i < g_nmaps; ++i)
+            if (g_maps[i].key == key) {
+                *out = g_maps[i].map;
+                return true;
             }
     }
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
-        cudaSuccess)
-        return PA_ERR_CUDA;
-    int sms = 0, per_sm = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return PA_ERR_CUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, pa::kThreads, smem_bytes) !=
-        cudaSuccess)
-        return PA_ERR_CUDA;
-    if (per_sm < 1)
-        return PA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (g_nslots < 256)
-        g_slots[g_nslots++] = KernelSlot{fn, dev, sms * per_sm};
-    *grid_out = sms * per_sm;
-    return PA_OK;
-}
-
-// ---------------------------------------------------------------------------
-// Decode dispatch over (dtype, head_dim, group, math)
-// ---------------------------------------------------------------------------
-template <typename T, int D, int G, bool MMA>
-pa_status launch_decode_t(const DecodeParams &p, int64_t items_upper, cudaStream_t stream)
-{
-    const void *fn = reinterpret_cast<const void *>(&pa::decode_kernel<T, D, G, MMA>);
-    constexpr int smem = pa::Layout<T, D, G>::kSmem;
-    int grid = 0;
-    pa_status st = persistent_grid(fn, smem, &grid);
-    if (st != PA_OK)
-        return st;
-    if (items_upper < grid)
-        grid = (int)(items_upper > 0 ? items_upper : 1);
-    pa::decode_kernel<T, D, G, MMA><<<grid, pa::kThreads, smem, stream>>>(p);
-    ++g_launches;
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
-}
-
-template <typename T, int D, bool MMA>
-pa_status launch_decode_g(const DecodeParams &p, int group, int64_t items, cudaStream_t s)
-{
-    switch (group) {
-    case 1: return launch_decode_t<T, D, 1, MMA>(p, items, s);
-    case 2: return launch_decode_t<T, D, 2, MMA>(p, items, s);
-    case 4: return launch_decode_t<T, D, 4, MMA>(p, items, s);
-    case 8: return launch_decode_t<T, D, 8, MMA>(p, items, s);
-    default: return PA_ERR_UNSUPPORTED;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    const CUtensorMapDataType type =
+        dt == PA_DTYPE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint32_t epc = 128 / es;           // elements per 128-byte column
+    const cuuint64_t rowb = (cuuint64_t)d * es;
+    const cuuint32_t nch = (cuuint32_t)(rowb / 128);
+    alignas(64) CUtensorMap map;
+    CUresult r;
+    if (four_d) {
+        const cuuint64_t dims[4] = {epc, (cuuint64_t)(nb * bs), nch, (cuuint64_t)hkv};
+        const cuuint64_t strides[3] = {(cuuint64_t)hkv * rowb, 128, rowb};
+        const cuuint32_t box[4] = {epc, (cuuint32_t)tr, nch, 1};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        r = enc(&map, type, 4, const_cast<void *>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)(nb * bs)};
+        const cuuint64_t strides[2] = {rowb, (cuuint64_t)hkv * rowb};
+        const cuuint32_t box[3] = {epc, 1, (cuuint32_t)tr};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        r = enc(&map, type, 3, const_cast<void *>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     }
+    if (r != CUDA_SUCCESS)
+        return false;
+    *out = map;
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    const int slot = g_nmaps < 128 ? g_nmaps++ : (g_next_map++ % 128);
+    g_maps[slot].key = key;
+    g_maps[slot].map = map;
+    return true;
 }
 
-template <typename T, bool MMA>
-pa_status launch_decode_d(const DecodeParams &p, int head_dim, int group, int64_t items,
-                          cudaStream_t s)
+// =====================================================================
+// Geometry and launch plumbing
+// =====================================================================
+bool make_geo(TileGeo &g, int D, int es, int bs, int group, int four_d, int *smem)
 {
-    switch (head_dim) {
-    case 64: return launch_decode_g<T, 64, MMA>(p, group, items, s);
-    case 128: return launch_decode_g<T, 128, MMA>(p, group, items, s);
-    case 256: return launch_decode_g<T, 256, MMA>(p, group, items, s);
-    default: return PA_ERR_UNSUPPORTED;
+    const int rowb = D * es;
+    const int nch = rowb / 128;
+    g.tr = std::min(16, bs);
+    g.tr_log2 = ilog2_exact(g.tr);
+    g.bpt = 16 / g.tr;
+    if (four_d) {
+        g.ops_per_box = 1;
+        g.chunk_stride = g.tr * 128;
+        g.box_stride = (int)round_up((int64_t)nch * g.chunk_stride, 1024);
+    } else {
+        g.ops_per_box = nch;
+        g.chunk_stride = (int)round_up((int64_t)g.tr * 128, 1024);
+        g.box_stride = nch * g.chunk_stride;
     }
+    g.kv_bytes = g.bpt * g.box_stride;
+    g.q_bytes = group * D * es;
+    g.q_off = 2 * g.kv_bytes;
+    g.stage_bytes = (int)round_up((int64_t)g.q_off + g.q_bytes, 1024);
+    g.box_tx = g.tr * rowb;
+    const int fixed = pa::decode_smem_fixed(group);
+    const int spw =
+        std::min(pa::kMaxSpw, (pa::kSmemBudget - fixed) / (pa::kWarps * g.stage_bytes));
+    if (spw < 1)
+        return false;
+    g.spw = spw;
+    *smem = fixed + pa::kWarps * spw * g.stage_bytes;
+    return true;
 }
 
 // bf16 uses the tensor-core tile math unless PA_DECODE_MATH=simt is set
@@ -134,25 +231,21 @@ bool bf16_use_mma()
     return !(v && std::strcmp(v, "simt") == 0);
 }
 
-pa_status launch_decode(const DecodeParams &p, pa_dtype dtype, int head_dim, int group,
-                        int64_t items, cudaStream_t s)
+pa_status decode_call(DecodeLaunch &L, pa_dtype dtype, int *grid, bool launch)
 {
     if (dtype == PA_DTYPE_F32)
-        return launch_decode_d<float, false>(p, head_dim, group, items, s);
+        return pa::decode_f32(L, grid, launch);
     if (bf16_use_mma())
-        return launch_decode_d<__nv_bfloat16, true>(p, head_dim, group, items, s);
-    return launch_decode_d<__nv_bfloat16, false>(p, head_dim, group, items, s);
+        return pa::decode_bf16_mma(L, grid, launch);
+    return pa::decode_bf16_simt(L, grid, launch);
 }
 
-// ---------------------------------------------------------------------------
-// Shared argument checks of the attention calls
-// ---------------------------------------------------------------------------
 pa_status check_attention_args(const void *out, const void *query, const void *k_pool,
-                               const void *v_pool, const int32_t *block_tables,
-                               int max_blocks, const int32_t *context_lens, int num_seqs,
-                               int max_context_len, int num_q_heads, int num_kv_heads,
-                               int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
-                               int *group_out, int *bs_log2_out)
+                               const void *v_pool, const int32_t *block_tables, int max_blocks,
+                               const int32_t *context_lens, int num_seqs, int max_context_len,
+                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                               int64_t num_blocks, pa_dtype dtype, int *group_out,
+                               int *bs_log2_out)
 {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
         max_blocks <= 0 || max_context_len < 0)
@@ -171,8 +264,12 @@ pa_status check_attention_args(const void *out, const void *query, const void *k
         return PA_ERR_UNSUPPORTED;
     if ((int64_t)max_context_len > (int64_t)max_blocks * block_size)
         return PA_ERR_INVALID_ARG;
-    if (num_blocks > (int64_t)INT32_MAX)
-        return PA_ERR_INVALID_ARG;   // block ids are int32
+    if (num_blocks > (int64_t)INT32_MAX / block_size)
+        return PA_ERR_INVALID_ARG;   // token rows of the pool are int32 TMA coordinates
+    // every tile index of the batch must fit an int
+    if ((int64_t)num_seqs * num_kv_heads * (round_up((int64_t)max_blocks * block_size, 16) / 16) >
+        (int64_t)INT32_MAX / 2)
+        return PA_ERR_INVALID_ARG;
     if (num_seqs > 0) {
         if (!out || !query || !k_pool || !v_pool || !block_tables || !context_lens)
             return PA_ERR_INVALID_ARG;
@@ -184,24 +281,20 @@ pa_status check_attention_args(const void *out, const void *query, const void *k
     return PA_OK;
 }
 
-DecodeParams make_params(void *out, const void *query, const void *k_pool, const void *v_pool,
-                         const int32_t *block_tables, int max_blocks,
+// Fills everything of a decode launch but the work decomposition.
+pa_status prepare_decode(DecodeLaunch &L, void *out, const void *query, const void *k_pool,
+                         const void *v_pool, const int32_t *block_tables, int max_blocks,
                          const int32_t *context_lens, int num_seqs, int num_q_heads,
-                         int num_kv_heads, int block_size, int bs_log2, int64_t num_blocks,
-                         float scale, int partition_size, int max_parts, float *tmp_out,
-                         float *max_logits, float *exp_sums, int always_partials,
-                         int32_t *dev_status)
+                         int num_kv_heads, int head_dim, int block_size, int bs_log2,
+                         int64_t num_blocks, float scale, pa_dtype dtype, int group,
+                         int32_t *dev_status, void *stream)
 {
-    DecodeParams p;
+    std::memset(&L.p, 0, sizeof(L.p));
+    DecodeParams &p = L.p;
     p.out = out;
     p.q = query;
-    p.k_pool = k_pool;
-    p.v_pool = v_pool;
     p.block_tables = block_tables;
     p.context_lens = context_lens;
-    p.tmp_out = tmp_out;
-    p.max_logits = max_logits;
-    p.exp_sums = exp_sums;
     p.dev_status = dev_status;
     p.num_blocks = num_blocks;
     p.num_seqs = num_seqs;
@@ -210,26 +303,34 @@ DecodeParams make_params(void *out, const void *query, const void *k_pool, const
     p.max_blocks = max_blocks;
     p.block_size = block_size;
     p.bs_log2 = bs_log2;
-    p.partition_size = partition_size;
-    p.max_parts = max_parts;
-    const int64_t cap = std::min<int64_t>((int64_t)max_blocks * block_size,
-                                          (int64_t)max_parts * partition_size);
-    p.ctx_cap = (int)std::min<int64_t>(cap, INT32_MAX);
-    p.always_partials = always_partials;
     p.scale_log2 = scale * pa::kLog2e;
-    return p;
+    L.head_dim = head_dim;
+    L.group = group;
+    L.tr16 = block_size >= 16;
+    L.stream = static_cast<cudaStream_t>(stream);
+    const int es = elem_size(dtype);
+    const int tr = std::min(16, block_size);
+    for (;;) {
+        const int four_d = g_four_d.load();
+        if (!make_geo(p.geo, head_dim, es, block_size, group, four_d, &L.smem_bytes))
+            return PA_ERR_UNSUPPORTED;
+        const bool ok_k = encode_pool_map(&L.tmap_k, k_pool, num_blocks, block_size, num_kv_heads,
+                                          head_dim, dtype, tr, four_d);
+        const bool ok_v = ok_k && encode_pool_map(&L.tmap_v, v_pool, num_blocks, block_size,
+                                                  num_kv_heads, head_dim, dtype, tr, four_d);
+        if (ok_k && ok_v)
+            return PA_OK;
+        if (!four_d)
+            return PA_ERR_CUDA;
+        g_four_d.store(0);   // retry with 3-D maps
+    }
 }
 
-template <typename T>
-pa_status launch_reduce_t(const pa::ReduceParams &rp, int head_dim, int num_seqs,
-                          cudaStream_t stream)
+size_t stream_k_bytes(int64_t num_seqs, int64_t num_kv_heads, int64_t group, int64_t head_dim,
+                      int64_t warps)
 {
-    const int64_t grid = (int64_t)num_seqs * rp.num_q_heads;
-    if (grid > INT32_MAX)
-        return PA_ERR_INVALID_ARG;
-    pa::reduce_kernel<T><<<(unsigned)grid, 128, 0, stream>>>(rp, head_dim);
-    ++g_launches;
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const int64_t slot = round_up(group * head_dim + 2 * group + 1, 4);
+    return (size_t)(2 * warps * slot * 4 + round_up(num_seqs * num_kv_heads * 4, 16) + 16);
 }
 
 pa_status launch_reduce(void *out, const float *tmp_out, const float *max_logits,
@@ -248,9 +349,15 @@ pa_status launch_reduce(void *out, const float *tmp_out, const float *max_logits
     rp.partition_size = partition_size;
     rp.max_parts = max_parts;
     rp.ctx_cap = ctx_cap;
+    const int64_t grid = (int64_t)num_seqs * num_q_heads;
+    if (grid > INT32_MAX)
+        return PA_ERR_INVALID_ARG;
     if (dtype == PA_DTYPE_F32)
-        return launch_reduce_t<float>(rp, head_dim, num_seqs, stream);
-    return launch_reduce_t<__nv_bfloat16>(rp, head_dim, num_seqs, stream);
+        pa::reduce_kernel<float><<<(unsigned)grid, 128, 0, stream>>>(rp, head_dim);
+    else
+        pa::reduce_kernel<__nv_bfloat16><<<(unsigned)grid, 128, 0, stream>>>(rp, head_dim);
+    ++g_launches;
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 size_t splitk_bytes(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t parts)
@@ -290,13 +397,15 @@ size_t pa_splitk_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, in
     return splitk_bytes(num_seqs, num_q_heads, head_dim, max_partitions);
 }
 
-size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
+size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int max_context_len)
 {
-    if (max_context_len <= kPrefPartition)
+    (void)max_context_len;
+    if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        num_q_heads % num_kv_heads != 0)
         return 0;
-    return pa_splitk_workspace_bytes(num_seqs, num_q_heads, head_dim,
-                                     pa_num_partitions(max_context_len, kPrefPartition));
+    return stream_k_bytes(num_seqs, num_kv_heads, num_q_heads / num_kv_heads, head_dim,
+                          kWorkspaceWarps);
 }
 
 pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_pool, void *v_pool,
@@ -318,7 +427,7 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_pool,
         return PA_ERR_INVALID_ARG;
     if (!aligned16(key) || !aligned16(value) || !aligned16(k_pool) || !aligned16(v_pool))
         return PA_ERR_INVALID_ARG;
-    pa::CacheParams p;
+    CacheParams p;
     p.key = key;
     p.value = value;
     p.k_pool = k_pool;
@@ -328,12 +437,12 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_pool,
     p.num_slots = num_blocks * block_size;
     p.num_tokens = num_tokens;
     p.num_kv_heads = num_kv_heads;
-    p.row_bytes = head_dim * (dtype == PA_DTYPE_F32 ? 4 : 2);
+    p.row_bytes = head_dim * elem_size(dtype);
     const int64_t rows = (int64_t)num_tokens * num_kv_heads * 2;
     const int64_t blocks = (rows + 7) / 8;   // 8 warps per CTA
     if (blocks > INT32_MAX)
         return PA_ERR_INVALID_ARG;
-    pa::cache_write_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    cache_write_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     ++g_launches;
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -361,14 +470,32 @@ pa_status pa_decode_splitk(void *out, const void *query, const void *k_pool, con
         return PA_OK;
     if (!tmp_out || !max_logits || !exp_sums)
         return PA_ERR_INVALID_ARG;
-    const int64_t items = (int64_t)num_seqs * num_kv_heads * max_partitions;
-    if (items > INT32_MAX)
-        return PA_ERR_INVALID_ARG;
-    DecodeParams p = make_params(out, query, k_pool, v_pool, block_tables, max_blocks_per_seq,
-                                 context_lens, num_seqs, num_q_heads, num_kv_heads, block_size,
-                                 bs_log2, num_blocks, scale, partition_size, max_partitions,
-                                 tmp_out, max_logits, exp_sums, 1, dev_status);
-    return launch_decode(p, dtype, head_dim, group, items, static_cast<cudaStream_t>(stream));
+    DecodeLaunch L;
+    st = prepare_decode(L, out, query, k_pool, v_pool, block_tables, max_blocks_per_seq,
+                        context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                        bs_log2, num_blocks, scale, dtype, group, dev_status, stream);
+    if (st != PA_OK)
+        return st;
+    DecodeParams &p = L.p;
+    p.tmp_out = tmp_out;
+    p.max_logits = max_logits;
+    p.exp_sums = exp_sums;
+    p.partition_size = partition_size;
+    p.max_parts = max_partitions;
+    p.ctx_cap = (int)std::min<int64_t>((int64_t)max_blocks_per_seq * block_size,
+                                       (int64_t)max_partitions * partition_size);
+    p.mode = 1;
+    p.public_partials = 1;
+    int grid = 0;
+    st = decode_call(L, dtype, &grid, false);
+    if (st != PA_OK)
+        return st;
+    const int64_t tiles_up =
+        (int64_t)num_seqs * num_kv_heads * (round_up(std::max(max_context_len, 1), 16) / 16);
+    grid = (int)std::min<int64_t>(grid, (tiles_up + pa::kWarps - 1) / pa::kWarps);
+    st = decode_call(L, dtype, &grid, true);
+    ++g_launches;
+    return st;
 }
 
 pa_status pa_splitk_reduce(void *out, const float *tmp_out, const float *max_logits,
@@ -411,43 +538,61 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
         return st;
     if (num_seqs == 0)
         return PA_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-
-    // Partition size: kPrefPartition if the partials fit the workspace, else
-    // the smallest multiple of 16 whose partials fit, else no split.
-    const int full = round_up(max_context_len > 0 ? max_context_len : 1, pa::kTile);
-    int P = full;
-    int parts = 1;
-    if (max_context_len > kPrefPartition && workspace != nullptr) {
-        const size_t per_part = splitk_bytes(num_seqs, num_q_heads, head_dim, 1);
-        const int64_t fit = (int64_t)(workspace_bytes / per_part);
-        const int want = pa_num_partitions(max_context_len, kPrefPartition);
-        const int64_t use = std::min<int64_t>(fit, want);
-        if (use >= 2) {
-            P = round_up(pa_num_partitions(max_context_len, (int)use), pa::kTile);
-            P = std::max(P, kPrefPartition);
-            parts = pa_num_partitions(max_context_len, P);
-        }
-    }
-    const int64_t items = (int64_t)num_seqs * num_kv_heads * parts;
-    if (items > INT32_MAX)
-        return PA_ERR_INVALID_ARG;
-    float *tmp = nullptr, *ml = nullptr, *es = nullptr;
-    if (parts > 1) {
-        if (!aligned16(workspace))
-            return PA_ERR_INVALID_ARG;
-        tmp = static_cast<float *>(workspace);
-        ml = tmp + (int64_t)num_seqs * num_q_heads * parts * head_dim;
-        es = ml + (int64_t)num_seqs * num_q_heads * parts;
-    }
-    DecodeParams p = make_params(out, query, k_pool, v_pool, block_tables, max_blocks_per_seq,
-                                 context_lens, num_seqs, num_q_heads, num_kv_heads, block_size,
-                                 bs_log2, num_blocks, scale, P, parts, tmp, ml, es, 0, dev_status);
-    st = launch_decode(p, dtype, head_dim, group, items, s);
-    if (st != PA_OK || parts == 1)
+    DecodeLaunch L;
+    st = prepare_decode(L, out, query, k_pool, v_pool, block_tables, max_blocks_per_seq,
+                        context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                        bs_log2, num_blocks, scale, dtype, group, dev_status, stream);
+    if (st != PA_OK)
         return st;
-    return launch_reduce(out, tmp, ml, es, context_lens, num_seqs, num_q_heads, head_dim, P,
-                         parts, p.ctx_cap, dtype, s);
+    DecodeParams &p = L.p;
+    const int64_t cap_tokens = (int64_t)max_blocks_per_seq * block_size;
+    p.partition_size = (int)round_up(cap_tokens, 16);   // one partition: the whole context
+    p.max_parts = 1;
+    p.ctx_cap = (int)cap_tokens;
+
+    int grid = 0;
+    st = decode_call(L, dtype, &grid, false);
+    if (st != PA_OK)
+        return st;
+    const int64_t tiles_up =
+        (int64_t)num_seqs * num_kv_heads * (round_up(std::max(max_context_len, 1), 16) / 16);
+    grid = (int)std::min<int64_t>(grid, (tiles_up + pa::kWarps - 1) / pa::kWarps);
+    const int64_t warps = (int64_t)grid * pa::kWarps;
+    const size_t need = stream_k_bytes(num_seqs, num_kv_heads, group, head_dim, warps);
+    const bool stream_k = workspace != nullptr && workspace_bytes >= need && aligned16(workspace);
+    pa::MergeParams mp;
+    std::memset(&mp, 0, sizeof(mp));
+    if (stream_k) {
+        p.mode = 0;
+        p.slot_floats = (int)round_up((int64_t)group * head_dim + 2 * group + 1, 4);
+        p.wpart = static_cast<float *>(workspace);
+        p.seg_start = reinterpret_cast<int32_t *>(p.wpart + 2 * warps * p.slot_floats);
+        p.total_tiles = p.seg_start + round_up((int64_t)num_seqs * num_kv_heads, 4);
+        mp.out = out;
+        mp.wpart = p.wpart;
+        mp.seg_start = p.seg_start;
+        mp.total_tiles = p.total_tiles;
+        mp.context_lens = context_lens;
+        mp.num_seqs = num_seqs;
+        mp.num_q_heads = num_q_heads;
+        mp.num_kv_heads = num_kv_heads;
+        mp.ctx_cap = p.ctx_cap;
+        mp.total_warps = (int)warps;
+        mp.slot_floats = p.slot_floats;
+    } else {
+        p.mode = 1;
+    }
+    const int want = grid;
+    st = decode_call(L, dtype, &grid, true);
+    ++g_launches;
+    if (st != PA_OK || !stream_k)
+        return st;
+    if (grid != want)
+        return PA_ERR_CUDA;   // capacity changed between query and launch
+    st = dtype == PA_DTYPE_F32 ? pa::merge_f32(mp, head_dim, group, L.stream)
+                               : pa::merge_bf16(mp, head_dim, group, L.stream);
+    ++g_launches;
+    return st;
 }
 
 }  // extern "C"

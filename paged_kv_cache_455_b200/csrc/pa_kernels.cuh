@@ -1,28 +1,40 @@
-// pa_kernels.cuh -- sm_100a kernels of the paged KV-cache decode library.
+// pa_kernels.cuh -- sm_100a device code of the paged KV-cache decode library.
 //
-// Kernels
-//   cache_write_kernel   new token's K/V rows -> their pool slots (bit copy).
-//   decode_kernel        persistent split-K paged attention: every (sequence,
-//                        KV head, context partition) is one work item; each
-//                        CTA walks items with a grid stride.  Per warp, K/V
-//                        tiles of 16 tokens stream into shared memory through
-//                        bulk copies (one per 16-token row slice, addressed
-//                        through the block table) completed on mbarriers,
-//                        SPW tiles in flight.  All query heads of the GQA
-//                        group are served from one read of each K/V tile.
-//   reduce_kernel        log-sum-exp merge of the partitions of a sequence.
+// decode_kernel (persistent; warps never wait for one another)
+//   Work is cut into tiles: 16 consecutive tokens of one (sequence, KV head),
+//   inside one context partition (the whole context unless the caller asks
+//   for fixed-size partitions).  All tiles of the batch form one global
+//   sequence ordered by sequence, partition, KV head, token.  A "segment" is
+//   the run of tiles of one (sequence, partition, KV head).  Every warp of the
+//   grid owns one contiguous range of that sequence:
+//     mode 0 (stream-K): equal ranges.  A segment cut by range boundaries
+//       leaves one partial softmax state per piece (at most two per warp),
+//       merged afterwards by merge_kernel.  Balanced for any mix of lengths.
+//     mode 1: ranges snapped to segment starts, so one warp finishes every
+//       segment it starts (no partials; used without a workspace and for the
+//       explicit fixed-partition split-K API).
+//   Per warp, tiles stream into shared memory through TMA: one tensor-map box
+//   brings `tr` rows x d of K (or V) of one KV head, 128-byte swizzled,
+//   completing on the stage's mbarrier.  A warp keeps up to SPW tiles in
+//   flight and issues tile i + SPW once it has consumed tile i.  Block-table
+//   entries of the next 32 tiles are fetched in one lane-parallel batch ahead
+//   of use.  The query rows of a segment arrive with its first tile.
 //
-// The math of a tile is one of two policies:
-//   SimtMath  fp32 FMAs, one token row spread over a warp (or part of one),
-//             warp-shuffle dot products; used for fp32 data (and, on request,
-//             for bf16).
-//   MmaMath   bf16 tensor-core MMAs (m16n8k16, fp32 accumulate): S = K Q^T
-//             with the group's heads as the N = 8 columns, then
-//             O^T += V^T P^T with P transposed in registers by movmatrix.
-// Both keep an online softmax in fp32 in the log2 domain.
+// Tile math (one policy per instantiation)
+//   MmaMath   bf16 tensor cores (mma.sync m16n8k16, fp32 accumulate):
+//             S = K Q^T with the G query heads of the group as the N = 8
+//             columns, then O^T += V^T P^T with P transposed in registers.
+//   SimtMath  fp32 FMAs with warp-shuffle dot products (fp32 data; also
+//             available for bf16, for comparison).
+//   Both keep the online softmax (running max and sum) in fp32, in the log2
+//   domain (logits pre-multiplied by log2 e).
+//
+// merge_kernel    log-sum-exp merge of the warp pieces of cut segments.
+// reduce_kernel   log-sum-exp merge of fixed-size partitions (explicit API).
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <type_traits>
@@ -32,24 +44,56 @@
 
 namespace pa {
 
-constexpr int kThreads = 128;               // 4 warps per CTA
-constexpr int kWarps = kThreads / 32;
-constexpr int kTile = 16;                   // tokens per tile (= MMA M / K)
+#ifndef PA_WARPS
+#define PA_WARPS 4
+#endif
+#ifndef PA_MAX_SPW
+#define PA_MAX_SPW 4
+#endif
+
+constexpr int kWarps = PA_WARPS;            // warps per CTA
+constexpr int kThreads = 32 * kWarps;
+constexpr int kMaxSpw = PA_MAX_SPW;         // tiles in flight per warp, at most
+constexpr int kTile = 16;                   // tokens per tile (= MMA M and K)
 constexpr int kSmemBudget = 227 * 1024;     // opt-in dynamic shared memory per CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded copy waits: 2 s
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned kFull = 0xffffffffu;
 
+// Shared-memory geometry of one tile, fixed per launch (depends on the block
+// size).  A K (or V) region holds 16 token rows of one head as `bpt` boxes of
+// `tr` rows; a box is nch = d * elem / 128 columns of 128 bytes:
+//   byte(row r of box b, 16-byte unit u) = b*box_stride + (u/8)*chunk_stride
+//                                          + r*128 + ((u%8) ^ swz) * 16
+// where swz = bits 7..9 of the 128-byte line's offset (the TMA 128-byte
+// swizzle).  Boxes, and in 3-D mode every column, start on a 1024-byte
+// boundary.
+struct TileGeo {
+    int tr;            // rows per box = min(16, block_size)
+    int tr_log2;
+    int bpt;           // boxes per tile = 16 / tr
+    int ops_per_box;   // TMA operations per box: 1 (4-D map) or nch (3-D map)
+    int chunk_stride;  // bytes between the 128-byte columns of a box
+    int box_stride;    // bytes between boxes
+    int kv_bytes;      // bytes of a K (or V) region
+    int q_off;         // offset of the query slot in a stage
+    int stage_bytes;   // K + V + query, multiple of 1024
+    int spw;           // stages per warp
+    int box_tx;        // bytes one box delivers
+    int q_bytes;       // bytes of the query slot payload
+};
+
 struct DecodeParams {
     void *out;
     const void *q;
-    const void *k_pool;
-    const void *v_pool;
     const int32_t *block_tables;
     const int32_t *context_lens;
-    float *tmp_out;
-    float *max_logits;
-    float *exp_sums;
+    float *tmp_out;          // explicit split-K layout [B, Hq, max_parts, d]
+    float *max_logits;       // [B, Hq, max_parts]
+    float *exp_sums;         // [B, Hq, max_parts]
+    float *wpart;            // mode 0: two partial slots per warp
+    int32_t *seg_start;      // mode 0: first global tile of each (b, h) segment
+    int32_t *total_tiles;    // mode 0: total tile count (written by the kernel)
     int32_t *dev_status;
     int64_t num_blocks;
     int num_seqs;
@@ -58,24 +102,14 @@ struct DecodeParams {
     int max_blocks;
     int block_size;
     int bs_log2;
-    int partition_size;     // multiple of kTile
+    int partition_size;      // multiple of 16; >= ctx_cap means the whole context
     int max_parts;
-    int ctx_cap;            // lengths above this are invalid
-    int always_partials;    // write partials even for single-partition sequences
-    float scale_log2;       // softmax scale * log2(e)
-};
-
-struct CacheParams {
-    const void *key;
-    const void *value;
-    void *k_pool;
-    void *v_pool;
-    const int64_t *slot_mapping;
-    int32_t *dev_status;
-    int64_t num_slots;      // nb * bs
-    int num_tokens;
-    int num_kv_heads;
-    int row_bytes;          // d * element size
+    int ctx_cap;             // lengths above this are invalid
+    int mode;                // 0 stream-K, 1 whole segments
+    int public_partials;     // mode 1: write tmp_out / max_logits / exp_sums
+    int slot_floats;         // floats per partial slot (mode 0)
+    float scale_log2;
+    TileGeo geo;
 };
 
 struct ReduceParams {
@@ -91,80 +125,51 @@ struct ReduceParams {
     int ctx_cap;
 };
 
+struct MergeParams {
+    void *out;
+    const float *wpart;
+    const int32_t *seg_start;
+    const int32_t *total_tiles;
+    const int32_t *context_lens;
+    int num_seqs;
+    int num_q_heads;
+    int num_kv_heads;
+    int ctx_cap;
+    int total_warps;
+    int slot_floats;
+};
+
 __device__ __forceinline__ void report(int32_t *status, int bit)
 {
     if (status)
         atomicOr(status, bit);
 }
 
-// =====================================================================
-// Cache write: one warp per (token, KV head, K|V) row, 16-byte copies.
-// =====================================================================
-__global__ void __launch_bounds__(256) cache_write_kernel(const CacheParams p)
+template <typename T>
+__device__ __forceinline__ void store_out(T *dst, float v);
+template <>
+__device__ __forceinline__ void store_out<float>(float *dst, float v) { *dst = v; }
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16 *dst, float v)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int64_t nrows = (int64_t)p.num_tokens * p.num_kv_heads * 2;
-    if (row >= nrows)
-        return;
-    const int kv = (int)(row & 1);
-    const int64_t th = row >> 1;
-    const int64_t t = th / p.num_kv_heads;
-    const int64_t h = th - t * p.num_kv_heads;
-    const int64_t slot = p.slot_mapping[t];
-    if (slot < 0)
-        return;
-    if (slot >= p.num_slots) {
-        if (lane == 0 && h == 0 && kv == 0)
-            report(p.dev_status, PA_DEV_BAD_SLOT);
-        return;
-    }
-    const int4 *src = reinterpret_cast<const int4 *>(
-        static_cast<const uint8_t *>(kv ? p.value : p.key) + (t * p.num_kv_heads + h) * p.row_bytes);
-    int4 *dst = reinterpret_cast<int4 *>(static_cast<uint8_t *>(kv ? p.v_pool : p.k_pool) +
-                                         (slot * p.num_kv_heads + h) * p.row_bytes);
-    const int n16 = p.row_bytes >> 4;
-    for (int c = lane; c < n16; c += 32)
-        dst[c] = __ldg(src + c);
+    *dst = __float2bfloat16_rn(v);
 }
 
 // =====================================================================
-// Work items: (sequence b, context partition, KV head h), enumerated
-// sequence-major, then partition, then head.
+// Tile enumeration
 // =====================================================================
 __device__ __forceinline__ int eff_ctx(int ctx, int cap) { return (ctx < 0 || ctx > cap) ? 0 : ctx; }
 __device__ __forceinline__ int num_parts(int ctx, int P) { return ctx <= 0 ? 1 : (ctx + P - 1) / P; }
+__device__ __forceinline__ int ntiles(int ctx) { return (ctx + kTile - 1) / kTile; }
 
-struct SeqCursor {
-    int b;         // current sequence
-    int base;      // first item of sequence b
-    int cnt;       // items of sequence b (= parts * Hkv)
-    int ctx;       // effective length of b
-    int ctx_raw;   // length as given
-};
-
-struct Item {
-    int b, h, part, t0, t1, ctx, ctx_raw;
-};
-
-__device__ __forceinline__ void cursor_reset(SeqCursor &c)
-{
-    c.b = -1;
-    c.base = 0;
-    c.cnt = 0;
-    c.ctx = 0;
-    c.ctx_raw = 0;
-}
-
-// Total number of items (every lane gets it).
-__device__ int count_items(const DecodeParams &p, int lane)
+// Total tiles of the batch (every lane gets it).
+__device__ __forceinline__ int count_tiles(const DecodeParams &p, int lane)
 {
     int sum = 0;
     for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
         const int b = b0 + lane;
         if (b < p.num_seqs)
-            sum += num_parts(eff_ctx(p.context_lens[b], p.ctx_cap), p.partition_size) *
-                   p.num_kv_heads;
+            sum += ntiles(eff_ctx(p.context_lens[b], p.ctx_cap)) * p.num_kv_heads;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
@@ -172,252 +177,193 @@ __device__ int count_items(const DecodeParams &p, int lane)
     return sum;
 }
 
-// Moves the cursor forward to the sequence holding item g (g must not be
-// below the cursor's base and must be below the total).  Warp-cooperative:
-// 32 sequences per step with a shuffle prefix sum.
-__device__ void cursor_seek(SeqCursor &c, int g, const DecodeParams &p, int lane)
-{
-    while (g >= c.base + c.cnt) {
-        const int base = c.base + c.cnt;
-        const int b0 = c.b + 1;
-        const int bb = b0 + lane;
-        const bool in = bb < p.num_seqs;
-        const int raw = in ? p.context_lens[bb] : 0;
-        const int ctx = eff_ctx(raw, p.ctx_cap);
-        const int cnt = in ? num_parts(ctx, p.partition_size) * p.num_kv_heads : 0;
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o)
-                incl += v;
-        }
-        const unsigned hit = __ballot_sync(kFull, in && g < base + incl);
-        const int L = hit ? (__ffs(hit) - 1) : 31;
-        c.b = b0 + L;
-        c.base = base + __shfl_sync(kFull, incl - cnt, L);
-        c.cnt = __shfl_sync(kFull, cnt, L);
-        c.ctx = __shfl_sync(kFull, ctx, L);
-        c.ctx_raw = __shfl_sync(kFull, raw, L);
-    }
-}
-
-__device__ __forceinline__ Item locate(SeqCursor &c, int g, const DecodeParams &p, int lane)
-{
-    cursor_seek(c, g, p, lane);
-    Item it;
-    const int local = g - c.base;
-    it.b = c.b;
-    it.part = local / p.num_kv_heads;
-    it.h = local - it.part * p.num_kv_heads;
-    it.ctx = c.ctx;
-    it.ctx_raw = c.ctx_raw;
-    it.t0 = it.part * p.partition_size;
-    it.t1 = min(it.t0 + p.partition_size, it.ctx);
-    return it;
-}
-
-__device__ __forceinline__ int item_tiles(const Item &it)
-{
-    return it.t1 > it.t0 ? (it.t1 - it.t0 + kTile - 1) / kTile : 0;
-}
-
-// =====================================================================
-// Shared-memory layout of the decode kernel
-// =====================================================================
-template <typename T, int D, int G>
-struct Layout {
-    static constexpr int kRowBytes = D * (int)sizeof(T);
-    static constexpr int kRowStride = kRowBytes + 16;          // pad: conflict-free ldmatrix
-    static constexpr int kHalf = kTile * kRowStride;            // K (or V) part of a stage
-    static constexpr int kStage = 2 * kHalf;
-    static constexpr int kMergeFloats = G * D + 2 * G + 1;      // acc, m, l, bad flag
-    static constexpr int kMergeBytes = kWarps * kMergeFloats * 4;
-    static constexpr int kScoreBytes = kWarps * kTile * G * 4;
-    static constexpr int kFixed = ((kMergeBytes + kScoreBytes + 15) / 16) * 16 + 8 * kWarps * 4;
-    static constexpr int kSpwFit = (kSmemBudget - kFixed) / (kWarps * kStage);
-    static constexpr int kSPW = kSpwFit > 4 ? 4 : kSpwFit;     // stages per warp
-    static_assert(kSPW >= 1, "a stage must fit");
-    static constexpr int kStagesBytes = kWarps * kSPW * kStage;
-    static constexpr int kMergeOff = kStagesBytes;
-    static constexpr int kScoreOff = kMergeOff + kMergeBytes;
-    static constexpr int kBarOff = ((kScoreOff + kScoreBytes + 15) / 16) * 16;
-    static constexpr int kSmem = kBarOff + 8 * kWarps * kSPW;
-    static_assert(kSmem <= kSmemBudget, "shared memory over budget");
+// A window of 32 consecutive sequences with their tile counts, one per lane,
+// used to map global tile indices to sequences.
+struct SeqWindow {
+    int b0;      // first sequence of the window
+    int base;    // global index of the first tile of sequence b0
+    int cnt;     // this lane's sequence: tiles (Hkv * ntiles)
+    int incl;    // inclusive prefix of cnt over the window
+    int ctx;     // this lane's sequence: effective length
 };
 
-// =====================================================================
-// Tile math, CUDA cores
-// =====================================================================
-template <typename T, int D, int G>
-struct SimtMath {
-    static constexpr int VEC = 16 / (int)sizeof(T);   // elements per 16-byte chunk
-    static constexpr int NCH = D / VEC;                // chunks per row
-    static constexpr int LPR = NCH < 32 ? NCH : 32;    // lanes per row
-    static constexpr int RPI = 32 / LPR;               // rows side by side
-    static constexpr int CPL = NCH / LPR;              // chunks per lane
-    static constexpr int NE = CPL * VEC;               // elements per lane
-    static constexpr int RPL = kTile / RPI;            // rows per lane per tile
-    using L = Layout<T, D, G>;
-
-    float q[G][NE];
-    float acc[G][NE];
-    float m[G];   // running max, log2 domain (warp-uniform)
-    float l[G];   // running sum over this lane's rows
-
-    __device__ __forceinline__ static void load_chunk(const void *src, float (&x)[VEC])
-    {
-        const uint4 u = *reinterpret_cast<const uint4 *>(src);
-        if constexpr (sizeof(T) == 4) {
-            x[0] = __uint_as_float(u.x);
-            x[1] = __uint_as_float(u.y);
-            x[2] = __uint_as_float(u.z);
-            x[3] = __uint_as_float(u.w);
-        } else {
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+__device__ __forceinline__ void window_load(SeqWindow &w, int b0, int base, const DecodeParams &p,
+                                            int lane)
+{
+    w.b0 = b0;
+    w.base = base;
+    const int b = b0 + lane;
+    w.ctx = b < p.num_seqs ? eff_ctx(p.context_lens[b], p.ctx_cap) : 0;
+    w.cnt = ntiles(w.ctx) * p.num_kv_heads;
+    int incl = w.cnt;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                x[2 * i] = ptx::bf16lo_to_f32(w[i]);
-                x[2 * i + 1] = ptx::bf16hi_to_f32(w[i]);
-            }
-        }
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o)
+            incl += v;
     }
+    w.incl = incl;
+}
 
-    __device__ __forceinline__ void begin(const T *qhead, float scale_log2, int lane)
-    {
-        const int li = lane % LPR;
+// Resolves each lane's global tile index g (ignored where !want) to its
+// sequence: b, the global index of the sequence's first tile, and its
+// effective length.  The window only moves forward, so targets must not
+// precede it.  Warp-uniform control flow.
+__device__ __forceinline__ void window_find(SeqWindow &w, int g, bool want, int &b, int &seqbase,
+                                            int &ctx, const DecodeParams &p, int lane)
+{
+    bool done = !want;
+    b = 0;
+    seqbase = 0;
+    ctx = 0;
+    while (true) {
+        const int last = w.base + __shfl_sync(kFull, w.incl, 31);
+        const bool here = !done && g < last;
+        // pos = number of window sequences whose tiles all precede g
+        int pos = 0;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                float x[VEC];
-                load_chunk(qhead + g * D + (c * LPR + li) * VEC, x);
-#pragma unroll
-                for (int v = 0; v < VEC; ++v) {
-                    q[g][c * VEC + v] = x[v] * scale_log2;
-                    acc[g][c * VEC + v] = 0.f;
-                }
-            }
-            m[g] = -INFINITY;
-            l[g] = 0.f;
+        for (int s = 16; s > 0; s >>= 1) {
+            const int v = __shfl_sync(kFull, w.incl, pos + s - 1);
+            if (w.base + v <= g)
+                pos += s;
         }
+        const int src = pos < 32 ? pos : 31;
+        const int incl_at = __shfl_sync(kFull, w.incl, src);
+        const int cnt_at = __shfl_sync(kFull, w.cnt, src);
+        const int ctx_at = __shfl_sync(kFull, w.ctx, src);
+        if (here) {
+            b = w.b0 + pos;
+            seqbase = w.base + incl_at - cnt_at;
+            ctx = ctx_at;
+            done = true;
+        }
+        if (!__any_sync(kFull, !done))
+            break;
+        if (w.b0 + 32 >= p.num_seqs)   // targets past the last tile: leave them
+            break;
+        window_load(w, w.b0 + 32, last, p, lane);
     }
+}
 
-    __device__ __forceinline__ void tile(const uint8_t *ks, const uint8_t *vs, int n,
-                                         float *scores, int lane)
-    {
-        const int li = lane % LPR;
-        const int rg = lane / LPR;
-        float tmax[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-            tmax[g] = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-            const int r = rg + i * RPI;
-            float part[G];
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-                part[g] = 0.f;
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                float k[VEC];
-                load_chunk(ks + r * L::kRowStride + (c * LPR + li) * 16, k);
-#pragma unroll
-                for (int g = 0; g < G; ++g)
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v)
-                        part[g] = fmaf(q[g][c * VEC + v], k[v], part[g]);
-            }
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-#pragma unroll
-                for (int o = LPR / 2; o > 0; o >>= 1)
-                    part[g] += __shfl_xor_sync(kFull, part[g], o);
-                const float s = r < n ? part[g] : -INFINITY;
-                tmax[g] = fmaxf(tmax[g], s);
-                if (li == 0)
-                    scores[r * G + g] = s;
-            }
-        }
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-#pragma unroll
-            for (int o = LPR; o < 32; o <<= 1)
-                tmax[g] = fmaxf(tmax[g], __shfl_xor_sync(kFull, tmax[g], o));
-        }
-        __syncwarp();
-        float ref[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float mn = fmaxf(m[g], tmax[g]);
-            const float alpha = mn == -INFINITY ? 1.f : ptx::ex2(m[g] - mn);
-            m[g] = mn;
-            ref[g] = mn == -INFINITY ? 0.f : mn;
-            l[g] *= alpha;
-#pragma unroll
-            for (int e = 0; e < NE; ++e)
-                acc[g][e] *= alpha;
-        }
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-            const int r = rg + i * RPI;
-            if (r < n) {
-                float pr[G];
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    pr[g] = ptx::ex2(scores[r * G + g] - ref[g]);
-                    l[g] += pr[g];
-                }
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) {
-                    float v[VEC];
-                    load_chunk(vs + r * L::kRowStride + (c * LPR + li) * 16, v);
-#pragma unroll
-                    for (int g = 0; g < G; ++g)
-#pragma unroll
-                        for (int e = 0; e < VEC; ++e)
-                            acc[g][c * VEC + e] = fmaf(pr[g], v[e], acc[g][c * VEC + e]);
-                }
-            }
-        }
-        __syncwarp();
-    }
-
-    // Writes this warp's (acc, m, l) into its merge row; lanes of row group 0
-    // hold the sums over all row groups.
-    __device__ __forceinline__ void finish(float *mrow, int lane)
-    {
-        const int li = lane % LPR;
-        const int rg = lane / LPR;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-#pragma unroll
-            for (int o = LPR; o < 32; o <<= 1) {
-                l[g] += __shfl_xor_sync(kFull, l[g], o);
-#pragma unroll
-                for (int e = 0; e < NE; ++e)
-                    acc[g][e] += __shfl_xor_sync(kFull, acc[g][e], o);
-            }
-        }
-        if (rg == 0) {
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int c = 0; c < CPL; ++c)
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v)
-                        mrow[g * D + (c * LPR + li) * VEC + v] = acc[g][c * VEC + v];
-        }
-        if (lane == 0) {
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                mrow[G * D + g] = m[g];
-                mrow[G * D + G + g] = l[g];
-            }
-        }
-    }
+// Tile descriptor; a batch holds 32 consecutive tiles, one per lane.
+struct TileDesc {
+    int b, h, part, j, ns, t0, n, ctx;
+    int phys[4];
 };
+
+// Descriptor of lane `src` of batch d1 (sel) or d0 (!sel), to every lane.
+__device__ __forceinline__ TileDesc shfl_desc(const TileDesc &d0, const TileDesc &d1, bool sel,
+                                              int src)
+{
+    TileDesc o;
+    o.b = __shfl_sync(kFull, sel ? d1.b : d0.b, src);
+    o.h = __shfl_sync(kFull, sel ? d1.h : d0.h, src);
+    o.part = __shfl_sync(kFull, sel ? d1.part : d0.part, src);
+    o.j = __shfl_sync(kFull, sel ? d1.j : d0.j, src);
+    o.ns = __shfl_sync(kFull, sel ? d1.ns : d0.ns, src);
+    o.t0 = __shfl_sync(kFull, sel ? d1.t0 : d0.t0, src);
+    o.n = __shfl_sync(kFull, sel ? d1.n : d0.n, src);
+    o.ctx = __shfl_sync(kFull, sel ? d1.ctx : d0.ctx, src);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        o.phys[k] = __shfl_sync(kFull, sel ? d1.phys[k] : d0.phys[k], src);
+    return o;
+}
+
+// Fills the descriptors of tiles [base, base + 32) below `end` and starts
+// their block-table loads.
+__device__ __forceinline__ void fill_batch(TileDesc &d, SeqWindow &w, int base, int end,
+                                           const DecodeParams &p, int lane)
+{
+    const int g = base + lane;
+    const bool want = g < end;
+    int b, seqbase, ctx;
+    window_find(w, g, want, b, seqbase, ctx, p, lane);
+    d.b = b;
+    d.h = 0;
+    d.part = 0;
+    d.j = 0;
+    d.ns = 1;
+    d.t0 = 0;
+    d.n = 0;
+    d.ctx = ctx;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        d.phys[k] = -1;
+    if (!want)
+        return;
+    const int Hkv = p.num_kv_heads;
+    const int nt = ntiles(ctx);
+    const int PT = p.partition_size >> 4;             // tiles of a full partition
+    const int x = g - seqbase;
+    const int nparts = num_parts(ctx, p.partition_size);
+    int part = (int)((int64_t)x / ((int64_t)Hkv * PT));
+    if (part > nparts - 1)
+        part = nparts - 1;
+    const int rem = x - (int)((int64_t)part * Hkv * PT);
+    const int np = min(PT, nt - part * PT);             // tiles of this partition
+    d.h = rem / np;
+    d.j = rem - d.h * np;
+    d.ns = np;
+    d.part = part;
+    d.t0 = part * p.partition_size + kTile * d.j;
+    const int64_t pend = (int64_t)(part + 1) * p.partition_size;
+    const int seg_end = pend < ctx ? (int)pend : ctx;
+    d.n = min(kTile, seg_end - d.t0);
+    const int32_t *row = p.block_tables + (int64_t)b * p.max_blocks;
+    const int tr = p.geo.tr;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        if (k < p.geo.bpt && k * tr < d.n)
+            d.phys[k] = row[(d.t0 + k * tr) >> p.bs_log2];
+}
+
+// First tile of warp gw's range (T for gw == total_warps).
+__device__ __forceinline__ int range_begin(int gw, int total_warps, int T, const DecodeParams &p,
+                                           int lane)
+{
+    if (gw >= total_warps)
+        return T;
+    const int x = (int)((int64_t)gw * T / total_warps);
+    if (p.mode == 0 || x >= T)
+        return x;
+    // mode 1: the first segment start at or after x
+    SeqWindow w;
+    window_load(w, 0, 0, p, lane);
+    TileDesc d;
+    fill_batch(d, w, x, x + 1, p, lane);
+    const int j = __shfl_sync(kFull, d.j, 0);
+    const int ns = __shfl_sync(kFull, d.ns, 0);
+    return j == 0 ? x : x - j + ns;
+}
+
+// =====================================================================
+// Swizzled addressing of a K or V region
+// =====================================================================
+// Address of 16-byte unit u of token row t in a region starting at `reg`.
+__device__ __forceinline__ uint32_t kv_addr(uint32_t reg, int t, int u, const TileGeo &g)
+{
+    const int box = t >> g.tr_log2;
+    const int r = t & (g.tr - 1);
+    const uint32_t line = (uint32_t)(box * g.box_stride + (u >> 3) * g.chunk_stride + r * 128);
+    return reg + line + ((((uint32_t)u & 7u) ^ ((line >> 7) & 7u)) << 4);
+}
+
+// Same, for one 16-row box (block size >= 16): the swizzle phase is t & 7.
+__device__ __forceinline__ uint32_t kv_addr16(uint32_t reg, int t, int u)
+{
+    return reg + (uint32_t)((u >> 3) * (kTile * 128) + t * 128) +
+           ((((uint32_t)u & 7u) ^ ((uint32_t)t & 7u)) << 4);
+}
+
+template <bool TR16>
+__device__ __forceinline__ uint32_t tile_addr(uint32_t reg, int t, int u, const TileGeo &g)
+{
+    if constexpr (TR16)
+        return kv_addr16(reg, t, u);
+    else
+        return kv_addr(reg, t, u, g);
+}
 
 // =====================================================================
 // Tile math, bf16 tensor cores (warp-level MMA)
@@ -425,30 +371,30 @@ struct SimtMath {
 // Fragment maps (r = lane / 4, c = lane % 4):
 //   S = K Q^T, M = 16 tokens, N = 8 heads (G real), K = d in steps of 16.
 //     S frag: s0,s1 = S[tok r][head 2c, 2c+1], s2,s3 = S[tok r+8][...].
-//   O^T += V^T P^T, M = 16 d-rows per tile mt, N = 8 heads, K = 16 tokens.
+//   O^T += V^T P^T, M = 16 d-rows per step k, N = 8 heads, K = 16 tokens.
 //     P^T frag from movmatrix of the packed S frag; O^T frag:
-//     a0,a1 = O^T[d 16mt+r][head 2c, 2c+1], a2,a3 = O^T[d 16mt+r+8][...].
-// Each lane owns heads 2c and 2c+1 in both maps, so the running max, sum and
-// rescale of those heads never leave the lane (apart from the max reduce).
+//     a0,a1 = O^T[d 16k+r][head 2c, 2c+1], a2,a3 = O^T[d 16k+r+8][...].
+// A lane owns heads 2c and 2c+1 in both maps, so the running max, sum and
+// rescale of those heads stay in the lane (apart from the max reduction).
 // =====================================================================
-template <int D, int G>
+template <int D, int G, bool TR16>
 struct MmaMath {
     static_assert(G <= 8, "group must fit the N = 8 MMA");
     static constexpr int KS = D / 16;
-    using L = Layout<__nv_bfloat16, D, G>;
 
     uint32_t qf[KS][2];
     float acc[KS][4];
     float m[2];
     float l[2];
 
-    __device__ __forceinline__ void begin(const __nv_bfloat16 *qhead, float, int lane)
+    // Query fragments from the stage's query slot ([G][D] bf16, row-major).
+    __device__ __forceinline__ void begin(const uint8_t *qslot, int lane)
     {
         const int r = lane >> 2, c = lane & 3;
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
             if (r < G) {
-                const uint32_t *qr = reinterpret_cast<const uint32_t *>(qhead + r * D + 16 * k);
+                const uint32_t *qr = reinterpret_cast<const uint32_t *>(qslot + (r * D + 16 * k) * 2);
                 qf[k][0] = qr[c];
                 qf[k][1] = qr[4 + c];
             } else {
@@ -464,16 +410,16 @@ struct MmaMath {
     }
 
     __device__ __forceinline__ void tile(uint32_t ks, uint32_t vs, int n, float scale_log2,
-                                         int lane)
+                                         const TileGeo &geo, int lane)
     {
         const int r = lane >> 2;
         // ---- S = K Q^T (two accumulation chains)
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t kaddr = ks + (lane & 15) * L::kRowStride + (lane >> 4) * 16;
+        const int krow = lane & 15, khalf = lane >> 4;
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
             uint32_t a[4];
-            ptx::ldsm_x4(kaddr + k * 32, a);
+            ptx::ldsm_x4(tile_addr<TR16>(ks, krow, 2 * k + khalf, geo), a);
             if (k & 1)
                 ptx::mma_bf16_16816(sb, a, qf[k][0], qf[k][1]);
             else
@@ -522,282 +468,564 @@ struct MmaMath {
         const uint32_t b0 = ptx::movmatrix_trans(p01);
         const uint32_t b1 = ptx::movmatrix_trans(p23);
         // ---- O^T += V^T P^T
-        const uint32_t vaddr =
-            vs + ((lane & 7) + ((lane >> 4) << 3)) * L::kRowStride + ((lane >> 3) & 1) * 16;
+        const int vrow = (lane & 7) + ((lane >> 4) << 3), vhalf = (lane >> 3) & 1;
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
             uint32_t a[4];
-            ptx::ldsm_x4_trans(vaddr + k * 32, a);
+            ptx::ldsm_x4_trans(tile_addr<TR16>(vs, vrow, 2 * k + vhalf, geo), a);
             ptx::mma_bf16_16816(acc[k], a, b0, b1);
         }
     }
 
-    __device__ __forceinline__ void finish(float *mrow, int lane)
+    // Completes the running sums: afterwards every lane holds the sums of its
+    // two heads.
+    __device__ __forceinline__ void finish()
     {
-        const int r = lane >> 2, c = lane & 3;
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
             l[0] += __shfl_xor_sync(kFull, l[0], o);
             l[1] += __shfl_xor_sync(kFull, l[1], o);
         }
+    }
+
+    // Calls f(head, d, acc, sum) for every unnormalised accumulator this lane
+    // holds (heads < G), and fm(head, max, sum) once per head.
+    template <typename F, typename FM>
+    __device__ __forceinline__ void for_each(int lane, F f, FM fm) const
+    {
+        const int r = lane >> 2, c = lane & 3;
         const int h0 = 2 * c, h1 = 2 * c + 1;
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
             const int d0 = 16 * k + r;
             if (h0 < G) {
-                mrow[h0 * D + d0] = acc[k][0];
-                mrow[h0 * D + d0 + 8] = acc[k][2];
+                f(h0, d0, acc[k][0], l[0]);
+                f(h0, d0 + 8, acc[k][2], l[0]);
             }
             if (h1 < G) {
-                mrow[h1 * D + d0] = acc[k][1];
-                mrow[h1 * D + d0 + 8] = acc[k][3];
+                f(h1, d0, acc[k][1], l[1]);
+                f(h1, d0 + 8, acc[k][3], l[1]);
             }
         }
         if (r == 0) {
-            if (h0 < G) {
-                mrow[G * D + h0] = m[0];
-                mrow[G * D + G + h0] = l[0];
-            }
-            if (h1 < G) {
-                mrow[G * D + h1] = m[1];
-                mrow[G * D + G + h1] = l[1];
-            }
+            if (h0 < G)
+                fm(h0, m[0], l[0]);
+            if (h1 < G)
+                fm(h1, m[1], l[1]);
         }
     }
 };
 
 // =====================================================================
-// Decode kernel
+// Tile math, CUDA cores
 // =====================================================================
-template <typename T>
-__device__ __forceinline__ void store_out(T *dst, float v);
-template <>
-__device__ __forceinline__ void store_out<float>(float *dst, float v) { *dst = v; }
-template <>
-__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16 *dst, float v)
-{
-    *dst = __float2bfloat16_rn(v);
-}
+template <typename T, int D, int G, bool TR16>
+struct SimtMath {
+    static constexpr int VEC = 16 / (int)sizeof(T);   // elements per 16-byte unit
+    static constexpr int NU = D / VEC;                 // units per row
+    static constexpr int LPR = NU < 32 ? NU : 32;      // lanes per row
+    static constexpr int RPI = 32 / LPR;               // rows side by side
+    static constexpr int UPL = NU / LPR;               // units per lane
+    static constexpr int NE = UPL * VEC;               // elements per lane
+    static constexpr int RPL = kTile / RPI;            // rows per lane per tile
 
-template <typename T, int D, int G, bool MMA>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p)
-{
-    using L = Layout<T, D, G>;
-    constexpr int SPW = L::kSPW;
-    extern __shared__ __align__(128) uint8_t smem[];
+    float q[G][NE];
+    float acc[G][NE];
+    float m[G];   // running max, log2 domain (warp-uniform)
+    float l[G];   // running sum over this lane's rows
 
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    float *merge = reinterpret_cast<float *>(smem + L::kMergeOff);
-    float *scores = reinterpret_cast<float *>(smem + L::kScoreOff) + warp * kTile * G;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
-
-    // Rows that are never copied (past a sequence's end) must hold finite
-    // values: their weight is exactly 0 and 0 * finite = 0 in the MMA.
-    for (int i = threadIdx.x; i < L::kStagesBytes / 16; i += kThreads)
-        reinterpret_cast<int4 *>(smem)[i] = make_int4(0, 0, 0, 0);
-    if (threadIdx.x < kWarps * SPW)
-        ptx::mbar_init(ptx::smem_u32(&bars[threadIdx.x]), 1);
-    ptx::fence_mbar_init();
-    ptx::fence_proxy_async_smem();
-    __syncthreads();
-
-    const int total = count_items(p, lane);
-    const uint32_t stage0 = ptx::smem_u32(smem + warp * SPW * L::kStage);
-    const uint32_t bar0 = ptx::smem_u32(&bars[warp * SPW]);
-    const uint8_t *kpool = static_cast<const uint8_t *>(p.k_pool);
-    const uint8_t *vpool = static_cast<const uint8_t *>(p.v_pool);
-    const int Hkv = p.num_kv_heads;
-    const uint64_t policy = ptx::policy_evict_first();
-
-    // ---------------- producer: this warp's job stream, SPW jobs ahead
-    SeqCursor pc;
-    cursor_reset(pc);
-    int pk = -1, pj = 0, pnt = 0;
-    bool pdone = false;
-    Item pit{};
-    uint32_t badmask = 0;   // stage s holds a tile with a bad block id
-    uint32_t issued = 0, consumed = 0;
-    bool aborted = false;
-
-    auto next_job = [&](Item &it, int &j) -> bool {
-        while (!pdone) {
-            if (pk >= 0 && pj < pnt) {
-                it = pit;
-                j = pj;
-                pj += kWarps;
-                return true;
+    __device__ __forceinline__ static void cvt(const uint4 u, float (&x)[VEC])
+    {
+        if constexpr (sizeof(T) == 4) {
+            x[0] = __uint_as_float(u.x);
+            x[1] = __uint_as_float(u.y);
+            x[2] = __uint_as_float(u.z);
+            x[3] = __uint_as_float(u.w);
+        } else {
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                x[2 * i] = ptx::bf16lo_to_f32(w[i]);
+                x[2 * i + 1] = ptx::bf16hi_to_f32(w[i]);
             }
-            ++pk;
-            const long long g = (long long)blockIdx.x + (long long)pk * gridDim.x;
-            if (g >= total) {
-                pdone = true;
-                break;
-            }
-            pit = locate(pc, (int)g, p, lane);
-            pnt = item_tiles(pit);
-            pj = warp;
         }
-        return false;
-    };
-
-    auto issue = [&](const Item &it, int j, int s) {
-        const int tb = it.t0 + j * kTile;
-        const int n = min(kTile, it.t1 - tb);
-        const int row = lane & 15;
-        const int isv = lane >> 4;
-        const int t = tb + row;
-        const bool valid = row < n;
-        int phys = 0;
-        if (valid)
-            phys = p.block_tables[(int64_t)it.b * p.max_blocks + (t >> p.bs_log2)];
-        const bool bad = valid && (phys < 0 || (int64_t)phys >= p.num_blocks);
-        const bool go = valid && !bad;
-        const unsigned gom = __ballot_sync(kFull, go);
-        if (__ballot_sync(kFull, bad))
-            badmask |= 1u << s;
-        const uint32_t bar = bar0 + 8u * s;
-        if (lane == 0)
-            ptx::mbar_arrive_expect_tx(bar, (uint32_t)__popc(gom) * L::kRowBytes);
-        __syncwarp();
-        if (go) {
-            const int64_t src_row =
-                ((int64_t)phys * p.block_size + (t & (p.block_size - 1))) * Hkv + it.h;
-            const uint8_t *src = (isv ? vpool : kpool) + src_row * L::kRowBytes;
-            const uint32_t dst = stage0 + s * L::kStage + isv * L::kHalf + row * L::kRowStride;
-            ptx::bulk_g2s_hint(dst, src, L::kRowBytes, bar, policy);
-        }
-    };
-
-    for (int s = 0; s < SPW; ++s) {
-        Item it;
-        int j;
-        if (!next_job(it, j))
-            break;
-        issue(it, j, s);
-        ++issued;
     }
 
-    // ---------------- consumer: items in the same order
-    SeqCursor cc;
-    cursor_reset(cc);
-    for (int k = 0;; ++k) {
-        const long long g = (long long)blockIdx.x + (long long)k * gridDim.x;
-        if (g >= total)
-            break;
-        const Item it = locate(cc, (int)g, p, lane);
-        const int nt = item_tiles(it);
-        const T *qhead = static_cast<const T *>(p.q) +
-                         ((int64_t)it.b * p.num_q_heads + (int64_t)it.h * G) * D;
+    __device__ __forceinline__ static uint4 lds128(uint32_t addr)
+    {
+        uint4 v;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "r"(addr));
+        return v;
+    }
 
-        using Math = typename std::conditional<MMA, MmaMath<D, G>, SimtMath<T, D, G>>::type;
-        Math math;
-        if constexpr (MMA)
-            math.begin(reinterpret_cast<const __nv_bfloat16 *>(qhead), p.scale_log2, lane);
-        else
-            math.begin(qhead, p.scale_log2, lane);
+    __device__ __forceinline__ void begin(const uint8_t *qslot, int lane, float scale_log2)
+    {
+        const int li = lane % LPR;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int c = 0; c < UPL; ++c) {
+                float x[VEC];
+                cvt(*reinterpret_cast<const uint4 *>(qslot + (g * D + (c * LPR + li) * VEC) *
+                                                                 (int)sizeof(T)),
+                    x);
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    q[g][c * VEC + v] = x[v] * scale_log2;
+                    acc[g][c * VEC + v] = 0.f;
+                }
+            }
+            m[g] = -INFINITY;
+            l[g] = 0.f;
+        }
+    }
+
+    __device__ __forceinline__ void tile(uint32_t ks, uint32_t vs, int n, float *scores,
+                                         const TileGeo &geo, int lane)
+    {
+        const int li = lane % LPR;
+        const int rg = lane / LPR;
+        float tmax[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            tmax[g] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            const int r = rg + i * RPI;
+            float part[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+                part[g] = 0.f;
+#pragma unroll
+            for (int c = 0; c < UPL; ++c) {
+                float k[VEC];
+                cvt(lds128(tile_addr<TR16>(ks, r, c * LPR + li, geo)), k);
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v)
+                        part[g] = fmaf(q[g][c * VEC + v], k[v], part[g]);
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+#pragma unroll
+                for (int o = LPR / 2; o > 0; o >>= 1)
+                    part[g] += __shfl_xor_sync(kFull, part[g], o);
+                const float s = r < n ? part[g] : -INFINITY;
+                tmax[g] = fmaxf(tmax[g], s);
+                if (li == 0)
+                    scores[r * G + g] = s;
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int o = LPR; o < 32; o <<= 1)
+                tmax[g] = fmaxf(tmax[g], __shfl_xor_sync(kFull, tmax[g], o));
+        }
+        __syncwarp();
+        float ref[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float mn = fmaxf(m[g], tmax[g]);
+            const float alpha = mn == -INFINITY ? 1.f : ptx::ex2(m[g] - mn);
+            m[g] = mn;
+            ref[g] = mn == -INFINITY ? 0.f : mn;
+            l[g] *= alpha;
+#pragma unroll
+            for (int e = 0; e < NE; ++e)
+                acc[g][e] *= alpha;
+        }
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            const int r = rg + i * RPI;
+            if (r < n) {
+                float pr[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    pr[g] = ptx::ex2(scores[r * G + g] - ref[g]);
+                    l[g] += pr[g];
+                }
+#pragma unroll
+                for (int c = 0; c < UPL; ++c) {
+                    float v[VEC];
+                    cvt(lds128(tile_addr<TR16>(vs, r, c * LPR + li, geo)), v);
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+#pragma unroll
+                        for (int e = 0; e < VEC; ++e)
+                            acc[g][c * VEC + e] = fmaf(pr[g], v[e], acc[g][c * VEC + e]);
+                }
+            }
+        }
+        __syncwarp();
+    }
+
+    // Sums acc and l over the row groups: afterwards lanes of row group 0 hold
+    // the accumulator totals and every lane holds the sums.
+    __device__ __forceinline__ void finish()
+    {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int o = LPR; o < 32; o <<= 1) {
+                l[g] += __shfl_xor_sync(kFull, l[g], o);
+#pragma unroll
+                for (int e = 0; e < NE; ++e)
+                    acc[g][e] += __shfl_xor_sync(kFull, acc[g][e], o);
+            }
+        }
+    }
+
+    template <typename F, typename FM>
+    __device__ __forceinline__ void for_each(int lane, F f, FM fm) const
+    {
+        const int li = lane % LPR;
+        const int rg = lane / LPR;
+        if (rg == 0) {
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int c = 0; c < UPL; ++c)
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v)
+                        f(g, (c * LPR + li) * VEC + v, acc[g][c * VEC + v], l[g]);
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+                fm(g, m[g], l[g]);
+        }
+    }
+};
+
+// Bytes of the decode kernel's dynamic shared memory for a geometry.
+__host__ __device__ constexpr int decode_smem_fixed(int G)
+{
+    return 1024 + 8 * kWarps * kMaxSpw + kWarps * kTile * G * 4;
+}
+
+// =====================================================================
+// Decode kernel
+// =====================================================================
+template <typename T, int D, int G, bool MMA, bool TR16>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const TileGeo &geo = p.geo;
+    const int spw = geo.spw;
+    const int gw = blockIdx.x * kWarps + warp;
+    const int total_warps = gridDim.x * kWarps;
+    const int Hkv = p.num_kv_heads;
+    const int Hq = p.num_q_heads;
+
+    // 1024-byte aligned layout: [stages][barriers][score rows]
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t *sgen = smem_raw + (sbase - raw);
+    const int stages_bytes = kWarps * spw * geo.stage_bytes;
+    const uint32_t stage0 = sbase + (uint32_t)(warp * spw * geo.stage_bytes);
+    const uint8_t *stage0_gen = sgen + warp * spw * geo.stage_bytes;
+    const uint32_t bar0 = sbase + (uint32_t)stages_bytes + 8u * (uint32_t)(warp * kMaxSpw);
+    float *scores = reinterpret_cast<float *>(sgen + stages_bytes + 8 * kWarps * kMaxSpw) +
+                    warp * kTile * G;
+
+    if (lane == 0) {
+        for (int s = 0; s < spw; ++s)
+            ptx::mbar_init(bar0 + 8u * s, 1);
+        ptx::prefetch_tensormap(&tmap_k);
+        ptx::prefetch_tensormap(&tmap_v);
+    }
+    ptx::fence_mbar_init();
+    __syncwarp();
+
+    const int total = count_tiles(p, lane);
+    if (p.mode == 0 && gw == 0 && lane == 0)
+        *p.total_tiles = total;
+
+    // Sequences without tiles (length 0 or invalid) get a zero output.
+    for (int b = gw; b < p.num_seqs; b += total_warps) {
+        const int rawc = p.context_lens[b];
+        if (eff_ctx(rawc, p.ctx_cap) > 0)
+            continue;
+        if (rawc != 0 && lane == 0)
+            report(p.dev_status, PA_DEV_BAD_CONTEXT);
+        T *o = static_cast<T *>(p.out) + (int64_t)b * Hq * D;
+        for (int i = lane; i < Hq * D; i += 32)
+            store_out<T>(o + i, 0.f);
+        if (p.public_partials) {
+            for (int hq = 0; hq < Hq; ++hq) {
+                const int64_t slot = ((int64_t)b * Hq + hq) * p.max_parts;
+                for (int e = lane; e < D; e += 32)
+                    p.tmp_out[slot * D + e] = 0.f;
+                if (lane == 0) {
+                    p.max_logits[slot] = -INFINITY;
+                    p.exp_sums[slot] = 0.f;
+                }
+            }
+        }
+    }
+
+    const int R0 = range_begin(gw, total_warps, total, p, lane);
+    const int R1 = range_begin(gw + 1, total_warps, total, p, lane);
+    if (R0 >= R1)
+        return;
+
+    const uint64_t policy = ptx::policy_evict_first();
+    SeqWindow win;
+    window_load(win, 0, 0, p, lane);
+    TileDesc bat0, bat1;
+    fill_batch(bat0, win, R0, R1, p, lane);
+    fill_batch(bat1, win, R0 + 32, R1, p, lane);
+    int filled = 2;   // batches prepared so far
+
+    uint32_t badmask = 0;   // stage s holds a tile with a block id outside the pool
+    bool aborted = false;
+    int issued = R0;
+
+    auto issue = [&](int i) {
+        const int k = i - R0;
+        const int s = k % spw;
+        const TileDesc d = shfl_desc(bat0, bat1, (k >> 5) & 1, k & 31);
+        const bool newseg = d.j == 0 || i == R0;
+        const uint32_t stage = stage0 + (uint32_t)(s * geo.stage_bytes);
+        const uint32_t bar = bar0 + 8u * s;
+        int tx = newseg ? geo.q_bytes : 0;
         bool bad = false;
-
-        for (int j = warp; j < nt; j += kWarps) {
-            const int s = (int)(consumed % SPW);
-            bool ok = false;
-            if (consumed < issued) {
-                ok = ptx::mbar_wait_bounded(bar0 + 8u * s, (consumed / SPW) & 1u, kWaitLimitNs);
-                if (!ok) {
-                    aborted = true;
-                    if (lane == 0)
-                        report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
-                }
-            } else {
-                aborted = true;   // job was never issued (only after an abort)
-            }
-            if ((badmask >> s) & 1u) {
-                bad = true;
-                badmask &= ~(1u << s);
-            }
-            if (ok && !bad) {
-                const int n = min(kTile, it.t1 - (it.t0 + j * kTile));
-                if constexpr (MMA) {
-                    const uint32_t ks = stage0 + s * L::kStage;
-                    math.tile(ks, ks + L::kHalf, n, p.scale_log2, lane);
-                } else {
-                    const uint8_t *ks = smem + (warp * SPW + s) * L::kStage;
-                    math.tile(ks, ks + L::kHalf, n, scores, lane);
-                }
-            }
-            if (consumed < issued)
-                ++consumed;
-            // the stage is free again: refill it with the job SPW ahead
-            __syncwarp();
-            ptx::fence_proxy_async_smem();
-            Item nit;
-            int nj;
-            if (!aborted && next_job(nit, nj)) {
-                issue(nit, nj, s);
-                ++issued;
+#pragma unroll
+        for (int bx = 0; bx < 4; ++bx) {
+            if (bx < geo.bpt && bx * geo.tr < d.n) {
+                if (d.phys[bx] < 0 || (int64_t)d.phys[bx] >= p.num_blocks)
+                    bad = true;
+                else
+                    tx += 2 * geo.box_tx;
             }
         }
-
-        // ---------------- merge the warps' partial softmax states
-        float *mrow = merge + warp * L::kMergeFloats;
-        math.finish(mrow, lane);
-        if (lane == 0)
-            mrow[G * D + 2 * G] = bad ? 1.f : 0.f;
-        __syncthreads();
-
-        bool anybad = false;
+        if (bad)
+            badmask |= 1u << s;
+        else
+            badmask &= ~(1u << s);
+        if (lane == 0) {
+            ptx::mbar_arrive_expect_tx(bar, (uint32_t)tx);
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w)
-            anybad |= merge[w * L::kMergeFloats + G * D + 2 * G] != 0.f;
-        if (threadIdx.x == 0) {
-            if (anybad)
-                report(p.dev_status, PA_DEV_BAD_BLOCK);
-            if (it.ctx_raw != it.ctx && it.part == 0 && it.h == 0)
-                report(p.dev_status, PA_DEV_BAD_CONTEXT);
-        }
-        const int nparts = num_parts(it.ctx, p.partition_size);
-        const bool write_final = nparts == 1;
-        const bool write_part = nparts > 1 || p.always_partials;
-        for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
-            const int gq = idx / D;
-            const int e = idx - gq * D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w)
-                M = fmaxf(M, merge[w * L::kMergeFloats + G * D + gq]);
-            float Lsum = 0.f, O = 0.f;
-            if (!anybad && M != -INFINITY) {
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) {
-                    const float *row = merge + w * L::kMergeFloats;
-                    const float mw = row[G * D + gq];
-                    if (mw != -INFINITY) {
-                        const float f = ptx::ex2(mw - M);
-                        Lsum = fmaf(row[G * D + G + gq], f, Lsum);
-                        O = fmaf(row[idx], f, O);
+            for (int bx = 0; bx < 4; ++bx) {
+                if (bx >= geo.bpt || bx * geo.tr >= d.n || d.phys[bx] < 0 ||
+                    (int64_t)d.phys[bx] >= p.num_blocks)
+                    continue;
+                const int row =
+                    d.phys[bx] * p.block_size + ((d.t0 + bx * geo.tr) & (p.block_size - 1));
+                for (int op = 0; op < geo.ops_per_box; ++op) {
+                    const uint32_t off = (uint32_t)(bx * geo.box_stride + op * geo.chunk_stride);
+                    if (geo.ops_per_box == 1) {
+                        ptx::tma_load_4d(stage + off, &tmap_k, 0, row, 0, d.h, bar, policy);
+                        ptx::tma_load_4d(stage + (uint32_t)geo.kv_bytes + off, &tmap_v, 0, row, 0,
+                                         d.h, bar, policy);
+                    } else {
+                        const int c0 = op * (128 / (int)sizeof(T));
+                        ptx::tma_load_3d(stage + off, &tmap_k, c0, d.h, row, bar, policy);
+                        ptx::tma_load_3d(stage + (uint32_t)geo.kv_bytes + off, &tmap_v, c0, d.h,
+                                         row, bar, policy);
                     }
                 }
             }
-            const float res = Lsum > 0.f ? O / Lsum : 0.f;
-            const int64_t bh = (int64_t)it.b * p.num_q_heads + (int64_t)it.h * G + gq;
-            if (write_final)
-                store_out<T>(static_cast<T *>(p.out) + bh * D + e, res);
-            if (write_part) {
-                const int64_t slot = bh * p.max_parts + it.part;
-                p.tmp_out[slot * D + e] = res;
-                if (e == 0) {
-                    const bool empty = anybad || Lsum <= 0.f;
-                    p.max_logits[slot] = empty ? -INFINITY : M / kLog2e;
-                    p.exp_sums[slot] = empty ? 0.f : Lsum;
-                }
+            if (newseg) {
+                const T *qsrc =
+                    static_cast<const T *>(p.q) + ((int64_t)d.b * Hq + (int64_t)d.h * G) * D;
+                ptx::bulk_g2s(stage + (uint32_t)geo.q_off, qsrc, (uint32_t)geo.q_bytes, bar);
             }
         }
-        __syncthreads();
+        __syncwarp();
+    };
+
+    for (; issued < R1 && issued - R0 < spw; ++issued)
+        issue(issued);
+
+    using Math =
+        typename std::conditional<MMA, MmaMath<D, G, TR16>, SimtMath<T, D, G, TR16>>::type;
+    Math math;
+    int segS = 0;          // global index of the current segment's first tile
+    bool seg_bad = false;
+
+    for (int i = R0; i < R1; ++i) {
+        const int k = i - R0;
+        const int s = k % spw;
+        const TileDesc d = shfl_desc(bat0, bat1, (k >> 5) & 1, k & 31);
+        bool ok = false;
+        if (i < issued) {
+            ok = ptx::mbar_wait_bounded(bar0 + 8u * s, (uint32_t)((k / spw) & 1), kWaitLimitNs);
+            if (!ok) {
+                aborted = true;
+                if (lane == 0)
+                    report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+            }
+        }
+        const bool newseg = d.j == 0 || i == R0;
+        const uint32_t kreg = stage0 + (uint32_t)(s * geo.stage_bytes);
+        const uint32_t vreg = kreg + (uint32_t)geo.kv_bytes;
+        const uint8_t *qslot = stage0_gen + s * geo.stage_bytes + geo.q_off;
+        if (newseg) {
+            segS = i - d.j;
+            seg_bad = false;
+            if constexpr (MMA)
+                math.begin(qslot, lane);
+            else
+                math.begin(qslot, lane, p.scale_log2);
+            if (p.mode == 0 && d.j == 0 && lane == 0)
+                p.seg_start[(int64_t)d.b * Hkv + d.h] = i;
+        }
+        if ((badmask >> s) & 1u)
+            seg_bad = true;
+        if (ok && !seg_bad) {
+            if (d.n < kTile) {
+                // rows past the sequence end hold whatever the pool has there:
+                // zero them in V (their weight is 0, but 0 * NaN is NaN)
+                constexpr int NCH = D * (int)sizeof(T) / 128;
+                const int lines = (kTile - d.n) * NCH;
+                for (int idx = lane; idx < lines * 8; idx += 32) {
+                    const int line = idx >> 3;
+                    const int t = d.n + line / NCH;
+                    const int ch = line % NCH;
+                    const uint32_t a = tile_addr<TR16>(vreg, t, ch * 8 + (idx & 7), geo);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0)
+                                 : "memory");
+                }
+                __syncwarp();
+            }
+            if constexpr (MMA)
+                math.tile(kreg, vreg, d.n, p.scale_log2, geo, lane);
+            else
+                math.tile(kreg, vreg, d.n, scores, geo, lane);
+        }
+
+        // ---- end of a segment (or of this warp's range)
+        if (d.j == d.ns - 1 || i == R1 - 1) {
+            math.finish();
+            const int segE = segS + d.ns;
+            const bool complete = segS >= R0 && segE <= R1;
+            if (seg_bad && lane == 0)
+                report(p.dev_status, PA_DEV_BAD_BLOCK);
+            const int64_t bh0 = (int64_t)d.b * Hq + (int64_t)d.h * G;
+            if (p.mode == 0 && !complete) {
+                const int slot = segS < R0 ? 2 * gw : 2 * gw + 1;
+                float *ps = p.wpart + (int64_t)slot * p.slot_floats;
+                math.for_each(
+                    lane, [&](int hh, int e, float v, float) { ps[hh * D + e] = v; },
+                    [&](int hh, float mm, float ll) {
+                        ps[G * D + hh] = mm;
+                        ps[G * D + G + hh] = ll;
+                    });
+                if (lane == 0)
+                    ps[G * D + 2 * G] = seg_bad ? 1.f : 0.f;
+            } else {
+                const bool single = num_parts(d.ctx, p.partition_size) == 1;
+                math.for_each(
+                    lane,
+                    [&](int hh, int e, float v, float ll) {
+                        const float res = (seg_bad || !(ll > 0.f)) ? 0.f : v / ll;
+                        if (p.public_partials)
+                            p.tmp_out[((bh0 + hh) * p.max_parts + d.part) * D + e] = res;
+                        if (single)
+                            store_out<T>(static_cast<T *>(p.out) + (bh0 + hh) * D + e, res);
+                    },
+                    [&](int hh, float mm, float ll) {
+                        if (p.public_partials) {
+                            const int64_t slot = (bh0 + hh) * p.max_parts + d.part;
+                            const bool empty = seg_bad || !(ll > 0.f);
+                            p.max_logits[slot] = empty ? -INFINITY : mm / kLog2e;
+                            p.exp_sums[slot] = empty ? 0.f : ll;
+                        }
+                    });
+            }
+        }
+
+        // ---- the stage is free: refill it with the tile spw ahead
+        __syncwarp();
+        ptx::fence_proxy_async_smem();
+        if (!aborted && issued < R1) {
+            issue(issued);
+            ++issued;
+        }
+        // batch k/32 is fully consumed once k % 32 == 31: prepare the next
+        if ((k & 31) == 31) {
+            if (filled & 1)
+                fill_batch(bat1, win, R0 + 32 * filled, R1, p, lane);
+            else
+                fill_batch(bat0, win, R0 + 32 * filled, R1, p, lane);
+            ++filled;
+        }
+    }
+    if (aborted) {
+        // let copies still in flight land before the CTA exits (bounded)
+        for (int i = max(R0, issued - spw); i < issued; ++i) {
+            const int k = i - R0;
+            ptx::mbar_wait_bounded(bar0 + 8u * (k % spw), (uint32_t)((k / spw) & 1), kWaitLimitNs);
+        }
     }
 }
 
 // =====================================================================
-// Split-K reduce: one CTA per (sequence, query head).
+// Merge of cut segments (mode 0): one CTA per (sequence, KV head).
+// Warp w's range starts at tile floor(w T / W); the pieces of segment
+// [S, S + nt) are in slot 2 wf + 1 of its first warp wf and slot 2 w of every
+// later warp w <= wl.
+// =====================================================================
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(128) merge_kernel(const MergeParams p)
+{
+    const int seg = blockIdx.x;
+    const int b = seg / p.num_kv_heads;
+    const int h = seg - b * p.num_kv_heads;
+    const int ctx = eff_ctx(p.context_lens[b], p.ctx_cap);
+    if (ctx <= 0)
+        return;   // the decode kernel wrote zeros
+    const int nt = ntiles(ctx);
+    const int S = p.seg_start[seg];
+    const int64_t tot = *p.total_tiles;
+    const int64_t NW = p.total_warps;
+    const int wf = (int)((((int64_t)S + 1) * NW - 1) / tot);
+    const int wl = (int)((((int64_t)S + nt) * NW - 1) / tot);
+    if (wf == wl)
+        return;   // finished inside one warp
+    // warps with an empty range (more warps than tiles) hold no piece
+    auto empty = [&](int w) { return (int64_t)w * tot / NW == ((int64_t)w + 1) * tot / NW; };
+    auto slot_of = [&](int w) { return w == wf ? 2 * w + 1 : 2 * w; };
+    bool bad = false;
+    for (int w = wf; w <= wl; ++w)
+        if (!empty(w))
+            bad |= p.wpart[(int64_t)slot_of(w) * p.slot_floats + G * D + 2 * G] != 0.f;
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int g = idx / D;
+        float M = -INFINITY;
+        for (int w = wf; w <= wl; ++w)
+            if (!empty(w))
+                M = fmaxf(M, p.wpart[(int64_t)slot_of(w) * p.slot_floats + G * D + g]);
+        float L = 0.f, O = 0.f;
+        if (!bad && M != -INFINITY) {
+            for (int w = wf; w <= wl; ++w) {
+                if (empty(w))
+                    continue;
+                const float *ps = p.wpart + (int64_t)slot_of(w) * p.slot_floats;
+                const float mw = ps[G * D + g];
+                if (mw != -INFINITY) {
+                    const float f = ptx::ex2(mw - M);
+                    L = fmaf(ps[G * D + G + g], f, L);
+                    O = fmaf(ps[idx], f, O);
+                }
+            }
+        }
+        const int64_t bh = (int64_t)b * p.num_q_heads + (int64_t)h * G + g;
+        store_out<T>(static_cast<T *>(p.out) + bh * D + (idx - g * D), L > 0.f ? O / L : 0.f);
+    }
+}
+
+// =====================================================================
+// Explicit split-K reduce: one CTA per (sequence, query head).
 // =====================================================================
 template <typename T>
 __global__ void __launch_bounds__(128) reduce_kernel(const ReduceParams p, int head_dim)

@@ -1,0 +1,144 @@
+// pa_launch.cuh -- host-side launch templates shared by the translation units
+// that instantiate the decode and merge kernels (one per dtype / math).
+#pragma once
+
+#include <mutex>
+
+#include "pa_kernels.cuh"
+
+namespace pa {
+
+struct DecodeLaunch {
+    DecodeParams p;
+    CUtensorMap tmap_k;
+    CUtensorMap tmap_v;
+    int head_dim;
+    int group;
+    bool tr16;          // block size >= 16: one 16-row box per tile
+    int smem_bytes;
+    cudaStream_t stream;
+};
+
+// Persistent grid capacity (SMs x resident CTAs) of kernel `fn` with
+// `smem_bytes` of dynamic shared memory on the current device; cached.
+inline pa_status grid_capacity(const void *fn, int smem_bytes, int *cap)
+{
+    struct Slot {
+        const void *fn;
+        int dev, smem, cap;
+    };
+    static std::mutex mu;
+    static Slot slots[512];
+    static int nslots = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return PA_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < nslots; ++i)
+            if (slots[i].fn == fn && slots[i].dev == dev && slots[i].smem == smem_bytes) {
+                *cap = slots[i].cap;
+                return PA_OK;
+            }
+    }
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) !=
+        cudaSuccess)
+        return PA_ERR_CUDA;
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem_bytes) !=
+        cudaSuccess)
+        return PA_ERR_CUDA;
+    if (per_sm < 1)
+        return PA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (nslots < 512)
+        slots[nslots++] = Slot{fn, dev, smem_bytes, sms * per_sm};
+    *cap = sms * per_sm;
+    return PA_OK;
+}
+
+// With launch == false, *grid receives the capacity; otherwise the kernel is
+// launched with min(*grid, capacity) CTAs and *grid receives that count.
+template <typename T, int D, int G, bool MMA, bool TR16>
+pa_status decode_one(DecodeLaunch &L, int *grid, bool launch)
+{
+    auto fn = &decode_kernel<T, D, G, MMA, TR16>;
+    int cap = 0;
+    pa_status st = grid_capacity(reinterpret_cast<const void *>(fn), L.smem_bytes, &cap);
+    if (st != PA_OK)
+        return st;
+    if (!launch) {
+        *grid = cap;
+        return PA_OK;
+    }
+    const int g = *grid < cap ? (*grid > 0 ? *grid : 1) : cap;
+    *grid = g;
+    fn<<<g, kThreads, L.smem_bytes, L.stream>>>(L.tmap_k, L.tmap_v, L.p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int D, int G, bool MMA>
+pa_status decode_tr(DecodeLaunch &L, int *grid, bool launch)
+{
+    return L.tr16 ? decode_one<T, D, G, MMA, true>(L, grid, launch)
+                  : decode_one<T, D, G, MMA, false>(L, grid, launch);
+}
+
+template <typename T, int D, bool MMA>
+pa_status decode_g(DecodeLaunch &L, int *grid, bool launch)
+{
+    switch (L.group) {
+    case 1: return decode_tr<T, D, 1, MMA>(L, grid, launch);
+    case 2: return decode_tr<T, D, 2, MMA>(L, grid, launch);
+    case 4: return decode_tr<T, D, 4, MMA>(L, grid, launch);
+    case 8: return decode_tr<T, D, 8, MMA>(L, grid, launch);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T, bool MMA>
+pa_status decode_dispatch(DecodeLaunch &L, int *grid, bool launch)
+{
+    switch (L.head_dim) {
+    case 64: return decode_g<T, 64, MMA>(L, grid, launch);
+    case 128: return decode_g<T, 128, MMA>(L, grid, launch);
+    case 256: return decode_g<T, 256, MMA>(L, grid, launch);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T, int D>
+pa_status merge_g(const MergeParams &m, int group, cudaStream_t s)
+{
+    const unsigned grid = (unsigned)(m.num_seqs * m.num_kv_heads);
+    switch (group) {
+    case 1: merge_kernel<T, D, 1><<<grid, 128, 0, s>>>(m); break;
+    case 2: merge_kernel<T, D, 2><<<grid, 128, 0, s>>>(m); break;
+    case 4: merge_kernel<T, D, 4><<<grid, 128, 0, s>>>(m); break;
+    case 8: merge_kernel<T, D, 8><<<grid, 128, 0, s>>>(m); break;
+    default: return PA_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T>
+pa_status merge_dispatch(const MergeParams &m, int head_dim, int group, cudaStream_t s)
+{
+    switch (head_dim) {
+    case 64: return merge_g<T, 64>(m, group, s);
+    case 128: return merge_g<T, 128>(m, group, s);
+    case 256: return merge_g<T, 256>(m, group, s);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+// Entry points of the instantiation units.
+pa_status decode_f32(DecodeLaunch &L, int *grid, bool launch);
+pa_status decode_bf16_mma(DecodeLaunch &L, int *grid, bool launch);
+pa_status decode_bf16_simt(DecodeLaunch &L, int *grid, bool launch);
+pa_status merge_f32(const MergeParams &m, int head_dim, int group, cudaStream_t s);
+pa_status merge_bf16(const MergeParams &m, int head_dim, int group, cudaStream_t s);
+
+}  // namespace pa

@@ -38,7 +38,7 @@ SIGNATURES = {
     "pa_reshape_and_cache": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _P, _P]),
     "pa_decode_attention": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F,
                                  _I, _P, _SZ, _P, _P]),
-    "pa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "pa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "pa_num_partitions": (_I, [_I, _I]),
     "pa_splitk_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "pa_decode_splitk": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I,
@@ -92,9 +92,10 @@ def launch_count() -> int:
     return int(lib.pa_launch_count())
 
 
-def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
-                              max_context_len: int) -> int:
-    return int(lib.pa_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len))
+def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int,
+                              head_dim: int, max_context_len: int) -> int:
+    return int(lib.pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                             max_context_len))
 
 
 def pa_num_partitions(max_context_len: int, partition_size: int) -> int:

@@ -50,7 +50,7 @@ def gpu_step(pa, q, key, value, k_pool, v_pool, tables, lens, slots, max_ctx, sc
     B, hq, d = q.shape
     ws = None
     if workspace == "preferred":
-        nbytes = pa.pa_decode_workspace_bytes(B, hq, d, max_ctx)
+        nbytes = pa.pa_decode_workspace_bytes(B, hq, k_pool.shape[2], d, max_ctx)
         if nbytes:
             ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
     elif workspace is not None:
