@@ -28,8 +28,9 @@ using pa::TileGeo;
 
 std::atomic<unsigned long long> g_launches{0};
 
-// Bound on decode warps used to size the stream-K workspace (256 SMs x 4).
-constexpr int kWorkspaceWarps = 1024;
+// Bound on decode CTAs used to size the stream-K workspace (one per SM, up
+// to 256 SMs).
+constexpr int kWorkspaceCtas = 256;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -112,18 +113,14 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 4-D maps (one TMA operation per box) unless the driver has refused one;
-// then 3-D maps with one operation per 128-byte column.
-std::atomic<int> g_four_d{1};
-
 struct MapKey {
     const void *base;
     int64_t rows;
-    int hkv, d, es, tr, four_d;
+    int hkv, d, es, tr, hpc;
     bool operator==(const MapKey &o) const
     {
         return base == o.base && rows == o.rows && hkv == o.hkv && d == o.d && es == o.es &&
-               tr == o.tr && four_d == o.four_d;
+               tr == o.tr && hpc == o.hpc;
     }
 };
 
@@ -136,14 +133,15 @@ std::mutex g_map_mu;
 MapEntry g_maps[128];
 int g_nmaps = 0, g_next_map = 0;
 
-// Tensor map over a pool [nb, bs, Hkv, d] whose box is `tr` token rows x d of
-// one head, 128-byte swizzled.  4-D: dims (128-byte column elements, token
-// row, column, head); 3-D: dims (d, head, token row).
+// Tensor map over a pool [nb, bs, Hkv, d] with dims (elements of a 128-byte
+// column, token row, column, head) -- the row stride precedes the column
+// stride, so a box lands in shared memory as [head][column][row] -- and a box
+// of `tr` token rows x d of `hpc` heads, 128-byte swizzled.
 bool encode_pool_map(CUtensorMap *out, const void *base, int64_t nb, int bs, int hkv, int d,
-                     pa_dtype dt, int tr, int four_d)
+                     pa_dtype dt, int tr, int hpc)
 {
     const int es = elem_size(dt);
-    const MapKey key{base, nb * bs, hkv, d, es, tr, four_d};
+    const MapKey key{base, nb * bs, hkv, d, es, tr, hpc};
     {
         std::lock_guard<std::mutex> lock(g_map_mu);
         for (int i = 0; i < g_nmaps; ++i)
@@ -161,24 +159,13 @@ bool encode_pool_map(CUtensorMap *out, const void *base, int64_t nb, int bs, int
     const cuuint64_t rowb = (cuuint64_t)d * es;
     const cuuint32_t nch = (cuuint32_t)(rowb / 128);
     alignas(64) CUtensorMap map;
-    CUresult r;
-    if (four_d) {
-        const cuuint64_t dims[4] = {epc, (cuuint64_t)(nb * bs), nch, (cuuint64_t)hkv};
-        const cuuint64_t strides[3] = {(cuuint64_t)hkv * rowb, 128, rowb};
-        const cuuint32_t box[4] = {epc, (cuuint32_t)tr, nch, 1};
-        const cuuint32_t estr[4] = {1, 1, 1, 1};
-        r = enc(&map, type, 4, const_cast<void *>(base), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    } else {
-        const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)(nb * bs)};
-        const cuuint64_t strides[2] = {rowb, (cuuint64_t)hkv * rowb};
-        const cuuint32_t box[3] = {epc, 1, (cuuint32_t)tr};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        r = enc(&map, type, 3, const_cast<void *>(base), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    }
+    const cuuint64_t dims[4] = {epc, (cuuint64_t)(nb * bs), nch, (cuuint64_t)hkv};
+    const cuuint64_t strides[3] = {(cuuint64_t)hkv * rowb, 128, rowb};
+    const cuuint32_t box[4] = {epc, (cuuint32_t)tr, nch, (cuuint32_t)hpc};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = enc(&map, type, 4, const_cast<void *>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return false;
     *out = map;
@@ -192,34 +179,31 @@ bool encode_pool_map(CUtensorMap *out, const void *base, int64_t nb, int bs, int
 // =====================================================================
 // Geometry and launch plumbing
 // =====================================================================
-bool make_geo(TileGeo &g, int D, int es, int bs, int group, int four_d, int *smem)
+// KV heads per CTA tile: the largest of 4, 2, 1 dividing Hkv.
+int heads_per_cta(int hkv) { return hkv % 4 == 0 ? 4 : (hkv % 2 == 0 ? 2 : 1); }
+
+bool make_geo(TileGeo &g, int D, int es, int bs, int group, int hpc, int *smem)
 {
     const int rowb = D * es;
     const int nch = rowb / 128;
     g.tr = std::min(16, bs);
     g.tr_log2 = ilog2_exact(g.tr);
     g.bpt = 16 / g.tr;
-    if (four_d) {
-        g.ops_per_box = 1;
-        g.chunk_stride = g.tr * 128;
-        g.box_stride = (int)round_up((int64_t)nch * g.chunk_stride, 1024);
-    } else {
-        g.ops_per_box = nch;
-        g.chunk_stride = (int)round_up((int64_t)g.tr * 128, 1024);
-        g.box_stride = nch * g.chunk_stride;
-    }
+    g.hpc = hpc;
+    g.head_lines = nch * g.tr;
+    g.box_stride = (int)round_up((int64_t)hpc * g.head_lines * 128, 1024);
     g.kv_bytes = g.bpt * g.box_stride;
-    g.q_bytes = group * D * es;
+    g.q_head_bytes = group * D * es;
+    g.q_bytes = hpc * g.q_head_bytes;
     g.q_off = 2 * g.kv_bytes;
     g.stage_bytes = (int)round_up((int64_t)g.q_off + g.q_bytes, 1024);
-    g.box_tx = g.tr * rowb;
+    g.box_tx = hpc * g.tr * rowb;
     const int fixed = pa::decode_smem_fixed(group);
-    const int spw =
-        std::min(pa::kMaxSpw, (pa::kSmemBudget - fixed) / (pa::kWarps * g.stage_bytes));
+    const int spw = std::min(pa::kMaxSpw, (pa::kSmemBudget - fixed) / g.stage_bytes);
     if (spw < 1)
         return false;
     g.spw = spw;
-    *smem = fixed + pa::kWarps * spw * g.stage_bytes;
+    *smem = fixed + spw * g.stage_bytes;
     return true;
 }
 
@@ -266,6 +250,8 @@ pa_status check_attention_args(const void *out, const void *query, const void *k
         return PA_ERR_INVALID_ARG;
     if (num_blocks > (int64_t)INT32_MAX / block_size)
         return PA_ERR_INVALID_ARG;   // token rows of the pool are int32 TMA coordinates
+    if ((int64_t)num_kv_heads > 256)
+        return PA_ERR_UNSUPPORTED;   // TMA tensor dims
     // every tile index of the batch must fit an int
     if ((int64_t)num_seqs * num_kv_heads * (round_up((int64_t)max_blocks * block_size, 16) / 16) >
         (int64_t)INT32_MAX / 2)
@@ -310,27 +296,27 @@ pa_status prepare_decode(DecodeLaunch &L, void *out, const void *query, const vo
     L.stream = static_cast<cudaStream_t>(stream);
     const int es = elem_size(dtype);
     const int tr = std::min(16, block_size);
-    for (;;) {
-        const int four_d = g_four_d.load();
-        if (!make_geo(p.geo, head_dim, es, block_size, group, four_d, &L.smem_bytes))
-            return PA_ERR_UNSUPPORTED;
-        const bool ok_k = encode_pool_map(&L.tmap_k, k_pool, num_blocks, block_size, num_kv_heads,
-                                          head_dim, dtype, tr, four_d);
-        const bool ok_v = ok_k && encode_pool_map(&L.tmap_v, v_pool, num_blocks, block_size,
-                                                  num_kv_heads, head_dim, dtype, tr, four_d);
-        if (ok_k && ok_v)
-            return PA_OK;
-        if (!four_d)
-            return PA_ERR_CUDA;
-        g_four_d.store(0);   // retry with 3-D maps
-    }
+    const int hpc = heads_per_cta(num_kv_heads);
+    p.head_groups = num_kv_heads / hpc;
+    if (!make_geo(p.geo, head_dim, es, block_size, group, hpc, &L.smem_bytes))
+        return PA_ERR_UNSUPPORTED;
+    if (!encode_pool_map(&L.tmap_k, k_pool, num_blocks, block_size, num_kv_heads, head_dim, dtype,
+                         tr, hpc) ||
+        !encode_pool_map(&L.tmap_v, v_pool, num_blocks, block_size, num_kv_heads, head_dim, dtype,
+                         tr, hpc))
+        return PA_ERR_CUDA;
+    return PA_OK;
 }
 
+// Stream-K workspace: two partial slots per CTA and head of the group, the
+// first tile of every (sequence, head group) segment, and the tile count.
 size_t stream_k_bytes(int64_t num_seqs, int64_t num_kv_heads, int64_t group, int64_t head_dim,
-                      int64_t warps)
+                      int64_t ctas)
 {
+    const int64_t hpc = heads_per_cta((int)num_kv_heads);
     const int64_t slot = round_up(group * head_dim + 2 * group + 1, 4);
-    return (size_t)(2 * warps * slot * 4 + round_up(num_seqs * num_kv_heads * 4, 16) + 16);
+    return (size_t)(2 * ctas * hpc * slot * 4 + round_up(num_seqs * (num_kv_heads / hpc) * 4, 16) +
+                    16);
 }
 
 pa_status launch_reduce(void *out, const float *tmp_out, const float *max_logits,
@@ -405,7 +391,7 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads
         num_q_heads % num_kv_heads != 0)
         return 0;
     return stream_k_bytes(num_seqs, num_kv_heads, num_q_heads / num_kv_heads, head_dim,
-                          kWorkspaceWarps);
+                          kWorkspaceCtas);
 }
 
 pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_pool, void *v_pool,
@@ -491,8 +477,8 @@ pa_status pa_decode_splitk(void *out, const void *query, const void *k_pool, con
     if (st != PA_OK)
         return st;
     const int64_t tiles_up =
-        (int64_t)num_seqs * num_kv_heads * (round_up(std::max(max_context_len, 1), 16) / 16);
-    grid = (int)std::min<int64_t>(grid, (tiles_up + pa::kWarps - 1) / pa::kWarps);
+        (int64_t)num_seqs * p.head_groups * (round_up(std::max(max_context_len, 1), 16) / 16);
+    grid = (int)std::min<int64_t>(grid, tiles_up);
     st = decode_call(L, dtype, &grid, true);
     ++g_launches;
     return st;
@@ -555,10 +541,9 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
     if (st != PA_OK)
         return st;
     const int64_t tiles_up =
-        (int64_t)num_seqs * num_kv_heads * (round_up(std::max(max_context_len, 1), 16) / 16);
-    grid = (int)std::min<int64_t>(grid, (tiles_up + pa::kWarps - 1) / pa::kWarps);
-    const int64_t warps = (int64_t)grid * pa::kWarps;
-    const size_t need = stream_k_bytes(num_seqs, num_kv_heads, group, head_dim, warps);
+        (int64_t)num_seqs * p.head_groups * (round_up(std::max(max_context_len, 1), 16) / 16);
+    grid = (int)std::min<int64_t>(grid, tiles_up);
+    const size_t need = stream_k_bytes(num_seqs, num_kv_heads, group, head_dim, grid);
     const bool stream_k = workspace != nullptr && workspace_bytes >= need && aligned16(workspace);
     pa::MergeParams mp;
     std::memset(&mp, 0, sizeof(mp));
@@ -566,8 +551,9 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
         p.mode = 0;
         p.slot_floats = (int)round_up((int64_t)group * head_dim + 2 * group + 1, 4);
         p.wpart = static_cast<float *>(workspace);
-        p.seg_start = reinterpret_cast<int32_t *>(p.wpart + 2 * warps * p.slot_floats);
-        p.total_tiles = p.seg_start + round_up((int64_t)num_seqs * num_kv_heads, 4);
+        p.seg_start =
+            reinterpret_cast<int32_t *>(p.wpart + 2 * (int64_t)grid * p.geo.hpc * p.slot_floats);
+        p.total_tiles = p.seg_start + round_up((int64_t)num_seqs * p.head_groups, 4);
         mp.out = out;
         mp.wpart = p.wpart;
         mp.seg_start = p.seg_start;
@@ -577,7 +563,8 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
         mp.num_q_heads = num_q_heads;
         mp.num_kv_heads = num_kv_heads;
         mp.ctx_cap = p.ctx_cap;
-        mp.total_warps = (int)warps;
+        mp.total_ctas = grid;
+        mp.hpc = p.geo.hpc;
         mp.slot_floats = p.slot_floats;
     } else {
         p.mode = 1;

@@ -1,24 +1,27 @@
 // pa_kernels.cuh -- sm_100a device code of the paged KV-cache decode library.
 //
-// decode_kernel (persistent; warps never wait for one another)
-//   Work is cut into tiles: 16 consecutive tokens of one (sequence, KV head),
-//   inside one context partition (the whole context unless the caller asks
-//   for fixed-size partitions).  All tiles of the batch form one global
-//   sequence ordered by sequence, partition, KV head, token.  A "segment" is
-//   the run of tiles of one (sequence, partition, KV head).  Every warp of the
-//   grid owns one contiguous range of that sequence:
+// decode_kernel (persistent, warp-specialised)
+//   Work is cut into CTA tiles: 16 consecutive tokens of one sequence for a
+//   group of `hpc` KV heads (hpc = min(Hkv, 4)), inside one context partition
+//   (the whole context unless the caller asks for fixed-size partitions).  All
+//   CTA tiles of the batch form one global sequence ordered by sequence,
+//   partition, head group, token.  A "segment" is the run of tiles of one
+//   (sequence, partition, head group).  Every CTA owns one contiguous range of
+//   that sequence:
 //     mode 0 (stream-K): equal ranges.  A segment cut by range boundaries
-//       leaves one partial softmax state per piece (at most two per warp),
-//       merged afterwards by merge_kernel.  Balanced for any mix of lengths.
-//     mode 1: ranges snapped to segment starts, so one warp finishes every
+//       leaves one partial softmax state per piece and head (at most two
+//       pieces per CTA), merged afterwards by merge_kernel.  Balanced for any
+//       mix of lengths.
+//     mode 1: ranges snapped to segment starts, so one CTA finishes every
 //       segment it starts (no partials; used without a workspace and for the
 //       explicit fixed-partition split-K API).
-//   Per warp, tiles stream into shared memory through TMA: one tensor-map box
-//   brings `tr` rows x d of K (or V) of one KV head, 128-byte swizzled,
-//   completing on the stage's mbarrier.  A warp keeps up to SPW tiles in
-//   flight and issues tile i + SPW once it has consumed tile i.  Block-table
-//   entries of the next 32 tiles are fetched in one lane-parallel batch ahead
-//   of use.  The query rows of a segment arrive with its first tile.
+//   A producer warp streams the CTA's tiles into a ring of SPW shared-memory
+//   stages: one TMA tensor-map box brings 16 token rows x d of all hpc heads of
+//   K (and one of V), 128-byte swizzled, completing on the stage's "full"
+//   mbarrier; block-table entries of the next 32 tiles are fetched in one
+//   lane-parallel batch ahead of use; the query rows of a segment come with
+//   its first tile.  Consumer warp h (one per head of the group) computes its
+//   head's share of each tile and arrives on the stage's "empty" mbarrier.
 //
 // Tile math (one policy per instantiation)
 //   MmaMath   bf16 tensor cores (mma.sync m16n8k16, fp32 accumulate):
@@ -44,43 +47,39 @@
 
 namespace pa {
 
-#ifndef PA_WARPS
-#define PA_WARPS 4
-#endif
 #ifndef PA_MAX_SPW
 #define PA_MAX_SPW 4
 #endif
 
-constexpr int kWarps = PA_WARPS;            // warps per CTA
-constexpr int kThreads = 32 * kWarps;
-constexpr int kMaxSpw = PA_MAX_SPW;         // tiles in flight per warp, at most
+constexpr int kMaxHpc = 4;                  // KV heads per CTA tile, at most
+constexpr int kThreads = 32 * (kMaxHpc + 1);// launch bound: consumers + producer
+constexpr int kMaxSpw = PA_MAX_SPW;         // stages in the ring, at most
 constexpr int kTile = 16;                   // tokens per tile (= MMA M and K)
 constexpr int kSmemBudget = 227 * 1024;     // opt-in dynamic shared memory per CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded copy waits: 2 s
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned kFull = 0xffffffffu;
 
-// Shared-memory geometry of one tile, fixed per launch (depends on the block
-// size).  A K (or V) region holds 16 token rows of one head as `bpt` boxes of
-// `tr` rows; a box is nch = d * elem / 128 columns of 128 bytes:
-//   byte(row r of box b, 16-byte unit u) = b*box_stride + (u/8)*chunk_stride
-//                                          + r*128 + ((u%8) ^ swz) * 16
-// where swz = bits 7..9 of the 128-byte line's offset (the TMA 128-byte
-// swizzle).  Boxes, and in 3-D mode every column, start on a 1024-byte
-// boundary.
+// Shared-memory geometry of one CTA tile, fixed per launch (depends on the
+// block size).  A K (or V) region holds 16 token rows of hpc heads as `bpt`
+// boxes of `tr` rows; a box is [head][128-byte column][row] with nch = d*elem/128
+// columns, i.e. 128-byte line L = (head * nch + column) * tr + row, and
+//   byte(box b, line L, 16-byte unit u) = b*box_stride + L*128 + ((u % 8) ^ (L % 8)) * 16
+// (the TMA 128-byte swizzle).  Boxes start on 1024-byte boundaries.
 struct TileGeo {
     int tr;            // rows per box = min(16, block_size)
     int tr_log2;
     int bpt;           // boxes per tile = 16 / tr
-    int ops_per_box;   // TMA operations per box: 1 (4-D map) or nch (3-D map)
-    int chunk_stride;  // bytes between the 128-byte columns of a box
+    int hpc;           // KV heads per CTA tile (= consumer warps)
+    int head_lines;    // 128-byte lines per head in a box = nch * tr
     int box_stride;    // bytes between boxes
     int kv_bytes;      // bytes of a K (or V) region
     int q_off;         // offset of the query slot in a stage
     int stage_bytes;   // K + V + query, multiple of 1024
-    int spw;           // stages per warp
+    int spw;           // stages in the ring
     int box_tx;        // bytes one box delivers
     int q_bytes;       // bytes of the query slot payload
+    int q_head_bytes;  // query bytes of one KV head (G * d * elem)
 };
 
 struct DecodeParams {
@@ -91,8 +90,8 @@ struct DecodeParams {
     float *tmp_out;          // explicit split-K layout [B, Hq, max_parts, d]
     float *max_logits;       // [B, Hq, max_parts]
     float *exp_sums;         // [B, Hq, max_parts]
-    float *wpart;            // mode 0: two partial slots per warp
-    int32_t *seg_start;      // mode 0: first global tile of each (b, h) segment
+    float *wpart;            // mode 0: two partial slots per CTA and head
+    int32_t *seg_start;      // mode 0: first global tile of each (b, head group) segment
     int32_t *total_tiles;    // mode 0: total tile count (written by the kernel)
     int32_t *dev_status;
     int64_t num_blocks;
@@ -108,6 +107,7 @@ struct DecodeParams {
     int mode;                // 0 stream-K, 1 whole segments
     int public_partials;     // mode 1: write tmp_out / max_logits / exp_sums
     int slot_floats;         // floats per partial slot (mode 0)
+    int head_groups;         // Hkv / hpc
     float scale_log2;
     TileGeo geo;
 };
@@ -135,7 +135,8 @@ struct MergeParams {
     int num_q_heads;
     int num_kv_heads;
     int ctx_cap;
-    int total_warps;
+    int total_ctas;
+    int hpc;
     int slot_floats;
 };
 
@@ -169,7 +170,7 @@ __device__ __forceinline__ int count_tiles(const DecodeParams &p, int lane)
     for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
         const int b = b0 + lane;
         if (b < p.num_seqs)
-            sum += ntiles(eff_ctx(p.context_lens[b], p.ctx_cap)) * p.num_kv_heads;
+            sum += ntiles(eff_ctx(p.context_lens[b], p.ctx_cap)) * p.head_groups;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
@@ -182,7 +183,7 @@ __device__ __forceinline__ int count_tiles(const DecodeParams &p, int lane)
 struct SeqWindow {
     int b0;      // first sequence of the window
     int base;    // global index of the first tile of sequence b0
-    int cnt;     // this lane's sequence: tiles (Hkv * ntiles)
+    int cnt;     // this lane's sequence: tiles (head groups * ntiles)
     int incl;    // inclusive prefix of cnt over the window
     int ctx;     // this lane's sequence: effective length
 };
@@ -194,7 +195,7 @@ __device__ __forceinline__ void window_load(SeqWindow &w, int b0, int base, cons
     w.base = base;
     const int b = b0 + lane;
     w.ctx = b < p.num_seqs ? eff_ctx(p.context_lens[b], p.ctx_cap) : 0;
-    w.cnt = ntiles(w.ctx) * p.num_kv_heads;
+    w.cnt = ntiles(w.ctx) * p.head_groups;
     int incl = w.cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -245,7 +246,8 @@ __device__ __forceinline__ void window_find(SeqWindow &w, int g, bool want, int 
     }
 }
 
-// Tile descriptor; a batch holds 32 consecutive tiles, one per lane.
+// Tile descriptor (h is the head group); a batch holds 32 consecutive tiles,
+// one per lane.
 struct TileDesc {
     int b, h, part, j, ns, t0, n, ctx;
     int phys[4];
@@ -292,15 +294,15 @@ __device__ __forceinline__ void fill_batch(TileDesc &d, SeqWindow &w, int base, 
         d.phys[k] = -1;
     if (!want)
         return;
-    const int Hkv = p.num_kv_heads;
+    const int HG = p.head_groups;
     const int nt = ntiles(ctx);
     const int PT = p.partition_size >> 4;             // tiles of a full partition
     const int x = g - seqbase;
     const int nparts = num_parts(ctx, p.partition_size);
-    int part = (int)((int64_t)x / ((int64_t)Hkv * PT));
+    int part = (int)((int64_t)x / ((int64_t)HG * PT));
     if (part > nparts - 1)
         part = nparts - 1;
-    const int rem = x - (int)((int64_t)part * Hkv * PT);
+    const int rem = x - (int)((int64_t)part * HG * PT);
     const int np = min(PT, nt - part * PT);             // tiles of this partition
     d.h = rem / np;
     d.j = rem - d.h * np;
@@ -340,29 +342,32 @@ __device__ __forceinline__ int range_begin(int gw, int total_warps, int T, const
 // =====================================================================
 // Swizzled addressing of a K or V region
 // =====================================================================
-// Address of 16-byte unit u of token row t in a region starting at `reg`.
-__device__ __forceinline__ uint32_t kv_addr(uint32_t reg, int t, int u, const TileGeo &g)
+// Address of 16-byte unit u of token row t of the head whose lines start at
+// line `hline` (= head * head_lines) in a region starting at `reg`.
+__device__ __forceinline__ uint32_t kv_addr(uint32_t reg, int hline, int t, int u, const TileGeo &g)
 {
     const int box = t >> g.tr_log2;
     const int r = t & (g.tr - 1);
-    const uint32_t line = (uint32_t)(box * g.box_stride + (u >> 3) * g.chunk_stride + r * 128);
-    return reg + line + ((((uint32_t)u & 7u) ^ ((line >> 7) & 7u)) << 4);
+    const uint32_t line = (uint32_t)(hline + (u >> 3) * g.tr + r);
+    return reg + (uint32_t)(box * g.box_stride) + line * 128u +
+           ((((uint32_t)u & 7u) ^ (line & 7u)) << 4);
 }
 
 // Same, for one 16-row box (block size >= 16): the swizzle phase is t & 7.
-__device__ __forceinline__ uint32_t kv_addr16(uint32_t reg, int t, int u)
+__device__ __forceinline__ uint32_t kv_addr16(uint32_t reg, int hline, int t, int u)
 {
-    return reg + (uint32_t)((u >> 3) * (kTile * 128) + t * 128) +
+    return reg + (uint32_t)((hline + (u >> 3) * kTile + t) * 128) +
            ((((uint32_t)u & 7u) ^ ((uint32_t)t & 7u)) << 4);
 }
 
 template <bool TR16>
-__device__ __forceinline__ uint32_t tile_addr(uint32_t reg, int t, int u, const TileGeo &g)
+__device__ __forceinline__ uint32_t tile_addr(uint32_t reg, int hline, int t, int u,
+                                              const TileGeo &g)
 {
     if constexpr (TR16)
-        return kv_addr16(reg, t, u);
+        return kv_addr16(reg, hline, t, u);
     else
-        return kv_addr(reg, t, u, g);
+        return kv_addr(reg, hline, t, u, g);
 }
 
 // =====================================================================
@@ -409,8 +414,8 @@ struct MmaMath {
         l[0] = l[1] = 0.f;
     }
 
-    __device__ __forceinline__ void tile(uint32_t ks, uint32_t vs, int n, float scale_log2,
-                                         const TileGeo &geo, int lane)
+    __device__ __forceinline__ void tile(uint32_t ks, uint32_t vs, int hline, int n,
+                                         float scale_log2, const TileGeo &geo, int lane)
     {
         const int r = lane >> 2;
         // ---- S = K Q^T (two accumulation chains)
@@ -419,7 +424,7 @@ struct MmaMath {
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
             uint32_t a[4];
-            ptx::ldsm_x4(tile_addr<TR16>(ks, krow, 2 * k + khalf, geo), a);
+            ptx::ldsm_x4(tile_addr<TR16>(ks, hline, krow, 2 * k + khalf, geo), a);
             if (k & 1)
                 ptx::mma_bf16_16816(sb, a, qf[k][0], qf[k][1]);
             else
@@ -472,7 +477,7 @@ struct MmaMath {
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
             uint32_t a[4];
-            ptx::ldsm_x4_trans(tile_addr<TR16>(vs, vrow, 2 * k + vhalf, geo), a);
+            ptx::ldsm_x4_trans(tile_addr<TR16>(vs, hline, vrow, 2 * k + vhalf, geo), a);
             ptx::mma_bf16_16816(acc[k], a, b0, b1);
         }
     }
@@ -582,8 +587,8 @@ struct SimtMath {
         }
     }
 
-    __device__ __forceinline__ void tile(uint32_t ks, uint32_t vs, int n, float *scores,
-                                         const TileGeo &geo, int lane)
+    __device__ __forceinline__ void tile(uint32_t ks, uint32_t vs, int hline, int n,
+                                         float *scores, const TileGeo &geo, int lane)
     {
         const int li = lane % LPR;
         const int rg = lane / LPR;
@@ -601,7 +606,7 @@ struct SimtMath {
 #pragma unroll
             for (int c = 0; c < UPL; ++c) {
                 float k[VEC];
-                cvt(lds128(tile_addr<TR16>(ks, r, c * LPR + li, geo)), k);
+                cvt(lds128(tile_addr<TR16>(ks, hline, r, c * LPR + li, geo)), k);
 #pragma unroll
                 for (int g = 0; g < G; ++g)
 #pragma unroll
@@ -651,7 +656,7 @@ struct SimtMath {
 #pragma unroll
                 for (int c = 0; c < UPL; ++c) {
                     float v[VEC];
-                    cvt(lds128(tile_addr<TR16>(vs, r, c * LPR + li, geo)), v);
+                    cvt(lds128(tile_addr<TR16>(vs, hline, r, c * LPR + li, geo)), v);
 #pragma unroll
                     for (int g = 0; g < G; ++g)
 #pragma unroll
@@ -701,14 +706,28 @@ struct SimtMath {
     }
 };
 
-// Bytes of the decode kernel's dynamic shared memory for a geometry.
+// Bytes of the decode kernel's dynamic shared memory besides the stages:
+// alignment slack, full and empty barriers, per-stage tile metadata, and the
+// CUDA-core math's score rows.
 __host__ __device__ constexpr int decode_smem_fixed(int G)
 {
-    return 1024 + 8 * kWarps * kMaxSpw + kWarps * kTile * G * 4;
+    return 1024 + 16 * kMaxSpw + 32 * kMaxSpw + kMaxHpc * kTile * G * 4;
 }
 
+// Tile metadata the producer warp hands to the consumer warps with a stage.
+struct StageMeta {
+    int b, hg, part, j, ns, n, ctx, bad;
+};
+
 // =====================================================================
-// Decode kernel
+// Decode kernel: hpc consumer warps (one per KV head of the group) and one
+// producer warp per CTA; launched with 32 * (hpc + 1) threads.
+//
+// CTA x owns the CTA-tile range [range_begin(x), range_begin(x + 1)).  The
+// stages form a ring; each has a "full" mbarrier (the producer arrives with
+// the expected bytes, TMA completes them) and an "empty" mbarrier (each
+// consumer warp arrives once it is done with the stage).  No warp waits on
+// another CTA, and every wait is bounded.
 // =====================================================================
 template <typename T, int D, int G, bool MMA, bool TR16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -720,131 +739,158 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x & 31;
     const TileGeo &geo = p.geo;
     const int spw = geo.spw;
-    const int gw = blockIdx.x * kWarps + warp;
-    const int total_warps = gridDim.x * kWarps;
-    const int Hkv = p.num_kv_heads;
+    const int hpc = geo.hpc;
+    const int total_ctas = gridDim.x;
+    const int HG = p.head_groups;
     const int Hq = p.num_q_heads;
 
-    // 1024-byte aligned layout: [stages][barriers][score rows]
+    // 1024-byte aligned layout: [stages][full bars][empty bars][meta][score rows]
     const uint32_t raw = ptx::smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     uint8_t *sgen = smem_raw + (sbase - raw);
-    const int stages_bytes = kWarps * spw * geo.stage_bytes;
-    const uint32_t stage0 = sbase + (uint32_t)(warp * spw * geo.stage_bytes);
-    const uint8_t *stage0_gen = sgen + warp * spw * geo.stage_bytes;
-    const uint32_t bar0 = sbase + (uint32_t)stages_bytes + 8u * (uint32_t)(warp * kMaxSpw);
-    float *scores = reinterpret_cast<float *>(sgen + stages_bytes + 8 * kWarps * kMaxSpw) +
-                    warp * kTile * G;
+    const int stages_bytes = spw * geo.stage_bytes;
+    const uint32_t full0 = sbase + (uint32_t)stages_bytes;
+    const uint32_t empty0 = full0 + 8u * kMaxSpw;
+    StageMeta *meta = reinterpret_cast<StageMeta *>(sgen + stages_bytes + 16 * kMaxSpw);
+    float *scores_all = reinterpret_cast<float *>(sgen + stages_bytes + 48 * kMaxSpw);
 
-    if (lane == 0) {
-        for (int s = 0; s < spw; ++s)
-            ptx::mbar_init(bar0 + 8u * s, 1);
-        ptx::prefetch_tensormap(&tmap_k);
-        ptx::prefetch_tensormap(&tmap_v);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < spw; ++s) {
+            ptx::mbar_init(full0 + 8u * s, 1);
+            ptx::mbar_init(empty0 + 8u * s, hpc);
+        }
     }
     ptx::fence_mbar_init();
-    __syncwarp();
+    __syncthreads();
 
     const int total = count_tiles(p, lane);
-    if (p.mode == 0 && gw == 0 && lane == 0)
-        *p.total_tiles = total;
+    const int R0 = range_begin(blockIdx.x, total_ctas, total, p, lane);
+    const int R1 = range_begin(blockIdx.x + 1, total_ctas, total, p, lane);
+
+    if (warp == hpc) {
+        // =================================================== producer warp
+        if (R0 >= R1)
+            return;
+        ptx::prefetch_tensormap(&tmap_k);
+        ptx::prefetch_tensormap(&tmap_v);
+        const uint64_t policy = ptx::policy_evict_first();
+        SeqWindow win;
+        window_load(win, 0, 0, p, lane);
+        TileDesc bat0, bat1;
+        fill_batch(bat0, win, R0, R1, p, lane);
+        fill_batch(bat1, win, R0 + 32, R1, p, lane);
+        int filled = 2;
+        int issued = R0;
+        for (; issued < R1; ++issued) {
+            const int i = issued;
+            const int k = i - R0;
+            const int s = k % spw;
+            const uint32_t bar = full0 + 8u * s;
+            if (k >= spw && !ptx::mbar_wait_bounded(empty0 + 8u * s,
+                                                    (uint32_t)(((k / spw) - 1) & 1), kWaitLimitNs)) {
+                if (lane == 0)
+                    report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+                break;
+            }
+            const TileDesc d = shfl_desc(bat0, bat1, (k >> 5) & 1, k & 31);
+            const bool newseg = d.j == 0 || i == R0;
+            int tx = newseg ? geo.q_bytes : 0;
+            bool bad = false;
+#pragma unroll
+            for (int bx = 0; bx < 4; ++bx) {
+                if (bx < geo.bpt && bx * geo.tr < d.n) {
+                    if (d.phys[bx] < 0 || (int64_t)d.phys[bx] >= p.num_blocks)
+                        bad = true;
+                    else
+                        tx += 2 * geo.box_tx;
+                }
+            }
+            const uint32_t stage = sbase + (uint32_t)(s * geo.stage_bytes);
+            if (lane == 0) {
+                StageMeta m;
+                m.b = d.b;
+                m.hg = d.h;
+                m.part = d.part;
+                m.j = d.j;
+                m.ns = d.ns;
+                m.n = d.n;
+                m.ctx = d.ctx;
+                m.bad = bad ? 1 : 0;
+                meta[s] = m;
+                // release: consumers see the metadata once the phase completes
+                ptx::mbar_arrive_expect_tx(bar, (uint32_t)tx);
+                const int h0 = d.h * hpc;
+#pragma unroll
+                for (int bx = 0; bx < 4; ++bx) {
+                    if (bx >= geo.bpt || bx * geo.tr >= d.n || d.phys[bx] < 0 ||
+                        (int64_t)d.phys[bx] >= p.num_blocks)
+                        continue;
+                    const int row =
+                        d.phys[bx] * p.block_size + ((d.t0 + bx * geo.tr) & (p.block_size - 1));
+                    const uint32_t off = (uint32_t)(bx * geo.box_stride);
+                    ptx::tma_load_4d(stage + off, &tmap_k, 0, row, 0, h0, bar, policy);
+                    ptx::tma_load_4d(stage + (uint32_t)geo.kv_bytes + off, &tmap_v, 0, row, 0, h0,
+                                     bar, policy);
+                }
+                if (newseg) {
+                    const T *qsrc =
+                        static_cast<const T *>(p.q) + ((int64_t)d.b * Hq + (int64_t)h0 * G) * D;
+                    ptx::bulk_g2s(stage + (uint32_t)geo.q_off, qsrc, (uint32_t)geo.q_bytes, bar);
+                }
+            }
+            __syncwarp();
+            // descriptors of batch k/32 are used up: prepare the batch after next
+            if ((k & 31) == 31) {
+                if (filled & 1)
+                    fill_batch(bat1, win, R0 + 32 * filled, R1, p, lane);
+                else
+                    fill_batch(bat0, win, R0 + 32 * filled, R1, p, lane);
+                ++filled;
+            }
+        }
+        if (issued < R1) {
+            // aborted: let copies still in flight land before exiting (bounded)
+            for (int i = max(R0, issued - spw); i < issued; ++i) {
+                const int k = i - R0;
+                ptx::mbar_wait_bounded(full0 + 8u * (k % spw), (uint32_t)((k / spw) & 1),
+                                       kWaitLimitNs);
+            }
+        }
+        return;
+    }
+
+    // ====================================================== consumer warps
+    const int hl = warp;                        // head within the group
+    const int hline = hl * geo.head_lines;      // its first 128-byte line in a box
+    float *scores = scores_all + hl * kTile * G;
 
     // Sequences without tiles (length 0 or invalid) get a zero output.
-    for (int b = gw; b < p.num_seqs; b += total_warps) {
+    for (int b = blockIdx.x; b < p.num_seqs; b += total_ctas) {
         const int rawc = p.context_lens[b];
         if (eff_ctx(rawc, p.ctx_cap) > 0)
             continue;
-        if (rawc != 0 && lane == 0)
+        if (rawc != 0 && lane == 0 && hl == 0)
             report(p.dev_status, PA_DEV_BAD_CONTEXT);
-        T *o = static_cast<T *>(p.out) + (int64_t)b * Hq * D;
-        for (int i = lane; i < Hq * D; i += 32)
-            store_out<T>(o + i, 0.f);
-        if (p.public_partials) {
-            for (int hq = 0; hq < Hq; ++hq) {
-                const int64_t slot = ((int64_t)b * Hq + hq) * p.max_parts;
-                for (int e = lane; e < D; e += 32)
-                    p.tmp_out[slot * D + e] = 0.f;
-                if (lane == 0) {
-                    p.max_logits[slot] = -INFINITY;
-                    p.exp_sums[slot] = 0.f;
+        for (int hg = 0; hg < HG; ++hg) {
+            const int64_t bh0 = (int64_t)b * Hq + (int64_t)(hg * hpc + hl) * G;
+            T *o = static_cast<T *>(p.out) + bh0 * D;
+            for (int i = lane; i < G * D; i += 32)
+                store_out<T>(o + i, 0.f);
+            if (p.public_partials) {
+                for (int g = 0; g < G; ++g) {
+                    const int64_t slot = (bh0 + g) * p.max_parts;
+                    for (int e = lane; e < D; e += 32)
+                        p.tmp_out[slot * D + e] = 0.f;
+                    if (lane == 0) {
+                        p.max_logits[slot] = -INFINITY;
+                        p.exp_sums[slot] = 0.f;
+                    }
                 }
             }
         }
     }
-
-    const int R0 = range_begin(gw, total_warps, total, p, lane);
-    const int R1 = range_begin(gw + 1, total_warps, total, p, lane);
-    if (R0 >= R1)
-        return;
-
-    const uint64_t policy = ptx::policy_evict_first();
-    SeqWindow win;
-    window_load(win, 0, 0, p, lane);
-    TileDesc bat0, bat1;
-    fill_batch(bat0, win, R0, R1, p, lane);
-    fill_batch(bat1, win, R0 + 32, R1, p, lane);
-    int filled = 2;   // batches prepared so far
-
-    uint32_t badmask = 0;   // stage s holds a tile with a block id outside the pool
-    bool aborted = false;
-    int issued = R0;
-
-    auto issue = [&](int i) {
-        const int k = i - R0;
-        const int s = k % spw;
-        const TileDesc d = shfl_desc(bat0, bat1, (k >> 5) & 1, k & 31);
-        const bool newseg = d.j == 0 || i == R0;
-        const uint32_t stage = stage0 + (uint32_t)(s * geo.stage_bytes);
-        const uint32_t bar = bar0 + 8u * s;
-        int tx = newseg ? geo.q_bytes : 0;
-        bool bad = false;
-#pragma unroll
-        for (int bx = 0; bx < 4; ++bx) {
-            if (bx < geo.bpt && bx * geo.tr < d.n) {
-                if (d.phys[bx] < 0 || (int64_t)d.phys[bx] >= p.num_blocks)
-                    bad = true;
-                else
-                    tx += 2 * geo.box_tx;
-            }
-        }
-        if (bad)
-            badmask |= 1u << s;
-        else
-            badmask &= ~(1u << s);
-        if (lane == 0) {
-            ptx::mbar_arrive_expect_tx(bar, (uint32_t)tx);
-#pragma unroll
-            for (int bx = 0; bx < 4; ++bx) {
-                if (bx >= geo.bpt || bx * geo.tr >= d.n || d.phys[bx] < 0 ||
-                    (int64_t)d.phys[bx] >= p.num_blocks)
-                    continue;
-                const int row =
-                    d.phys[bx] * p.block_size + ((d.t0 + bx * geo.tr) & (p.block_size - 1));
-                for (int op = 0; op < geo.ops_per_box; ++op) {
-                    const uint32_t off = (uint32_t)(bx * geo.box_stride + op * geo.chunk_stride);
-                    if (geo.ops_per_box == 1) {
-                        ptx::tma_load_4d(stage + off, &tmap_k, 0, row, 0, d.h, bar, policy);
-                        ptx::tma_load_4d(stage + (uint32_t)geo.kv_bytes + off, &tmap_v, 0, row, 0,
-                                         d.h, bar, policy);
-                    } else {
-                        const int c0 = op * (128 / (int)sizeof(T));
-                        ptx::tma_load_3d(stage + off, &tmap_k, c0, d.h, row, bar, policy);
-                        ptx::tma_load_3d(stage + (uint32_t)geo.kv_bytes + off, &tmap_v, c0, d.h,
-                                         row, bar, policy);
-                    }
-                }
-            }
-            if (newseg) {
-                const T *qsrc =
-                    static_cast<const T *>(p.q) + ((int64_t)d.b * Hq + (int64_t)d.h * G) * D;
-                ptx::bulk_g2s(stage + (uint32_t)geo.q_off, qsrc, (uint32_t)geo.q_bytes, bar);
-            }
-        }
-        __syncwarp();
-    };
-
-    for (; issued < R1 && issued - R0 < spw; ++issued)
-        issue(issued);
+    if (p.mode == 0 && blockIdx.x == 0 && warp == 0 && lane == 0)
+        *p.total_tiles = total;
 
     using Math =
         typename std::conditional<MMA, MmaMath<D, G, TR16>, SimtMath<T, D, G, TR16>>::type;
@@ -855,20 +901,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = R0; i < R1; ++i) {
         const int k = i - R0;
         const int s = k % spw;
-        const TileDesc d = shfl_desc(bat0, bat1, (k >> 5) & 1, k & 31);
-        bool ok = false;
-        if (i < issued) {
-            ok = ptx::mbar_wait_bounded(bar0 + 8u * s, (uint32_t)((k / spw) & 1), kWaitLimitNs);
-            if (!ok) {
-                aborted = true;
-                if (lane == 0)
-                    report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
-            }
+        if (!ptx::mbar_wait_bounded(full0 + 8u * s, (uint32_t)((k / spw) & 1), kWaitLimitNs)) {
+            if (lane == 0)
+                report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+            break;
         }
+        const StageMeta d = meta[s];
         const bool newseg = d.j == 0 || i == R0;
-        const uint32_t kreg = stage0 + (uint32_t)(s * geo.stage_bytes);
+        const uint32_t kreg = sbase + (uint32_t)(s * geo.stage_bytes);
         const uint32_t vreg = kreg + (uint32_t)geo.kv_bytes;
-        const uint8_t *qslot = stage0_gen + s * geo.stage_bytes + geo.q_off;
+        const uint8_t *qslot = sgen + s * geo.stage_bytes + geo.q_off + hl * geo.q_head_bytes;
         if (newseg) {
             segS = i - d.j;
             seg_bad = false;
@@ -876,43 +918,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                 math.begin(qslot, lane);
             else
                 math.begin(qslot, lane, p.scale_log2);
-            if (p.mode == 0 && d.j == 0 && lane == 0)
-                p.seg_start[(int64_t)d.b * Hkv + d.h] = i;
+            if (p.mode == 0 && d.j == 0 && hl == 0 && lane == 0)
+                p.seg_start[(int64_t)d.b * HG + d.hg] = i;
         }
-        if ((badmask >> s) & 1u)
+        if (d.bad)
             seg_bad = true;
-        if (ok && !seg_bad) {
+        if (!seg_bad) {
             if (d.n < kTile) {
                 // rows past the sequence end hold whatever the pool has there:
-                // zero them in V (their weight is 0, but 0 * NaN is NaN)
+                // zero them in this head's V (their weight is 0, but 0 * NaN is NaN)
                 constexpr int NCH = D * (int)sizeof(T) / 128;
                 const int lines = (kTile - d.n) * NCH;
                 for (int idx = lane; idx < lines * 8; idx += 32) {
                     const int line = idx >> 3;
                     const int t = d.n + line / NCH;
                     const int ch = line % NCH;
-                    const uint32_t a = tile_addr<TR16>(vreg, t, ch * 8 + (idx & 7), geo);
+                    const uint32_t a = tile_addr<TR16>(vreg, hline, t, ch * 8 + (idx & 7), geo);
                     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0)
                                  : "memory");
                 }
                 __syncwarp();
             }
             if constexpr (MMA)
-                math.tile(kreg, vreg, d.n, p.scale_log2, geo, lane);
+                math.tile(kreg, vreg, hline, d.n, p.scale_log2, geo, lane);
             else
-                math.tile(kreg, vreg, d.n, scores, geo, lane);
+                math.tile(kreg, vreg, hline, d.n, scores, geo, lane);
         }
+        // the stage may be refilled: order this warp's shared-memory accesses
+        // before the producer's next TMA into it, then release it
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0)
+            ptx::mbar_arrive(empty0 + 8u * s);
 
-        // ---- end of a segment (or of this warp's range)
+        // ---- end of a segment (or of this CTA's range)
         if (d.j == d.ns - 1 || i == R1 - 1) {
             math.finish();
             const int segE = segS + d.ns;
             const bool complete = segS >= R0 && segE <= R1;
             if (seg_bad && lane == 0)
                 report(p.dev_status, PA_DEV_BAD_BLOCK);
-            const int64_t bh0 = (int64_t)d.b * Hq + (int64_t)d.h * G;
+            const int64_t bh0 = (int64_t)d.b * Hq + (int64_t)(d.hg * hpc + hl) * G;
             if (p.mode == 0 && !complete) {
-                const int slot = segS < R0 ? 2 * gw : 2 * gw + 1;
+                const int slot = ((segS < R0 ? 2 * blockIdx.x : 2 * blockIdx.x + 1) * hpc) + hl;
                 float *ps = p.wpart + (int64_t)slot * p.slot_floats;
                 math.for_each(
                     lane, [&](int hh, int e, float v, float) { ps[hh * D + e] = v; },
@@ -943,84 +991,132 @@ __global__ void __launch_bounds__(kThreads, 1)
                     });
             }
         }
-
-        // ---- the stage is free: refill it with the tile spw ahead
-        __syncwarp();
-        ptx::fence_proxy_async_smem();
-        if (!aborted && issued < R1) {
-            issue(issued);
-            ++issued;
-        }
-        // batch k/32 is fully consumed once k % 32 == 31: prepare the next
-        if ((k & 31) == 31) {
-            if (filled & 1)
-                fill_batch(bat1, win, R0 + 32 * filled, R1, p, lane);
-            else
-                fill_batch(bat0, win, R0 + 32 * filled, R1, p, lane);
-            ++filled;
-        }
-    }
-    if (aborted) {
-        // let copies still in flight land before the CTA exits (bounded)
-        for (int i = max(R0, issued - spw); i < issued; ++i) {
-            const int k = i - R0;
-            ptx::mbar_wait_bounded(bar0 + 8u * (k % spw), (uint32_t)((k / spw) & 1), kWaitLimitNs);
-        }
     }
 }
 
 // =====================================================================
-// Merge of cut segments (mode 0): one CTA per (sequence, KV head).
-// Warp w's range starts at tile floor(w T / W); the pieces of segment
-// [S, S + nt) are in slot 2 wf + 1 of its first warp wf and slot 2 w of every
-// later warp w <= wl.
+// Merge of cut segments (mode 0): one CTA of merge_warps() warps per
+// (sequence, KV head).  CTA x's range starts at tile floor(x T / C); the pieces
+// of segment [S, S + nt) are in slot pair 2 xf + 1 of its first CTA xf and
+// slot pair 2 x of every later non-empty CTA x <= xl (slot = pair * hpc +
+// head within the group).  Each warp of this CTA accumulates a strided subset
+// of the pieces for all G*D outputs (independent loads, so the latency is a
+// few round trips whatever the piece count); the warps' sums are then added
+// in shared memory.
 // =====================================================================
+template <int G, int D>
+__host__ __device__ constexpr int merge_warps() { return G * D <= 1024 ? 8 : 4; }
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(128) merge_kernel(const MergeParams p)
+__global__ void __launch_bounds__(32 * merge_warps<G, D>()) merge_kernel(const MergeParams p)
 {
+    constexpr int kMergeWarps = merge_warps<G, D>();
+    __shared__ float s_max[G];
+    __shared__ float s_l[kMergeWarps][G];
+    __shared__ float s_o[kMergeWarps][G * D];
+    __shared__ int s_bad;
     const int seg = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = seg / p.num_kv_heads;
     const int h = seg - b * p.num_kv_heads;
+    const int hg = h / p.hpc, hl = h - hg * p.hpc;
     const int ctx = eff_ctx(p.context_lens[b], p.ctx_cap);
     if (ctx <= 0)
         return;   // the decode kernel wrote zeros
     const int nt = ntiles(ctx);
-    const int S = p.seg_start[seg];
+    const int S = p.seg_start[(int64_t)b * (p.num_kv_heads / p.hpc) + hg];
     const int64_t tot = *p.total_tiles;
-    const int64_t NW = p.total_warps;
+    const int64_t NW = p.total_ctas;
     const int wf = (int)((((int64_t)S + 1) * NW - 1) / tot);
     const int wl = (int)((((int64_t)S + nt) * NW - 1) / tot);
     if (wf == wl)
-        return;   // finished inside one warp
-    // warps with an empty range (more warps than tiles) hold no piece
+        return;   // finished inside one CTA
+    // CTAs with an empty range (more CTAs than tiles) hold no piece
     auto empty = [&](int w) { return (int64_t)w * tot / NW == ((int64_t)w + 1) * tot / NW; };
-    auto slot_of = [&](int w) { return w == wf ? 2 * w + 1 : 2 * w; };
-    bool bad = false;
-    for (int w = wf; w <= wl; ++w)
-        if (!empty(w))
-            bad |= p.wpart[(int64_t)slot_of(w) * p.slot_floats + G * D + 2 * G] != 0.f;
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int g = idx / D;
-        float M = -INFINITY;
-        for (int w = wf; w <= wl; ++w)
-            if (!empty(w))
-                M = fmaxf(M, p.wpart[(int64_t)slot_of(w) * p.slot_floats + G * D + g]);
-        float L = 0.f, O = 0.f;
-        if (!bad && M != -INFINITY) {
-            for (int w = wf; w <= wl; ++w) {
-                if (empty(w))
-                    continue;
-                const float *ps = p.wpart + (int64_t)slot_of(w) * p.slot_floats;
-                const float mw = ps[G * D + g];
-                if (mw != -INFINITY) {
-                    const float f = ptx::ex2(mw - M);
-                    L = fmaf(ps[G * D + G + g], f, L);
-                    O = fmaf(ps[idx], f, O);
+    auto slot_of = [&](int w) { return (w == wf ? 2 * w + 1 : 2 * w) * p.hpc + hl; };
+    const int npieces = wl - wf + 1;
+
+    // pass 1: maxima and the bad flag
+    if (threadIdx.x < G)
+        s_max[threadIdx.x] = -INFINITY;
+    if (threadIdx.x == 0)
+        s_bad = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < npieces; i += blockDim.x) {
+        const int w = wf + i;
+        if (empty(w))
+            continue;
+        const float *ps = p.wpart + (int64_t)slot_of(w) * p.slot_floats;
+        if (ps[G * D + 2 * G] != 0.f)
+            atomicOr(&s_bad, 1);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float mw = ps[G * D + g];
+            // float max through the int ordering of non-negative / negative halves
+            if (mw > -INFINITY) {
+                float cur = s_max[g];
+                while (mw > cur) {
+                    const int old = atomicCAS(reinterpret_cast<int *>(&s_max[g]), __float_as_int(cur),
+                                              __float_as_int(mw));
+                    if (old == __float_as_int(cur))
+                        break;
+                    cur = __int_as_float(old);
                 }
             }
         }
+    }
+    __syncthreads();
+    const bool bad = s_bad != 0;
+
+    // pass 2: warp `warp` sums pieces warp, warp + kMergeWarps, ...
+    float o[G * D / 32];
+    float lsum[G];
+#pragma unroll
+    for (int i = 0; i < G * D / 32; ++i)
+        o[i] = 0.f;
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+        lsum[g] = 0.f;
+    if (!bad) {
+        for (int i = warp; i < npieces; i += kMergeWarps) {
+            const int w = wf + i;
+            if (empty(w))
+                continue;
+            const float *ps = p.wpart + (int64_t)slot_of(w) * p.slot_floats;
+            float f[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float mw = ps[G * D + g];
+                f[g] = (mw == -INFINITY || s_max[g] == -INFINITY) ? 0.f : ptx::ex2(mw - s_max[g]);
+                lsum[g] = fmaf(ps[G * D + G + g], f[g], lsum[g]);
+            }
+#pragma unroll
+            for (int i2 = 0; i2 < G * D / 32; ++i2) {
+                const int idx = i2 * 32 + lane;
+                o[i2] = fmaf(ps[idx], f[idx / D], o[i2]);
+            }
+        }
+    }
+#pragma unroll
+    for (int i2 = 0; i2 < G * D / 32; ++i2)
+        s_o[warp][i2 * 32 + lane] = o[i2];
+    if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            s_l[warp][g] = lsum[g];
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int g = idx / D;
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMergeWarps; ++w) {
+            L += s_l[w][g];
+            O += s_o[w][idx];
+        }
         const int64_t bh = (int64_t)b * p.num_q_heads + (int64_t)h * G + g;
-        store_out<T>(static_cast<T *>(p.out) + bh * D + (idx - g * D), L > 0.f ? O / L : 0.f);
+        store_out<T>(static_cast<T *>(p.out) + bh * D + (idx - g * D),
+                     (!bad && L > 0.f) ? O / L : 0.f);
     }
 }
 

@@ -21,11 +21,11 @@ struct DecodeLaunch {
 
 // Persistent grid capacity (SMs x resident CTAs) of kernel `fn` with
 // `smem_bytes` of dynamic shared memory on the current device; cached.
-inline pa_status grid_capacity(const void *fn, int smem_bytes, int *cap)
+inline pa_status grid_capacity(const void *fn, int threads, int smem_bytes, int *cap)
 {
     struct Slot {
         const void *fn;
-        int dev, smem, cap;
+        int dev, threads, smem, cap;
     };
     static std::mutex mu;
     static Slot slots[512];
@@ -36,7 +36,8 @@ inline pa_status grid_capacity(const void *fn, int smem_bytes, int *cap)
     {
         std::lock_guard<std::mutex> lock(mu);
         for (int i = 0; i < nslots; ++i)
-            if (slots[i].fn == fn && slots[i].dev == dev && slots[i].smem == smem_bytes) {
+            if (slots[i].fn == fn && slots[i].dev == dev && slots[i].threads == threads &&
+                slots[i].smem == smem_bytes) {
                 *cap = slots[i].cap;
                 return PA_OK;
             }
@@ -47,14 +48,14 @@ inline pa_status grid_capacity(const void *fn, int smem_bytes, int *cap)
     int sms = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return PA_ERR_CUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem_bytes) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem_bytes) !=
         cudaSuccess)
         return PA_ERR_CUDA;
     if (per_sm < 1)
         return PA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(mu);
     if (nslots < 512)
-        slots[nslots++] = Slot{fn, dev, smem_bytes, sms * per_sm};
+        slots[nslots++] = Slot{fn, dev, threads, smem_bytes, sms * per_sm};
     *cap = sms * per_sm;
     return PA_OK;
 }
@@ -65,8 +66,9 @@ template <typename T, int D, int G, bool MMA, bool TR16>
 pa_status decode_one(DecodeLaunch &L, int *grid, bool launch)
 {
     auto fn = &decode_kernel<T, D, G, MMA, TR16>;
+    const int threads = 32 * (L.p.geo.hpc + 1);
     int cap = 0;
-    pa_status st = grid_capacity(reinterpret_cast<const void *>(fn), L.smem_bytes, &cap);
+    pa_status st = grid_capacity(reinterpret_cast<const void *>(fn), threads, L.smem_bytes, &cap);
     if (st != PA_OK)
         return st;
     if (!launch) {
@@ -75,7 +77,7 @@ pa_status decode_one(DecodeLaunch &L, int *grid, bool launch)
     }
     const int g = *grid < cap ? (*grid > 0 ? *grid : 1) : cap;
     *grid = g;
-    fn<<<g, kThreads, L.smem_bytes, L.stream>>>(L.tmap_k, L.tmap_v, L.p);
+    fn<<<g, threads, L.smem_bytes, L.stream>>>(L.tmap_k, L.tmap_v, L.p);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -114,10 +116,10 @@ pa_status merge_g(const MergeParams &m, int group, cudaStream_t s)
 {
     const unsigned grid = (unsigned)(m.num_seqs * m.num_kv_heads);
     switch (group) {
-    case 1: merge_kernel<T, D, 1><<<grid, 128, 0, s>>>(m); break;
-    case 2: merge_kernel<T, D, 2><<<grid, 128, 0, s>>>(m); break;
-    case 4: merge_kernel<T, D, 4><<<grid, 128, 0, s>>>(m); break;
-    case 8: merge_kernel<T, D, 8><<<grid, 128, 0, s>>>(m); break;
+    case 1: merge_kernel<T, D, 1><<<grid, 32 * merge_warps<1, D>(), 0, s>>>(m); break;
+    case 2: merge_kernel<T, D, 2><<<grid, 32 * merge_warps<2, D>(), 0, s>>>(m); break;
+    case 4: merge_kernel<T, D, 4><<<grid, 32 * merge_warps<4, D>(), 0, s>>>(m); break;
+    case 8: merge_kernel<T, D, 8><<<grid, 32 * merge_warps<8, D>(), 0, s>>>(m); break;
     default: return PA_ERR_UNSUPPORTED;
     }
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
