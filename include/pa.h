@@ -180,6 +180,42 @@ pa_status pa_splitk_reduce(void *out, const float *tmp_out, const float *max_log
                            int num_q_heads, int head_dim, int partition_size,
                            int max_partitions, pa_dtype dtype, void *stream);
 
+/*
+ * pa_decode_attention_static -- pa_decode_attention for callers that cannot
+ * allocate device memory.  The pages have no counterpart to this call; it is
+ * an addition of this library.
+ *
+ * Some callers can only hand a library their inputs and outputs: plug-in
+ * interfaces of inference engines that pass no workspace, callers whose
+ * device memory is owned by another framework, and code paths where an
+ * allocation (which may synchronise the device) is not allowed.  This call
+ * computes the same result as pa_decode_attention with a sufficient
+ * workspace, using instead a fixed scratch array of PA_STATIC_SCRATCH_BYTES
+ * that every device holds in device memory from the moment it loads the
+ * library until the process exits.  It never calls cudaMalloc, cudaFree or
+ * any allocating routine.
+ *
+ *   Arguments are those of pa_decode_attention without the workspace.
+ *   Returns PA_ERR_WORKSPACE, launching nothing, when these sizes need more
+ *   scratch than PA_STATIC_SCRATCH_BYTES (about 33 KB per SM for
+ *   Hq / Hkv = 4, d = 256, plus 4 bytes per sequence and group of KV heads).
+ *   The first call on a device looks up the array's device address (a CUDA
+ *   runtime query, no allocation); make that first call before any stream
+ *   capture.  All calls share the one array: calls whose kernels overlap on
+ *   the GPU (other streams, other threads) race and corrupt each other's
+ *   results, so serialise them.  The array keeps the last call's contents;
+ *   no word of it needs to start at zero (each call writes every word it
+ *   reads before reading it).
+ */
+#define PA_STATIC_SCRATCH_BYTES (8u << 20)
+pa_status pa_decode_attention_static(void *out, const void *query, const void *k_pool,
+                                     const void *v_pool, const int32_t *block_tables,
+                                     int max_blocks_per_seq, const int32_t *context_lens,
+                                     int num_seqs, int max_context_len, int num_q_heads,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int64_t num_blocks, float scale, pa_dtype dtype,
+                                     int32_t *dev_status, void *stream);
+
 /* Static description of a status code. */
 const char *pa_status_string(pa_status status);
 

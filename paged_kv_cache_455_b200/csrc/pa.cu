@@ -351,6 +351,70 @@ size_t splitk_bytes(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int
     return (size_t)(num_seqs * num_q_heads * parts * (head_dim + 2) * 4);
 }
 
+// =====================================================================
+// Scratch for pa_decode_attention_static: a fixed array in device memory,
+// allocated when the library is loaded on a device and held until exit.
+// Host code must not pass `g_static_scratch` to a kernel (on the host the
+// name is only a stand-in for the symbol); its device address comes from
+// cudaGetSymbolAddress, looked up once per device below.
+// =====================================================================
+static __device__ __align__(256) unsigned char g_static_scratch[PA_STATIC_SCRATCH_BYTES];
+
+std::mutex g_static_mu;
+void *g_static_addr[64] = {};
+
+// Device address of g_static_scratch on the current device (nullptr on error).
+void *static_scratch_address()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_addr[dev] == nullptr) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess)
+            return nullptr;
+        g_static_addr[dev] = ptr;
+    }
+    return g_static_addr[dev];
+}
+
+// Scratch bytes pa_decode_attention needs for its split over the current
+// device's grid (0 when these sizes run without one).
+pa_status stream_k_need(size_t *need, const void *out, const void *query, const void *k_pool,
+                        const void *v_pool, const int32_t *block_tables, int max_blocks_per_seq,
+                        const int32_t *context_lens, int num_seqs, int max_context_len,
+                        int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                        int64_t num_blocks, float scale, pa_dtype dtype)
+{
+    int group = 0, bs_log2 = 0;
+    pa_status st = check_attention_args(out, query, k_pool, v_pool, block_tables,
+                                        max_blocks_per_seq, context_lens, num_seqs,
+                                        max_context_len, num_q_heads, num_kv_heads, head_dim,
+                                        block_size, num_blocks, dtype, &group, &bs_log2);
+    if (st != PA_OK)
+        return st;
+    *need = 0;
+    if (num_seqs == 0)
+        return PA_OK;
+    DecodeLaunch L;
+    st = prepare_decode(L, const_cast<void *>(out), query, k_pool, v_pool, block_tables,
+                        max_blocks_per_seq, context_lens, num_seqs, num_q_heads, num_kv_heads,
+                        head_dim, block_size, bs_log2, num_blocks, scale, dtype, group, nullptr,
+                        nullptr);
+    if (st != PA_OK)
+        return st;
+    int grid = 0;
+    st = decode_call(L, dtype, &grid, false);
+    if (st != PA_OK)
+        return st;
+    const int64_t tiles_up = (int64_t)num_seqs * L.p.head_groups *
+                             (round_up(std::max(max_context_len, 1), 16) / 16);
+    grid = (int)std::min<int64_t>(grid, tiles_up);
+    *need = stream_k_bytes(num_seqs, num_kv_heads, group, head_dim, grid);
+    return PA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -580,6 +644,34 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
                                : pa::merge_bf16(mp, head_dim, group, L.stream);
     ++g_launches;
     return st;
+}
+
+pa_status pa_decode_attention_static(void *out, const void *query, const void *k_pool,
+                                     const void *v_pool, const int32_t *block_tables,
+                                     int max_blocks_per_seq, const int32_t *context_lens,
+                                     int num_seqs, int max_context_len, int num_q_heads,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int64_t num_blocks, float scale, pa_dtype dtype,
+                                     int32_t *dev_status, void *stream)
+{
+    size_t need = 0;
+    pa_status st = stream_k_need(&need, out, query, k_pool, v_pool, block_tables,
+                                 max_blocks_per_seq, context_lens, num_seqs, max_context_len,
+                                 num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                 scale, dtype);
+    if (st != PA_OK)
+        return st;
+    if (num_seqs == 0)
+        return PA_OK;
+    if (need > (size_t)PA_STATIC_SCRATCH_BYTES)
+        return PA_ERR_WORKSPACE;   // these sizes need more than the fixed scratch
+    void *scratch = static_scratch_address();
+    if (scratch == nullptr)
+        return PA_ERR_CUDA;
+    return pa_decode_attention(out, query, k_pool, v_pool, block_tables, max_blocks_per_seq,
+                               context_lens, num_seqs, max_context_len, num_q_heads, num_kv_heads,
+                               head_dim, block_size, num_blocks, scale, dtype, scratch,
+                               (size_t)PA_STATIC_SCRATCH_BYTES, dev_status, stream);
 }
 
 }  // extern "C"

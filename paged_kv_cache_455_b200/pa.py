@@ -44,6 +44,8 @@ SIGNATURES = {
     "pa_decode_splitk": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I,
                               _I, _I, _P, _P, _P, _P, _P]),
     "pa_splitk_reduce": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "pa_decode_attention_static": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                                        _I64, _F, _I, _P, _P]),
     "pa_status_string": (ctypes.c_char_p, [_I]),
     "pa_launch_count": (ctypes.c_ulonglong, []),
 }
@@ -159,6 +161,25 @@ def pa_decode_attention(out: torch.Tensor, query: torch.Tensor, k_pool: torch.Te
                                    _ptr(dev_status), _stream(stream)), "pa_decode_attention")
 
 
+PA_STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def pa_decode_attention_static(out: torch.Tensor, query: torch.Tensor, k_pool: torch.Tensor,
+                               v_pool: torch.Tensor, block_tables: torch.Tensor,
+                               context_lens: torch.Tensor, max_context_len: int, scale: float,
+                               dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """pa_decode_attention without a workspace: the library's fixed device
+    scratch array is used instead (for callers that cannot allocate)."""
+    B, hq, hkv, d, bs, nb, maxb = _attn_sizes(out, query, k_pool, v_pool, block_tables,
+                                              context_lens)
+    _cuda(dev_status)
+    _check(lib.pa_decode_attention_static(_ptr(out), _ptr(query), _ptr(k_pool), _ptr(v_pool),
+                                          _ptr(block_tables), maxb, _ptr(context_lens), B,
+                                          int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+                                          _dtype_code(query), _ptr(dev_status), _stream(stream)),
+           "pa_decode_attention_static")
+
+
 def pa_decode_splitk(out: torch.Tensor, query: torch.Tensor, k_pool: torch.Tensor,
                      v_pool: torch.Tensor, block_tables: torch.Tensor,
                      context_lens: torch.Tensor, max_context_len: int, scale: float,
@@ -198,6 +219,7 @@ def pa_splitk_reduce(out: torch.Tensor, tmp_out: torch.Tensor, max_logits: torch
 __all__ = [
     "lib", "LIB_PATH", "SIGNATURES", "PaError", "launch_count",
     "pa_reshape_and_cache", "pa_decode_attention", "pa_decode_workspace_bytes",
+    "pa_decode_attention_static", "PA_STATIC_SCRATCH_BYTES",
     "pa_num_partitions", "pa_splitk_workspace_bytes", "pa_decode_splitk", "pa_splitk_reduce",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA", "PA_ERR_WORKSPACE",
     "PA_DTYPE_F32", "PA_DTYPE_BF16",

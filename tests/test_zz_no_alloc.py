@@ -1,0 +1,84 @@
+"""pa_decode_attention_static: the entry point for callers that cannot
+allocate device memory (plug-in interfaces that pass only inputs and outputs,
+memory owned by another framework, code paths where an allocation is not
+allowed).  It must give the same result as pa_decode_attention with a
+workspace, through the C ABI, on consecutive calls that share its fixed
+scratch array.  This file is collected last on purpose."""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+TOL = 2e-2   # bf16 attention tolerance used by every GPU test
+
+
+def _case(seed, B, lens, hq=16, hkv=4, d=256, bs=16):
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens, np.int32)
+    need = -(-lens // bs)
+    nb = int(need.sum()) + 16
+    perm = rng.permutation(nb)
+    tables = np.full((B, int(need.max())), -1, np.int32)
+    pos = 0
+    for b in range(B):
+        tables[b, :need[b]] = perm[pos:pos + need[b]]
+        pos += need[b]
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    q = torch.randn(B, hq, d, generator=g, device=DEV).to(torch.bfloat16)
+    kp = torch.randn(nb, bs, hkv, d, generator=g, device=DEV).to(torch.bfloat16)
+    vp = torch.randn(nb, bs, hkv, d, generator=g, device=DEV).to(torch.bfloat16)
+    return (q, kp, vp, torch.from_numpy(tables).to(DEV), torch.from_numpy(lens).to(DEV),
+            int(lens.max()), d ** -0.5)
+
+
+def _with_workspace(pa, q, kp, vp, tab, lens, mc, scale):
+    out = torch.empty_like(q)
+    B, hq, d = q.shape
+    ws = torch.empty(pa.pa_decode_workspace_bytes(B, hq, kp.shape[2], d, mc), dtype=torch.uint8,
+                     device=DEV)
+    pa.pa_decode_attention(out, q, kp, vp, tab, lens, mc, scale, ws)
+    return out
+
+
+def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
+    from paged_kv_cache_455_b200 import pa
+    # long contexts so that sequences are spread over several CTAs and the
+    # scratch really holds partial results; the second batch differs, so it
+    # runs on the first call's leftover scratch contents
+    cases = [_case(11, 6, [3000, 1, 777, 4096, 1500, 2049]),
+             _case(12, 9, [5000, 64, 65, 1, 2500, 4100, 300, 3333, 17])]
+    for args in cases + cases[:1]:
+        ref = _with_workspace(pa, *args)
+        out = torch.full_like(ref, float("nan"))
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        q, kp, vp, tab, lens, mc, scale = args
+        pa.pa_decode_attention_static(out, q, kp, vp, tab, lens, mc, scale, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.isfinite(out.float()).all()
+        assert (out.float() - ref.float()).abs().max().item() <= TOL
+
+
+def test_static_scratch_rejects_sizes_beyond_its_maximum():
+    from paged_kv_cache_455_b200 import pa
+    # group 8, d = 256 over a batch of many sequences: the per-SM partials
+    # alone exceed the fixed scratch, so the call must refuse (and launch
+    # nothing) rather than fall back silently
+    B = 4096
+    q = torch.zeros(B, 32, 256, dtype=torch.bfloat16, device=DEV)
+    kp = torch.zeros(8, 16, 4, 256, dtype=torch.bfloat16, device=DEV)
+    tab = torch.zeros(B, 1, dtype=torch.int32, device=DEV)
+    lens = torch.ones(B, dtype=torch.int32, device=DEV)
+    # partials: two slots per CTA (one CTA per SM) and head of the 4-head
+    # group, each G*d + 2G + 1 floats rounded up to 4
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    slot = -(-(8 * 256 + 2 * 8 + 1) // 4) * 4
+    if 2 * sms * 4 * slot * 4 <= pa.PA_STATIC_SCRATCH_BYTES:
+        pytest.skip("this GPU's grid fits the scratch")
+    out = torch.zeros_like(q)
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode_attention_static(out, q, kp, kp, tab, lens, 16, 0.0625)
+    assert e.value.status == pa.PA_ERR_WORKSPACE
