@@ -149,13 +149,14 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 class Workload:
-    def __init__(self, cfg: W.DecodeConfig, device, shard: int, length_scale: float = 1.0):
+    def __init__(self, cfg: W.DecodeConfig, device, shard: int, length_scale: float = 1.0,
+                 layers=None):
         from paged_kv_cache_455_b200 import pa
         self.pa = pa
         self.cfg = cfg
         self.device = device
         self.layout = W.make_layout(cfg, length_scale=length_scale, shard=shard)
-        self.layers = W.make_layers(self.layout, device)
+        self.layers = W.make_layers(self.layout, device, layers=layers)
         self.tables, self.lens, self.slots = W.device_metadata(self.layout, device)
         L = self.layout
         nbytes = pa.pa_decode_workspace_bytes(cfg.num_seqs, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
@@ -164,22 +165,22 @@ class Workload:
         self.outs = [torch.empty_like(l.query) for l in self.layers]
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
-    def layer_step(self, i, tables=None, lens=None, slots=None, events=None):
+    def attention(self, i, tables=None, lens=None):
         pa, l, L = self.pa, self.layers[i], self.layout
-        tables = self.tables if tables is None else tables
-        lens = self.lens if lens is None else lens
-        slots = self.slots if slots is None else slots
-        pa.pa_reshape_and_cache(l.key, l.value, l.k_pool, l.v_pool, slots, self.status)
-        if events is not None:
-            events[0].record()
-        pa.pa_decode_attention(self.outs[i], l.query, l.k_pool, l.v_pool, tables, lens,
-                               L.max_context_len, self.cfg.scale, self.workspace, self.status)
-        if events is not None:
-            events[1].record()
+        pa.pa_decode_attention(self.outs[i], l.query, l.k_pool, l.v_pool,
+                               self.tables if tables is None else tables,
+                               self.lens if lens is None else lens, L.max_context_len,
+                               self.cfg.scale, self.workspace, self.status)
 
-    def step(self, attn_events=None):
+    def layer_step(self, i, tables=None, lens=None, slots=None):
+        l = self.layers[i]
+        self.pa.pa_reshape_and_cache(l.key, l.value, l.k_pool, l.v_pool,
+                                     self.slots if slots is None else slots, self.status)
+        self.attention(i, tables, lens)
+
+    def step(self):
         for i in range(len(self.layers)):
-            self.layer_step(i, events=None if attn_events is None else attn_events[i])
+            self.layer_step(i)
 
 
 def run_ours(args, rank, world, device, dist):
@@ -189,9 +190,9 @@ def run_ours(args, rank, world, device, dist):
     if cfg.name == "pressure":
         free, _ = torch.cuda.mem_get_info(device)
         length_scale = W.fit_length_scale(cfg, free)
-    wl = Workload(cfg, device, shard=rank, length_scale=length_scale)
+    wl = Workload(cfg, device, shard=rank, length_scale=length_scale, layers=args.layers)
     L = wl.layout
-    nl = cfg.layers
+    nl = len(wl.layers)
     bytes_layer = attention_bytes(L)
     torch.cuda.synchronize(device)
 
@@ -201,44 +202,72 @@ def run_ours(args, rank, world, device, dist):
     if int(wl.status.item()) != 0:
         raise RuntimeError(f"device status {int(wl.status.item())} during warm-up")
 
-    # ---- timed region: K steps, device events, clocks sampled meanwhile
+    # ---- one decode step (every layer: cache write then attention) and the
+    # attention calls alone, each captured once as a CUDA graph and replayed;
+    # the library launches on the current stream, which is the capture stream
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))
+    step_graph, attn_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        wl.step()
+        torch.cuda.synchronize(device)
+        l0 = pa.launch_count()
+        with torch.cuda.graph(step_graph, stream=side):
+            wl.step()
+        launches_per_step = pa.launch_count() - l0
+        with torch.cuda.graph(attn_graph, stream=side):
+            for i in range(nl):
+                wl.attention(i)
+    torch.cuda.synchronize(device)
+    for _ in range(2):
+        step_graph.replay()
+        attn_graph.replay()
+    torch.cuda.synchronize(device)
+
+    # ---- timed region: K replays of the step graph, device events, clocks
+    # sampled meanwhile
     stream = torch.cuda.current_stream(device)
-    attn_ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-                for _ in range(nl)] for _ in range(args.steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    launches0 = pa.launch_count()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(device)
     with ClockSampler(torch.cuda.current_device()) as clocks:
         t0.record(stream)
-        for k in range(args.steps):
-            wl.step(attn_ev[k])
+        for _ in range(args.steps):
+            step_graph.replay()
         t1.record(stream)
         torch.cuda.synchronize(device)
     if dist is not None:
         dist.barrier()
-    launches = pa.launch_count() - launches0
+    launches = launches_per_step * args.steps
     ms_total = t0.elapsed_time(t1)
-    attn_ms = [s.elapsed_time(e) for step in attn_ev for (s, e) in step]
-    attn_ms_mean = float(np.mean(attn_ms))
 
-    # max over ranks of the step time
-    ms_per_step = ms_total / args.steps
-    step_bytes_rank = bytes_layer * nl
-    seqs_rank = cfg.num_seqs
-    if dist is not None:
-        t = torch.tensor([ms_per_step, attn_ms_mean], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step, attn_ms_worst = float(t[0]), float(t[1])
-        tot = torch.tensor([float(step_bytes_rank), float(seqs_rank)], dtype=torch.float64,
-                           device=device)
-        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
-        step_bytes_all, seqs_all = float(tot[0]), float(tot[1])
-    else:
-        attn_ms_worst = attn_ms_mean
-        step_bytes_all, seqs_all = float(step_bytes_rank), float(seqs_rank)
+    # ---- attention alone (the roofline's kernel): K replays of the
+    # attention graph, events on the same stream
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        attn_graph.replay()
+    a1.record(stream)
+    torch.cuda.synchronize(device)
+    attn_ms_mean = a0.elapsed_time(a1) / (args.steps * nl)
+
+    # ---- the same step launched eagerly (host overhead included), for context
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(max(3, args.steps // 4)):
+        wl.step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    eager_ms = e0.elapsed_time(e1) / max(3, args.steps // 4)
+    del step_graph, attn_graph
+
+    # max over ranks of the step time, sum over ranks of the work
+    ms_per_step, attn_ms_worst, step_bytes_all, seqs_all = combine_ranks(
+        dist, device, ms_total / args.steps, attn_ms_mean, bytes_layer * nl, cfg.num_seqs)
     if int(wl.status.item()) != 0:
         raise RuntimeError(f"device status {int(wl.status.item())} in the timed region")
 
@@ -280,11 +309,13 @@ def run_ours(args, rank, world, device, dist):
         "pct_of_8tbs_per_gpu": round(100 * value / (NOMINAL_HBM_GBS * world), 2),
         "tokens_per_s_per_layer": round(tokens_per_s_layer, 1),
         "attention_only_gbs_per_gpu": round(achieved, 1),
+        "timing": "each step replays one CUDA graph of all layers (cache write + attention); "
+                  "eager launches of the same step take %.4f ms" % eager_ms,
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
             "peak_source": f"{peak_kind} HBM copy bandwidth",
             "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": "pa_decode_attention (decode_kernel + split-K reduce)",
+            "kernel": "pa_decode_attention (decode_kernel + merge_kernel), replayed in a graph",
             "algorithmic_bytes_per_launch": bytes_layer,
             "launch_ms_mean": round(attn_ms_mean, 5), "launch_ms_worst_rank": round(attn_ms_worst, 5),
         },
@@ -295,6 +326,18 @@ def run_ours(args, rank, world, device, dist):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg, L, wl.layers[0], budget_s=args.cpu_seconds)
     return out
+
+
+def combine_ranks(dist, device, ms_per_step, attn_ms, step_bytes, seqs):
+    """Maximum of the times and sum of the work over the ranks of `dist`
+    (no process group: the values as they are).  Every rank calls it."""
+    if dist is None:
+        return ms_per_step, attn_ms, float(step_bytes), float(seqs)
+    t = torch.tensor([ms_per_step, attn_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    w = torch.tensor([float(step_bytes), float(seqs)], dtype=torch.float64, device=device)
+    dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return float(t[0]), float(t[1]), float(w[0]), float(w[1])
 
 
 def run_e2e(wl: Workload, args, device, dist, world, bytes_layer):
@@ -343,7 +386,7 @@ def run_e2e(wl: Workload, args, device, dist, world, bytes_layer):
         t = torch.tensor([ms], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t[0])
-    value = world * bytes_layer * cfg.layers / (ms * 1e-3) / 1e9
+    value = world * bytes_layer * len(wl.layers) / (ms * 1e-3) / 1e9
     return {"value": round(value, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
@@ -448,13 +491,15 @@ def run_reference(args, rank, world, device):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="qwen", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers per step (default: the workload's 16); fewer only for profiling")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
