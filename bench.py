@@ -315,7 +315,7 @@ def run_ours(args, rank, world, device, dist):
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
             "peak_source": f"{peak_kind} HBM copy bandwidth",
             "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": "pa_decode_attention (decode_kernel + merge_kernel), replayed in a graph",
+            "kernel": "pa_decode_attention (decode_kernel, one launch per layer), replayed in a graph",
             "algorithmic_bytes_per_launch": bytes_layer,
             "launch_ms_mean": round(attn_ms_mean, 5), "launch_ms_worst_rank": round(attn_ms_worst, 5),
         },

@@ -37,6 +37,11 @@
  *     dev_status is not NULL), skips the offending access, and the affected
  *     output is zeros (attention) or left untouched (cache write).
  *   - Inputs and outputs must not overlap.
+ *   - Every call is asynchronous on `stream` and keeps stream order.  The
+ *     attention kernels are launched as programmatic dependents of the
+ *     kernel before them on the stream, so their set-up overlaps its tail;
+ *     they read and write no memory before that kernel has completed.  The
+ *     cache write lets the attention that follows start its set-up early.
  */
 #ifndef PA_H_
 #define PA_H_
@@ -110,14 +115,14 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_pool,
  *   scale          softmax scale (usually 1 / sqrt(d)).
  *   workspace      device scratch of workspace_bytes bytes (may be NULL / 0).
  *                  With at least pa_decode_workspace_bytes() bytes the work is
- *                  split evenly over the GPU's warps (each warp owns an equal
+ *                  split evenly over the GPU's SMs (each CTA owns an equal
  *                  share of the batch's 16-token tiles, whatever the lengths)
- *                  and the pieces of a sequence that straddles warps are
- *                  merged by a second kernel; with less, every (sequence, KV
- *                  head) is processed by one warp.  Both are exact to the
- *                  same tolerance.  Contents need no initialisation and are
- *                  garbage afterwards; calls sharing a workspace must not run
- *                  concurrently.
+ *                  and the pieces of a sequence that straddles CTAs are
+ *                  merged inside the kernel through the workspace; with less,
+ *                  every (sequence, group of KV heads) is processed by one
+ *                  CTA.  Both are exact to the same tolerance.  Contents need
+ *                  no initialisation and are garbage afterwards; calls
+ *                  sharing a workspace must not run concurrently.
  *   dev_status     device int32 or NULL (see PA_DEV_*).
  */
 pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
@@ -129,8 +134,9 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
                               int32_t *dev_status, void *stream);
 
 /* Workspace bytes pa_decode_attention wants for these sizes (enough for GPUs
- * of up to 256 SMs; about 8.5 MB for Hq/Hkv = 4, d = 256).  Host only;
- * touches no device.  max_context_len is accepted for symmetry and unused. */
+ * of up to 256 SMs; about 8.5 MB for Hkv = 4, Hq/Hkv = 4, d = 256).  Host
+ * only; touches no device.  num_seqs and max_context_len are accepted for
+ * symmetry and unused. */
 size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int max_context_len);
 
@@ -197,15 +203,17 @@ pa_status pa_splitk_reduce(void *out, const float *tmp_out, const float *max_log
  *
  *   Arguments are those of pa_decode_attention without the workspace.
  *   Returns PA_ERR_WORKSPACE, launching nothing, when these sizes need more
- *   scratch than PA_STATIC_SCRATCH_BYTES (about 33 KB per SM for
- *   Hq / Hkv = 4, d = 256, plus 4 bytes per sequence and group of KV heads).
+ *   scratch than PA_STATIC_SCRATCH_BYTES: about 33 KB per SM for
+ *   Hkv = 4, Hq / Hkv = 4, d = 256 (fits), 66 KB per SM for Hq / Hkv = 8,
+ *   d = 256 (refused on a 148-SM GPU).
  *   The first call on a device looks up the array's device address (a CUDA
  *   runtime query, no allocation); make that first call before any stream
  *   capture.  All calls share the one array: calls whose kernels overlap on
  *   the GPU (other streams, other threads) race and corrupt each other's
- *   results, so serialise them.  The array keeps the last call's contents;
- *   no word of it needs to start at zero (each call writes every word it
- *   reads before reading it).
+ *   results, so serialise them.  The array keeps the last call's contents
+ *   and no word of it needs to start at zero: a call reads a partial result
+ *   only after a flag word holds that call's own tag, which earlier calls
+ *   never wrote.
  */
 #define PA_STATIC_SCRATCH_BYTES (8u << 20)
 pa_status pa_decode_attention_static(void *out, const void *query, const void *k_pool,

@@ -1,13 +1,15 @@
 // pa.cu -- C ABI of the paged KV-cache decode library: argument checks,
 // shared-memory geometry, TMA tensor maps, work-decomposition choice and
-// launches.  Device code lives in pa_kernels.cuh; the decode / merge kernels
+// launches.  Device code lives in pa_kernels.cuh; the decode kernels
 // are instantiated in pa_inst_*.cu.
 //
 // pa_decode_attention uses the stream-K decomposition (mode 0) when the
-// caller's workspace holds the per-warp partials, and whole segments per warp
-// (mode 1) otherwise.  pa_decode_splitk runs mode 1 over fixed partitions.
+// caller's workspace holds the partial states of the cut segments, and whole
+// segments per CTA (mode 1) otherwise.  pa_decode_splitk runs mode 1 over
+// fixed partitions.
 #include <algorithm>
 #include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -64,6 +66,9 @@ struct CacheParams {
 
 __global__ void __launch_bounds__(256) cache_write_kernel(const CacheParams p)
 {
+    // the decode kernel that follows may start its set-up now; it waits for
+    // this grid to finish before reading the pools
+    pa::ptx::grid_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t nrows = (int64_t)p.num_tokens * p.num_kv_heads * 2;
@@ -308,15 +313,44 @@ pa_status prepare_decode(DecodeLaunch &L, void *out, const void *query, const vo
     return PA_OK;
 }
 
-// Stream-K workspace: two partial slots per CTA and head of the group, the
-// first tile of every (sequence, head group) segment, and the tile count.
+// Floats of one partial slot: acc [G][D], max [G], sum [G], bad mark.
+int64_t slot_floats(int64_t group, int64_t head_dim)
+{
+    return round_up(group * head_dim + 2 * group + 1, 4);
+}
+
+// Stream-K workspace: two partial slots per CTA and head of the group (a CTA
+// holds at most two pieces of cut segments: one met at the start of its
+// range, one running past its end) and one publication flag per slot.
 size_t stream_k_bytes(int64_t num_seqs, int64_t num_kv_heads, int64_t group, int64_t head_dim,
                       int64_t ctas)
 {
-    const int64_t hpc = heads_per_cta((int)num_kv_heads);
-    const int64_t slot = round_up(group * head_dim + 2 * group + 1, 4);
-    return (size_t)(2 * ctas * hpc * slot * 4 + round_up(num_seqs * (num_kv_heads / hpc) * 4, 16) +
-                    16);
+    (void)num_seqs;
+    const int64_t slots = 2 * ctas * heads_per_cta((int)num_kv_heads);
+    return (size_t)(slots * slot_floats(group, head_dim) * 4 + round_up(slots * 4, 16));
+}
+
+// Epoch of a stream-K call: the value its published slots' flags hold.
+// Distinct for consecutive calls of this process and never 0; the sequence
+// starts at a clock-derived value, so flags another process left in reused
+// device memory are unlikely (about 2^-32 per flag) to match.
+uint32_t epoch_seed()
+{
+    uint64_t x = (uint64_t)std::chrono::high_resolution_clock::now().time_since_epoch().count();
+    x ^= x >> 33;
+    x *= 0xff51afd7ed558ccdull;
+    x ^= x >> 33;
+    return (uint32_t)x;
+}
+
+uint32_t next_epoch()
+{
+    static std::atomic<uint32_t> counter{epoch_seed()};
+    uint32_t e;
+    do {
+        e = ++counter;
+    } while (e == 0);
+    return e;
 }
 
 pa_status launch_reduce(void *out, const float *tmp_out, const float *max_logits,
@@ -608,41 +642,26 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
         (int64_t)num_seqs * p.head_groups * (round_up(std::max(max_context_len, 1), 16) / 16);
     grid = (int)std::min<int64_t>(grid, tiles_up);
     const size_t need = stream_k_bytes(num_seqs, num_kv_heads, group, head_dim, grid);
-    const bool stream_k = workspace != nullptr && workspace_bytes >= need && aligned16(workspace);
-    pa::MergeParams mp;
-    std::memset(&mp, 0, sizeof(mp));
+    // the merges use a warp's share of the stage ring as scratch
+    const int64_t ring_share = (int64_t)p.geo.spw * p.geo.stage_bytes / p.geo.hpc & ~(int64_t)15;
+    const bool stream_k = workspace != nullptr && workspace_bytes >= need &&
+                          aligned16(workspace) &&
+                          pa::merge_scratch_bytes(group, head_dim, grid) <= ring_share;
     if (stream_k) {
         p.mode = 0;
-        p.slot_floats = (int)round_up((int64_t)group * head_dim + 2 * group + 1, 4);
+        p.slot_floats = (int)slot_floats(group, head_dim);
         p.wpart = static_cast<float *>(workspace);
-        p.seg_start =
-            reinterpret_cast<int32_t *>(p.wpart + 2 * (int64_t)grid * p.geo.hpc * p.slot_floats);
-        p.total_tiles = p.seg_start + round_up((int64_t)num_seqs * p.head_groups, 4);
-        mp.out = out;
-        mp.wpart = p.wpart;
-        mp.seg_start = p.seg_start;
-        mp.total_tiles = p.total_tiles;
-        mp.context_lens = context_lens;
-        mp.num_seqs = num_seqs;
-        mp.num_q_heads = num_q_heads;
-        mp.num_kv_heads = num_kv_heads;
-        mp.ctx_cap = p.ctx_cap;
-        mp.total_ctas = grid;
-        mp.hpc = p.geo.hpc;
-        mp.slot_floats = p.slot_floats;
+        p.flags = reinterpret_cast<uint32_t *>(p.wpart +
+                                               2 * (int64_t)grid * p.geo.hpc * p.slot_floats);
+        p.epoch = next_epoch();
     } else {
         p.mode = 1;
     }
     const int want = grid;
     st = decode_call(L, dtype, &grid, true);
     ++g_launches;
-    if (st != PA_OK || !stream_k)
-        return st;
-    if (grid != want)
+    if (st == PA_OK && stream_k && grid != want)
         return PA_ERR_CUDA;   // capacity changed between query and launch
-    st = dtype == PA_DTYPE_F32 ? pa::merge_f32(mp, head_dim, group, L.stream)
-                               : pa::merge_bf16(mp, head_dim, group, L.stream);
-    ++g_launches;
     return st;
 }
 

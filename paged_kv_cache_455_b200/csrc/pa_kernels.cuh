@@ -8,10 +8,10 @@
 //   partition, head group, token.  A "segment" is the run of tiles of one
 //   (sequence, partition, head group).  Every CTA owns one contiguous range of
 //   that sequence:
-//     mode 0 (stream-K): equal ranges.  A segment cut by range boundaries
-//       leaves one partial softmax state per piece and head (at most two
-//       pieces per CTA), merged afterwards by merge_kernel.  Balanced for any
-//       mix of lengths.
+//     mode 0 (stream-K): equal ranges.  Every CTA holding a piece of a
+//       segment cut by range boundaries publishes the piece's partial softmax
+//       state, and after its range each of them merges an equal share of the
+//       segment's outputs from all pieces.  Balanced for any mix of lengths.
 //     mode 1: ranges snapped to segment starts, so one CTA finishes every
 //       segment it starts (no partials; used without a workspace and for the
 //       explicit fixed-partition split-K API).
@@ -32,7 +32,6 @@
 //   Both keep the online softmax (running max and sum) in fp32, in the log2
 //   domain (logits pre-multiplied by log2 e).
 //
-// merge_kernel    log-sum-exp merge of the warp pieces of cut segments.
 // reduce_kernel   log-sum-exp merge of fixed-size partitions (explicit API).
 #pragma once
 
@@ -91,8 +90,7 @@ struct DecodeParams {
     float *max_logits;       // [B, Hq, max_parts]
     float *exp_sums;         // [B, Hq, max_parts]
     float *wpart;            // mode 0: two partial slots per CTA and head
-    int32_t *seg_start;      // mode 0: first global tile of each (b, head group) segment
-    int32_t *total_tiles;    // mode 0: total tile count (written by the kernel)
+    uint32_t *flags;         // mode 0: slot published (holds the call's epoch)
     int32_t *dev_status;
     int64_t num_blocks;
     int num_seqs;
@@ -108,6 +106,7 @@ struct DecodeParams {
     int public_partials;     // mode 1: write tmp_out / max_logits / exp_sums
     int slot_floats;         // floats per partial slot (mode 0)
     int head_groups;         // Hkv / hpc
+    uint32_t epoch;          // mode 0: value a published slot's flag holds (never 0)
     float scale_log2;
     TileGeo geo;
 };
@@ -123,21 +122,6 @@ struct ReduceParams {
     int partition_size;
     int max_parts;
     int ctx_cap;
-};
-
-struct MergeParams {
-    void *out;
-    const float *wpart;
-    const int32_t *seg_start;
-    const int32_t *total_tiles;
-    const int32_t *context_lens;
-    int num_seqs;
-    int num_q_heads;
-    int num_kv_heads;
-    int ctx_cap;
-    int total_ctas;
-    int hpc;
-    int slot_floats;
 };
 
 __device__ __forceinline__ void report(int32_t *status, int bit)
@@ -156,6 +140,21 @@ __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16 *dst, flo
     *dst = __float2bfloat16_rn(v);
 }
 
+// 16 bytes of outputs from VEC = 16 / sizeof(T) floats.
+__device__ __forceinline__ void store16(float *dst, const float *x)
+{
+    *reinterpret_cast<float4 *>(dst) = make_float4(x[0], x[1], x[2], x[3]);
+}
+__device__ __forceinline__ void store16(__nv_bfloat16 *dst, const float *x)
+{
+    uint4 u;
+    u.x = ptx::pack_bf16x2(x[0], x[1]);
+    u.y = ptx::pack_bf16x2(x[2], x[3]);
+    u.z = ptx::pack_bf16x2(x[4], x[5]);
+    u.w = ptx::pack_bf16x2(x[6], x[7]);
+    *reinterpret_cast<uint4 *>(dst) = u;
+}
+
 // =====================================================================
 // Tile enumeration
 // =====================================================================
@@ -163,19 +162,45 @@ __device__ __forceinline__ int eff_ctx(int ctx, int cap) { return (ctx < 0 || ct
 __device__ __forceinline__ int num_parts(int ctx, int P) { return ctx <= 0 ? 1 : (ctx + P - 1) / P; }
 __device__ __forceinline__ int ntiles(int ctx) { return (ctx + kTile - 1) / kTile; }
 
-// Total tiles of the batch (every lane gets it).
-__device__ __forceinline__ int count_tiles(const DecodeParams &p, int lane)
+constexpr int kMaxChunks = 1024;   // sequences / 32, i.e. batches of up to 32768 sequences
+
+// CTA-cooperative: cbase[c] = global index of the first tile of sequence
+// 32 c, for c = 0 .. ceil(B / 32); returns the total tile count.  Must be
+// called by every thread of the CTA (contains __syncthreads).
+__device__ __forceinline__ int chunk_prefix(const DecodeParams &p, int *cbase)
 {
-    int sum = 0;
-    for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
-        const int b = b0 + lane;
-        if (b < p.num_seqs)
-            sum += ntiles(eff_ctx(p.context_lens[b], p.ctx_cap)) * p.head_groups;
-    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int nch = (p.num_seqs + 31) >> 5;
+    for (int c = warp; c < nch; c += nwarps) {
+        const int b = c * 32 + lane;
+        int t = b < p.num_seqs ? ntiles(eff_ctx(p.context_lens[b], p.ctx_cap)) * p.head_groups : 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        sum += __shfl_xor_sync(kFull, sum, o);
-    return sum;
+        for (int o = 16; o > 0; o >>= 1)
+            t += __shfl_xor_sync(kFull, t, o);
+        if (lane == 0)
+            cbase[c + 1] = t;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        if (lane == 0)
+            cbase[0] = 0;
+        for (int c0 = 0; c0 < nch; c0 += 32) {
+            const int c = c0 + lane;
+            int v = c < nch ? cbase[c + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(kFull, v, o);
+                if (lane >= o)
+                    v += u;
+            }
+            if (c < nch)
+                cbase[c + 1] = carry + v;
+            carry += __shfl_sync(kFull, v, 31);
+        }
+    }
+    __syncthreads();
+    return cbase[nch];
 }
 
 // A window of 32 consecutive sequences with their tile counts, one per lane,
@@ -206,12 +231,29 @@ __device__ __forceinline__ void window_load(SeqWindow &w, int b0, int base, cons
     w.incl = incl;
 }
 
+// Index of the chunk of 32 sequences holding global tile g (binary search
+// over the chunk prefix; g must be below the total).
+__device__ __forceinline__ int chunk_of(const int *cbase, int nch, int g)
+{
+    int lo = 0, hi = nch - 1;   // largest c with cbase[c] <= g
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cbase[mid] <= g)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
 // Resolves each lane's global tile index g (ignored where !want) to its
 // sequence: b, the global index of the sequence's first tile, and its
-// effective length.  The window only moves forward, so targets must not
-// precede it.  Warp-uniform control flow.
+// effective length.  The window moves forward by jumping to the chunk of the
+// smallest unresolved target, so targets must not precede the window.
+// Warp-uniform control flow.
 __device__ __forceinline__ void window_find(SeqWindow &w, int g, bool want, int &b, int &seqbase,
-                                            int &ctx, const DecodeParams &p, int lane)
+                                            int &ctx, const DecodeParams &p, const int *cbase,
+                                            int lane)
 {
     bool done = !want;
     b = 0;
@@ -242,7 +284,12 @@ __device__ __forceinline__ void window_find(SeqWindow &w, int g, bool want, int 
             break;
         if (w.b0 + 32 >= p.num_seqs)   // targets past the last tile: leave them
             break;
-        window_load(w, w.b0 + 32, last, p, lane);
+        int gmin = done ? INT32_MAX : g;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            gmin = min(gmin, __shfl_xor_sync(kFull, gmin, o));
+        const int c = max(chunk_of(cbase, (p.num_seqs + 31) >> 5, gmin), (w.b0 >> 5) + 1);
+        window_load(w, c * 32, cbase[c], p, lane);
     }
 }
 
@@ -253,34 +300,33 @@ struct TileDesc {
     int phys[4];
 };
 
-// Descriptor of lane `src` of batch d1 (sel) or d0 (!sel), to every lane.
-__device__ __forceinline__ TileDesc shfl_desc(const TileDesc &d0, const TileDesc &d1, bool sel,
-                                              int src)
+// Descriptor of lane `src` of batch d, to every lane.
+__device__ __forceinline__ TileDesc shfl_desc(const TileDesc &d, int src)
 {
     TileDesc o;
-    o.b = __shfl_sync(kFull, sel ? d1.b : d0.b, src);
-    o.h = __shfl_sync(kFull, sel ? d1.h : d0.h, src);
-    o.part = __shfl_sync(kFull, sel ? d1.part : d0.part, src);
-    o.j = __shfl_sync(kFull, sel ? d1.j : d0.j, src);
-    o.ns = __shfl_sync(kFull, sel ? d1.ns : d0.ns, src);
-    o.t0 = __shfl_sync(kFull, sel ? d1.t0 : d0.t0, src);
-    o.n = __shfl_sync(kFull, sel ? d1.n : d0.n, src);
-    o.ctx = __shfl_sync(kFull, sel ? d1.ctx : d0.ctx, src);
+    o.b = __shfl_sync(kFull, d.b, src);
+    o.h = __shfl_sync(kFull, d.h, src);
+    o.part = __shfl_sync(kFull, d.part, src);
+    o.j = __shfl_sync(kFull, d.j, src);
+    o.ns = __shfl_sync(kFull, d.ns, src);
+    o.t0 = __shfl_sync(kFull, d.t0, src);
+    o.n = __shfl_sync(kFull, d.n, src);
+    o.ctx = __shfl_sync(kFull, d.ctx, src);
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-        o.phys[k] = __shfl_sync(kFull, sel ? d1.phys[k] : d0.phys[k], src);
+        o.phys[k] = __shfl_sync(kFull, d.phys[k], src);
     return o;
 }
 
 // Fills the descriptors of tiles [base, base + 32) below `end` and starts
 // their block-table loads.
 __device__ __forceinline__ void fill_batch(TileDesc &d, SeqWindow &w, int base, int end,
-                                           const DecodeParams &p, int lane)
+                                           const DecodeParams &p, const int *cbase, int lane)
 {
     const int g = base + lane;
     const bool want = g < end;
     int b, seqbase, ctx;
-    window_find(w, g, want, b, seqbase, ctx, p, lane);
+    window_find(w, g, want, b, seqbase, ctx, p, cbase, lane);
     d.b = b;
     d.h = 0;
     d.part = 0;
@@ -322,7 +368,7 @@ __device__ __forceinline__ void fill_batch(TileDesc &d, SeqWindow &w, int base, 
 
 // First tile of warp gw's range (T for gw == total_warps).
 __device__ __forceinline__ int range_begin(int gw, int total_warps, int T, const DecodeParams &p,
-                                           int lane)
+                                           const int *cbase, int lane)
 {
     if (gw >= total_warps)
         return T;
@@ -331,9 +377,10 @@ __device__ __forceinline__ int range_begin(int gw, int total_warps, int T, const
         return x;
     // mode 1: the first segment start at or after x
     SeqWindow w;
-    window_load(w, 0, 0, p, lane);
+    const int c = chunk_of(cbase, (p.num_seqs + 31) >> 5, x);
+    window_load(w, c * 32, cbase[c], p, lane);
     TileDesc d;
-    fill_batch(d, w, x, x + 1, p, lane);
+    fill_batch(d, w, x, x + 1, p, cbase, lane);
     const int j = __shfl_sync(kFull, d.j, 0);
     const int ns = __shfl_sync(kFull, d.ns, 0);
     return j == 0 ? x : x - j + ns;
@@ -490,6 +537,29 @@ struct MmaMath {
         for (int o = 4; o < 32; o <<= 1) {
             l[0] += __shfl_xor_sync(kFull, l[0], o);
             l[1] += __shfl_xor_sync(kFull, l[1], o);
+        }
+    }
+
+    // Writes acc / sum (zeros where `zero` or the sum is 0) to o[head * D + d]
+    // for the heads this lane holds: one reciprocal per head, no division.
+    template <typename T>
+    __device__ __forceinline__ void store_final(T *o, bool zero, int lane) const
+    {
+        const int r = lane >> 2, c = lane & 3;
+        const int h0 = 2 * c, h1 = 2 * c + 1;
+        const float i0 = (zero || !(l[0] > 0.f)) ? 0.f : __frcp_rn(l[0]);
+        const float i1 = (zero || !(l[1] > 0.f)) ? 0.f : __frcp_rn(l[1]);
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            const int d0 = 16 * k + r;
+            if (h0 < G) {
+                store_out<T>(o + h0 * D + d0, acc[k][0] * i0);
+                store_out<T>(o + h0 * D + d0 + 8, acc[k][2] * i0);
+            }
+            if (h1 < G) {
+                store_out<T>(o + h1 * D + d0, acc[k][1] * i1);
+                store_out<T>(o + h1 * D + d0 + 8, acc[k][3] * i1);
+            }
         }
     }
 
@@ -684,6 +754,27 @@ struct SimtMath {
         }
     }
 
+    // Writes acc / sum (zeros where `zero` or the sum is 0) to o[g * D + d],
+    // VEC consecutive d per 16-byte store; lanes of row group 0 hold them.
+    __device__ __forceinline__ void store_final(T *o, bool zero, int lane) const
+    {
+        const int li = lane % LPR;
+        if (lane / LPR != 0)
+            return;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float inv = (zero || !(l[g] > 0.f)) ? 0.f : __frcp_rn(l[g]);
+#pragma unroll
+            for (int c = 0; c < UPL; ++c) {
+                float x[VEC];
+#pragma unroll
+                for (int v = 0; v < VEC; ++v)
+                    x[v] = acc[g][c * VEC + v] * inv;
+                store16(o + g * D + (c * LPR + li) * VEC, x);
+            }
+        }
+    }
+
     template <typename F, typename FM>
     __device__ __forceinline__ void for_each(int lane, F f, FM fm) const
     {
@@ -707,11 +798,11 @@ struct SimtMath {
 };
 
 // Bytes of the decode kernel's dynamic shared memory besides the stages:
-// alignment slack, full and empty barriers, per-stage tile metadata, and the
-// CUDA-core math's score rows.
+// alignment slack, full and empty barriers, per-stage tile metadata, the
+// CUDA-core math's score rows, and the chunk prefix of the tile counts.
 __host__ __device__ constexpr int decode_smem_fixed(int G)
 {
-    return 1024 + 16 * kMaxSpw + 32 * kMaxSpw + kMaxHpc * kTile * G * 4;
+    return 1024 + 16 * kMaxSpw + 32 * kMaxSpw + kMaxHpc * kTile * G * 4 + 4 * (kMaxChunks + 1);
 }
 
 // Tile metadata the producer warp hands to the consumer warps with a stage.
@@ -719,15 +810,178 @@ struct StageMeta {
     int b, hg, part, j, ns, n, ctx, bad;
 };
 
+// Index of the CTA whose range [R(x), R(x + 1)), R(x) = x T / C, holds tile t.
+__device__ __forceinline__ int cta_of(int t, int C, int T)
+{
+    return (int)((((int64_t)t + 1) * C - 1) / T);
+}
+
+// Slot of the piece that CTA x holds of a cut segment: 2x + 1 when the
+// segment starts inside the CTA's range (its first piece), 2x otherwise (a
+// later piece, met at the start of the range).  Times hpc, plus the head.
+__device__ __forceinline__ int piece_slot(int x, bool first, int hpc, int hl)
+{
+    return (2 * x + (first ? 1 : 0)) * hpc + hl;
+}
+
+// Bytes of per-warp shared scratch a cut-segment merge over np pieces needs:
+// np x G maxima (then weights) and np slices of at most G*D/np + 1 floats.
+__host__ __device__ constexpr int64_t merge_scratch_bytes(int G, int D, int64_t np)
+{
+    return 4 * (np * G + (int64_t)G * D + np);
+}
+
+// Merge of a segment cut across the CTAs x0..xl (mode 0), run by one warp
+// of every one of those CTAs for its head of the group, after all of the
+// CTA's own pieces are published.  Participant q = blockIdx.x - x0 of np
+// writes the outputs [q G D / np, (q + 1) G D / np) of that head's G query
+// heads (flattened [G][D]).  The result is the log-sum-exp combination of
+// the pieces' partial softmax states (max m_i, sum l_i, accumulator a_i, in
+// the log2 domain):
+//     M = max_i m_i,   L = sum_i l_i 2^(m_i - M),   o = sum_i a_i 2^(m_i - M) / L,
+// the same identity the split-K reduction uses, with the pieces summed in
+// piece order so that the result does not depend on timing.  Round trips to
+// L2: one for the flags, one for the (max, sum) pairs, one for all slices.
+template <typename T, int D, int G>
+__device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, int total, int segS,
+                                               int ns, int64_t bh0, int hl, float *buf, int lane)
+{
+    constexpr int GD = G * D;
+    constexpr int NL = GD / 32 + 1 < 33 ? GD / 32 + 1 : 33;   // loads in flight per lane
+    const int hpc = p.geo.hpc;
+    const int x0 = cta_of(segS, C, total);
+    const int np = cta_of(segS + ns - 1, C, total) - x0 + 1;
+    const int q = (int)blockIdx.x - x0;
+    const int lo = (int)((int64_t)q * GD / np);
+    const int S = (int)((int64_t)(q + 1) * GD / np) - lo;
+    float *wbuf = buf;            // [np][G]
+    float *raw = buf + np * G;    // [np][S]
+    T *out = static_cast<T *>(p.out);
+
+    // 1. every piece's flag (lane i waits for pieces i, i + 32, ...), its bad
+    //    mark and its (max, sum) per query head, merged per lane
+    bool late = false, bad = false;
+    float M[G], L[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        M[g] = -INFINITY;
+        L[g] = 0.f;
+    }
+    for (int i = lane; i < np; i += 32) {
+        const int slot = piece_slot(x0 + i, i == 0, hpc, hl);
+        if (!ptx::flag_wait_bounded(p.flags + slot, p.epoch, kWaitLimitNs)) {
+            late = true;
+            continue;
+        }
+        const float *ps = p.wpart + (int64_t)slot * p.slot_floats;
+        bad |= __ldcg(ps + GD + 2 * G) != 0.f;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float m = __ldcg(ps + GD + g), l = __ldcg(ps + GD + G + g);
+            wbuf[i * G + g] = m;
+            const float Mn = fmaxf(M[g], m);
+            if (Mn != -INFINITY) {
+                L[g] = L[g] * ptx::ex2(M[g] - Mn) + l * ptx::ex2(m - Mn);
+                M[g] = Mn;
+            }
+        }
+    }
+    late = __any_sync(kFull, late);
+    bad = __any_sync(kFull, bad);
+    // butterfly: the merge is symmetric, so every lane ends with equal values
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float M2 = __shfl_xor_sync(kFull, M[g], o);
+            const float L2 = __shfl_xor_sync(kFull, L[g], o);
+            const float Mn = fmaxf(M[g], M2);
+            if (Mn != -INFINITY) {
+                L[g] = L[g] * ptx::ex2(M[g] - Mn) + L2 * ptx::ex2(M2 - Mn);
+                M[g] = Mn;
+            }
+        }
+    }
+    // the warp barrier orders the lanes' loads below after the acquiring
+    // loads of the flags (those loads bypass L1)
+    __syncwarp();
+    if (late || bad) {
+        if (lane == 0)
+            report(p.dev_status, late ? PA_DEV_WAIT_TIMEOUT : PA_DEV_BAD_BLOCK);
+        for (int e = lane; e < S; e += 32)
+            store_out<T>(out + (bh0 + (lo + e) / D) * D + (lo + e) % D, 0.f);
+        return;
+    }
+
+    // 2. weights 2^(m_i - M) / L in place of the maxima
+    for (int i = lane; i < np; i += 32) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float m = wbuf[i * G + g];
+            wbuf[i * G + g] = (m == -INFINITY || !(L[g] > 0.f)) ? 0.f : ptx::ex2(m - M[g]) / L[g];
+        }
+    }
+
+    // 3. this participant's slice of every piece, all loads in flight at once
+    const int items = np * S;
+    // item f is element f mod S of piece f / S; the quotient comes from a
+    // float reciprocal: (f + 1/2) / S lies at least 1/(2S) from an integer and
+    // the two roundings move it by less than 2^-23 f / S, so it truncates
+    // exactly for f < 2^22 (f < G*D + np here)
+    const float invS = S > 0 ? 1.f / (float)S : 0.f;
+    for (int f0 = 0; f0 < items; f0 += 32 * NL) {
+        float v[NL];
+#pragma unroll
+        for (int k = 0; k < NL; ++k) {
+            const int f = f0 + lane + 32 * k;
+            v[k] = 0.f;
+            if (f < items) {
+                const int i = __float2int_rz(((float)f + 0.5f) * invS);
+                const int slot = piece_slot(x0 + i, i == 0, hpc, hl);
+                v[k] = __ldcg(p.wpart + (int64_t)slot * p.slot_floats + lo + (f - i * S));
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < NL; ++k) {
+            const int f = f0 + lane + 32 * k;
+            if (f < items)
+                raw[f] = v[k];
+        }
+    }
+    __syncwarp();
+
+    // 4. weighted sums in piece order
+    for (int e = lane; e < S; e += 32) {
+        const int idx = lo + e;
+        const int g = idx / D;
+        float o = 0.f;
+        for (int i = 0; i < np; ++i)
+            o = fmaf(wbuf[i * G + g], raw[i * S + e], o);
+        store_out<T>(out + (bh0 + g) * D + idx % D, o);
+    }
+    __syncwarp();
+}
+
 // =====================================================================
 // Decode kernel: hpc consumer warps (one per KV head of the group) and one
 // producer warp per CTA; launched with 32 * (hpc + 1) threads.
 //
-// CTA x owns the CTA-tile range [range_begin(x), range_begin(x + 1)).  The
-// stages form a ring; each has a "full" mbarrier (the producer arrives with
-// the expected bytes, TMA completes them) and an "empty" mbarrier (each
-// consumer warp arrives once it is done with the stage).  No warp waits on
-// another CTA, and every wait is bounded.
+// CTA x owns the CTA-tile range [R(x), R(x + 1)).  The stages form a ring;
+// each has a "full" mbarrier (the producer arrives with the expected bytes,
+// TMA completes them) and an "empty" mbarrier (each consumer warp arrives
+// once it is done with the stage).
+//
+// Mode 0 cuts segments at range borders and merges them inside the kernel.
+// Each CTA holding a piece of a cut segment publishes the piece's partial
+// state (acc [G][D], max [G], sum [G], bad) in its slot with a release store
+// of the call's epoch to the slot's flag, when it reaches the piece's end.
+// After its whole range, each such CTA merges its share of the segment's
+// outputs (merge_cut_segment).  A CTA waits only after all of its own pieces
+// are published and every CTA of the persistent grid is resident, so every
+// wait ends; each is bounded all the same.
+//
+// Nothing touches global memory before griddepcontrol.wait: the kernel is
+// launched as a programmatic dependent of the kernel before it on the stream.
 // =====================================================================
 template <typename T, int D, int G, bool MMA, bool TR16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -744,7 +998,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int HG = p.head_groups;
     const int Hq = p.num_q_heads;
 
-    // 1024-byte aligned layout: [stages][full bars][empty bars][meta][score rows]
+    // 1024-byte aligned layout: [stages][full bars][empty bars][meta][score rows][chunk prefix]
     const uint32_t raw = ptx::smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     uint8_t *sgen = smem_raw + (sbase - raw);
@@ -753,6 +1007,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t empty0 = full0 + 8u * kMaxSpw;
     StageMeta *meta = reinterpret_cast<StageMeta *>(sgen + stages_bytes + 16 * kMaxSpw);
     float *scores_all = reinterpret_cast<float *>(sgen + stages_bytes + 48 * kMaxSpw);
+    int *cbase = reinterpret_cast<int *>(scores_all + kMaxHpc * kTile * G);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < spw; ++s) {
@@ -761,11 +1016,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     ptx::fence_mbar_init();
-    __syncthreads();
-
-    const int total = count_tiles(p, lane);
-    const int R0 = range_begin(blockIdx.x, total_ctas, total, p, lane);
-    const int R1 = range_begin(blockIdx.x + 1, total_ctas, total, p, lane);
+    ptx::grid_wait_prerequisites();
+    const int total = chunk_prefix(p, cbase);   // contains __syncthreads
+    // C <= T CTAs take part, so that every participating range is non-empty
+    const int C = min(total_ctas, max(total, 1));
+    const int R0 = range_begin(blockIdx.x, C, total, p, cbase, lane);
+    const int R1 = range_begin(blockIdx.x + 1, C, total, p, cbase, lane);
 
     if (warp == hpc) {
         // =================================================== producer warp
@@ -775,10 +1031,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::prefetch_tensormap(&tmap_v);
         const uint64_t policy = ptx::policy_evict_first();
         SeqWindow win;
-        window_load(win, 0, 0, p, lane);
+        {
+            const int c = chunk_of(cbase, (p.num_seqs + 31) >> 5, R0);
+            window_load(win, c * 32, cbase[c], p, lane);
+        }
         TileDesc bat0, bat1;
-        fill_batch(bat0, win, R0, R1, p, lane);
-        fill_batch(bat1, win, R0 + 32, R1, p, lane);
+        fill_batch(bat0, win, R0, R1, p, cbase, lane);
+        fill_batch(bat1, win, R0 + 32, R1, p, cbase, lane);
         int filled = 2;
         int issued = R0;
         for (; issued < R1; ++issued) {
@@ -792,7 +1051,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
                 break;
             }
-            const TileDesc d = shfl_desc(bat0, bat1, (k >> 5) & 1, k & 31);
+            const TileDesc d = ((k >> 5) & 1) ? shfl_desc(bat1, k & 31) : shfl_desc(bat0, k & 31);
             const bool newseg = d.j == 0 || i == R0;
             int tx = newseg ? geo.q_bytes : 0;
             bool bad = false;
@@ -842,9 +1101,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // descriptors of batch k/32 are used up: prepare the batch after next
             if ((k & 31) == 31) {
                 if (filled & 1)
-                    fill_batch(bat1, win, R0 + 32 * filled, R1, p, lane);
+                    fill_batch(bat1, win, R0 + 32 * filled, R1, p, cbase, lane);
                 else
-                    fill_batch(bat0, win, R0 + 32 * filled, R1, p, lane);
+                    fill_batch(bat0, win, R0 + 32 * filled, R1, p, cbase, lane);
                 ++filled;
             }
         }
@@ -889,14 +1148,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     }
-    if (p.mode == 0 && blockIdx.x == 0 && warp == 0 && lane == 0)
-        *p.total_tiles = total;
 
     using Math =
         typename std::conditional<MMA, MmaMath<D, G, TR16>, SimtMath<T, D, G, TR16>>::type;
     Math math;
     int segS = 0;          // global index of the current segment's first tile
     bool seg_bad = false;
+    bool timed_out = false;
+    // cut segments this warp holds a piece of (mode 0): a later piece met at
+    // the start of the range, and the first piece of one that runs past its end
+    int laterS = -1, laterN = 0, laterB = 0, laterHG = 0;
+    int firstS = -1, firstN = 0, firstB = 0, firstHG = 0;
 
     for (int i = R0; i < R1; ++i) {
         const int k = i - R0;
@@ -904,6 +1166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ptx::mbar_wait_bounded(full0 + 8u * s, (uint32_t)((k / spw) & 1), kWaitLimitNs)) {
             if (lane == 0)
                 report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+            timed_out = true;
             break;
         }
         const StageMeta d = meta[s];
@@ -918,8 +1181,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 math.begin(qslot, lane);
             else
                 math.begin(qslot, lane, p.scale_log2);
-            if (p.mode == 0 && d.j == 0 && hl == 0 && lane == 0)
-                p.seg_start[(int64_t)d.b * HG + d.hg] = i;
         }
         if (d.bad)
             seg_bad = true;
@@ -956,11 +1217,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             math.finish();
             const int segE = segS + d.ns;
             const bool complete = segS >= R0 && segE <= R1;
-            if (seg_bad && lane == 0)
-                report(p.dev_status, PA_DEV_BAD_BLOCK);
             const int64_t bh0 = (int64_t)d.b * Hq + (int64_t)(d.hg * hpc + hl) * G;
             if (p.mode == 0 && !complete) {
-                const int slot = ((segS < R0 ? 2 * blockIdx.x : 2 * blockIdx.x + 1) * hpc) + hl;
+                // a piece of a cut segment: publish it, merge after the range
+                const bool first = segS >= R0;
+                const int slot = piece_slot(blockIdx.x, first, hpc, hl);
                 float *ps = p.wpart + (int64_t)slot * p.slot_floats;
                 math.for_each(
                     lane, [&](int hh, int e, float v, float) { ps[hh * D + e] = v; },
@@ -970,153 +1231,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                     });
                 if (lane == 0)
                     ps[G * D + 2 * G] = seg_bad ? 1.f : 0.f;
-            } else {
-                const bool single = num_parts(d.ctx, p.partition_size) == 1;
-                math.for_each(
-                    lane,
-                    [&](int hh, int e, float v, float ll) {
-                        const float res = (seg_bad || !(ll > 0.f)) ? 0.f : v / ll;
-                        if (p.public_partials)
-                            p.tmp_out[((bh0 + hh) * p.max_parts + d.part) * D + e] = res;
-                        if (single)
-                            store_out<T>(static_cast<T *>(p.out) + (bh0 + hh) * D + e, res);
-                    },
-                    [&](int hh, float mm, float ll) {
-                        if (p.public_partials) {
-                            const int64_t slot = (bh0 + hh) * p.max_parts + d.part;
-                            const bool empty = seg_bad || !(ll > 0.f);
-                            p.max_logits[slot] = empty ? -INFINITY : mm / kLog2e;
-                            p.exp_sums[slot] = empty ? 0.f : ll;
-                        }
-                    });
-            }
-        }
-    }
-}
-
-// =====================================================================
-// Merge of cut segments (mode 0): one CTA of merge_warps() warps per
-// (sequence, KV head).  CTA x's range starts at tile floor(x T / C); the pieces
-// of segment [S, S + nt) are in slot pair 2 xf + 1 of its first CTA xf and
-// slot pair 2 x of every later non-empty CTA x <= xl (slot = pair * hpc +
-// head within the group).  Each warp of this CTA accumulates a strided subset
-// of the pieces for all G*D outputs (independent loads, so the latency is a
-// few round trips whatever the piece count); the warps' sums are then added
-// in shared memory.
-// =====================================================================
-template <int G, int D>
-__host__ __device__ constexpr int merge_warps() { return G * D <= 1024 ? 8 : 4; }
-
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(32 * merge_warps<G, D>()) merge_kernel(const MergeParams p)
-{
-    constexpr int kMergeWarps = merge_warps<G, D>();
-    __shared__ float s_max[G];
-    __shared__ float s_l[kMergeWarps][G];
-    __shared__ float s_o[kMergeWarps][G * D];
-    __shared__ int s_bad;
-    const int seg = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = seg / p.num_kv_heads;
-    const int h = seg - b * p.num_kv_heads;
-    const int hg = h / p.hpc, hl = h - hg * p.hpc;
-    const int ctx = eff_ctx(p.context_lens[b], p.ctx_cap);
-    if (ctx <= 0)
-        return;   // the decode kernel wrote zeros
-    const int nt = ntiles(ctx);
-    const int S = p.seg_start[(int64_t)b * (p.num_kv_heads / p.hpc) + hg];
-    const int64_t tot = *p.total_tiles;
-    const int64_t NW = p.total_ctas;
-    const int wf = (int)((((int64_t)S + 1) * NW - 1) / tot);
-    const int wl = (int)((((int64_t)S + nt) * NW - 1) / tot);
-    if (wf == wl)
-        return;   // finished inside one CTA
-    // CTAs with an empty range (more CTAs than tiles) hold no piece
-    auto empty = [&](int w) { return (int64_t)w * tot / NW == ((int64_t)w + 1) * tot / NW; };
-    auto slot_of = [&](int w) { return (w == wf ? 2 * w + 1 : 2 * w) * p.hpc + hl; };
-    const int npieces = wl - wf + 1;
-
-    // pass 1: maxima and the bad flag
-    if (threadIdx.x < G)
-        s_max[threadIdx.x] = -INFINITY;
-    if (threadIdx.x == 0)
-        s_bad = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < npieces; i += blockDim.x) {
-        const int w = wf + i;
-        if (empty(w))
-            continue;
-        const float *ps = p.wpart + (int64_t)slot_of(w) * p.slot_floats;
-        if (ps[G * D + 2 * G] != 0.f)
-            atomicOr(&s_bad, 1);
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float mw = ps[G * D + g];
-            // float max through the int ordering of non-negative / negative halves
-            if (mw > -INFINITY) {
-                float cur = s_max[g];
-                while (mw > cur) {
-                    const int old = atomicCAS(reinterpret_cast<int *>(&s_max[g]), __float_as_int(cur),
-                                              __float_as_int(mw));
-                    if (old == __float_as_int(cur))
-                        break;
-                    cur = __int_as_float(old);
+                // the warp barrier orders every lane's stores before lane 0's
+                // release of the flag
+                __syncwarp();
+                if (lane == 0)
+                    ptx::st_release_gpu(p.flags + slot, p.epoch);
+                if (first) {
+                    firstS = segS;
+                    firstN = d.ns;
+                    firstB = d.b;
+                    firstHG = d.hg;
+                } else {
+                    laterS = segS;
+                    laterN = d.ns;
+                    laterB = d.b;
+                    laterHG = d.hg;
                 }
-            }
-        }
-    }
-    __syncthreads();
-    const bool bad = s_bad != 0;
-
-    // pass 2: warp `warp` sums pieces warp, warp + kMergeWarps, ...
-    float o[G * D / 32];
-    float lsum[G];
-#pragma unroll
-    for (int i = 0; i < G * D / 32; ++i)
-        o[i] = 0.f;
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-        lsum[g] = 0.f;
-    if (!bad) {
-        for (int i = warp; i < npieces; i += kMergeWarps) {
-            const int w = wf + i;
-            if (empty(w))
                 continue;
-            const float *ps = p.wpart + (int64_t)slot_of(w) * p.slot_floats;
-            float f[G];
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float mw = ps[G * D + g];
-                f[g] = (mw == -INFINITY || s_max[g] == -INFINITY) ? 0.f : ptx::ex2(mw - s_max[g]);
-                lsum[g] = fmaf(ps[G * D + G + g], f[g], lsum[g]);
             }
-#pragma unroll
-            for (int i2 = 0; i2 < G * D / 32; ++i2) {
-                const int idx = i2 * 32 + lane;
-                o[i2] = fmaf(ps[idx], f[idx / D], o[i2]);
+            if (seg_bad && lane == 0)
+                report(p.dev_status, PA_DEV_BAD_BLOCK);
+            const bool single = num_parts(d.ctx, p.partition_size) == 1;
+            if (single && !p.public_partials) {
+                math.store_final(static_cast<T *>(p.out) + bh0 * D, seg_bad, lane);
+                continue;
             }
+            math.for_each(
+                lane,
+                [&](int hh, int e, float v, float ll) {
+                    const float res = (seg_bad || !(ll > 0.f)) ? 0.f : v / ll;
+                    if (p.public_partials)
+                        p.tmp_out[((bh0 + hh) * p.max_parts + d.part) * D + e] = res;
+                    if (single)
+                        store_out<T>(static_cast<T *>(p.out) + (bh0 + hh) * D + e, res);
+                },
+                [&](int hh, float mm, float ll) {
+                    if (p.public_partials) {
+                        const int64_t slot = (bh0 + hh) * p.max_parts + d.part;
+                        const bool empty = seg_bad || !(ll > 0.f);
+                        p.max_logits[slot] = empty ? -INFINITY : mm / kLog2e;
+                        p.exp_sums[slot] = empty ? 0.f : ll;
+                    }
+                });
         }
     }
-#pragma unroll
-    for (int i2 = 0; i2 < G * D / 32; ++i2)
-        s_o[warp][i2 * 32 + lane] = o[i2];
-    if (lane == 0) {
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-            s_l[warp][g] = lsum[g];
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int g = idx / D;
-        float L = 0.f, O = 0.f;
-#pragma unroll
-        for (int w = 0; w < kMergeWarps; ++w) {
-            L += s_l[w][g];
-            O += s_o[w][idx];
-        }
-        const int64_t bh = (int64_t)b * p.num_q_heads + (int64_t)h * G + g;
-        store_out<T>(static_cast<T *>(p.out) + bh * D + (idx - g * D),
-                     (!bad && L > 0.f) ? O / L : 0.f);
+
+    if (p.mode == 0) {
+        // every consumer warp is past its last stage (and with it every copy
+        // into the ring has landed): the ring is free scratch for the merges
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * hpc) : "memory");
+        if (timed_out)
+            return;
+        float *buf = reinterpret_cast<float *>(
+            sgen + (int64_t)hl * ((int64_t)stages_bytes / hpc & ~(int64_t)15));
+        if (laterS >= 0)
+            merge_cut_segment<T, D, G>(p, C, total, laterS, laterN,
+                                       (int64_t)laterB * Hq + (int64_t)(laterHG * hpc + hl) * G,
+                                       hl, buf, lane);
+        if (firstS >= 0)
+            merge_cut_segment<T, D, G>(p, C, total, firstS, firstN,
+                                       (int64_t)firstB * Hq + (int64_t)(firstHG * hpc + hl) * G,
+                                       hl, buf, lane);
     }
 }
 

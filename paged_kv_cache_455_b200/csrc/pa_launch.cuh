@@ -1,5 +1,5 @@
 // pa_launch.cuh -- host-side launch templates shared by the translation units
-// that instantiate the decode and merge kernels (one per dtype / math).
+// that instantiate the decode kernels (one per dtype / math).
 #pragma once
 
 #include <mutex>
@@ -77,7 +77,21 @@ pa_status decode_one(DecodeLaunch &L, int *grid, bool launch)
     }
     const int g = *grid < cap ? (*grid > 0 ? *grid : 1) : cap;
     *grid = g;
-    fn<<<g, threads, L.smem_bytes, L.stream>>>(L.tmap_k, L.tmap_v, L.p);
+    // programmatic dependent launch: may start while the previous kernel on
+    // the stream runs, if that kernel allows it (the cache write does); the
+    // producer waits for it before touching the pools
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = (size_t)L.smem_bytes;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, fn, L.tmap_k, L.tmap_v, L.p) != cudaSuccess)
+        return PA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -111,36 +125,9 @@ pa_status decode_dispatch(DecodeLaunch &L, int *grid, bool launch)
     }
 }
 
-template <typename T, int D>
-pa_status merge_g(const MergeParams &m, int group, cudaStream_t s)
-{
-    const unsigned grid = (unsigned)(m.num_seqs * m.num_kv_heads);
-    switch (group) {
-    case 1: merge_kernel<T, D, 1><<<grid, 32 * merge_warps<1, D>(), 0, s>>>(m); break;
-    case 2: merge_kernel<T, D, 2><<<grid, 32 * merge_warps<2, D>(), 0, s>>>(m); break;
-    case 4: merge_kernel<T, D, 4><<<grid, 32 * merge_warps<4, D>(), 0, s>>>(m); break;
-    case 8: merge_kernel<T, D, 8><<<grid, 32 * merge_warps<8, D>(), 0, s>>>(m); break;
-    default: return PA_ERR_UNSUPPORTED;
-    }
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
-}
-
-template <typename T>
-pa_status merge_dispatch(const MergeParams &m, int head_dim, int group, cudaStream_t s)
-{
-    switch (head_dim) {
-    case 64: return merge_g<T, 64>(m, group, s);
-    case 128: return merge_g<T, 128>(m, group, s);
-    case 256: return merge_g<T, 256>(m, group, s);
-    default: return PA_ERR_UNSUPPORTED;
-    }
-}
-
 // Entry points of the instantiation units.
 pa_status decode_f32(DecodeLaunch &L, int *grid, bool launch);
 pa_status decode_bf16_mma(DecodeLaunch &L, int *grid, bool launch);
 pa_status decode_bf16_simt(DecodeLaunch &L, int *grid, bool launch);
-pa_status merge_f32(const MergeParams &m, int head_dim, int group, cudaStream_t s);
-pa_status merge_bf16(const MergeParams &m, int head_dim, int group, cudaStream_t s);
 
 }  // namespace pa

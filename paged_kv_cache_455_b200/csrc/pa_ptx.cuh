@@ -17,6 +17,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p)
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+__device__ __forceinline__ uint64_t globaltimer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 {
@@ -47,6 +54,50 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// ---------------------------------------------------- grid dependencies
+// Programmatic dependent launch: the kernel that follows on the stream (when
+// launched with programmatic serialisation) may start once every CTA of this
+// grid has executed launch_dependents; it must execute wait before touching
+// memory this grid writes.
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_wait_prerequisites()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// ------------------------------------------------- cross-CTA flags (gpu scope)
+__device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Waits until *p == v.  Gives up after limit_ns nanoseconds and returns false.
+__device__ __forceinline__ bool flag_wait_bounded(const uint32_t *p, uint32_t v, uint64_t limit_ns)
+{
+    if (ld_acquire_gpu(p) == v)
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1; i < (1u << 26); ++i) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(p) == v)
+            return true;
+        if ((i & 15u) == 0 && globaltimer_ns() - t0 > limit_ns)
+            return false;
+    }
+    return false;
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t done;
@@ -58,13 +109,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
         : "r"(bar), "r"(parity)
         : "memory");
     return done != 0;
-}
-
-__device__ __forceinline__ uint64_t globaltimer_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after

@@ -64,21 +64,20 @@ def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
 
 def test_static_scratch_rejects_sizes_beyond_its_maximum():
     from paged_kv_cache_455_b200 import pa
-    # group 8, d = 256 over a batch of many sequences: the per-SM partials
-    # alone exceed the fixed scratch, so the call must refuse (and launch
+    # group 8 at d = 256: two partial slots per SM and KV head of 8*256 + 17
+    # floats (rounded to 2068) plus a flag each; on a GPU with enough SMs that
+    # is more than the fixed scratch, and the call must refuse (launching
     # nothing) rather than fall back silently
-    B = 4096
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    need = 2 * sms * 4 * 2068 * 4 + 2 * sms * 4 * 4
+    if need <= pa.PA_STATIC_SCRATCH_BYTES:
+        pytest.skip("this GPU's grid fits the scratch")
+    B = 64
     q = torch.zeros(B, 32, 256, dtype=torch.bfloat16, device=DEV)
     kp = torch.zeros(8, 16, 4, 256, dtype=torch.bfloat16, device=DEV)
-    tab = torch.zeros(B, 1, dtype=torch.int32, device=DEV)
-    lens = torch.ones(B, dtype=torch.int32, device=DEV)
-    # partials: two slots per CTA (one CTA per SM) and head of the 4-head
-    # group, each G*d + 2G + 1 floats rounded up to 4
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    slot = -(-(8 * 256 + 2 * 8 + 1) // 4) * 4
-    if 2 * sms * 4 * slot * 4 <= pa.PA_STATIC_SCRATCH_BYTES:
-        pytest.skip("this GPU's grid fits the scratch")
+    tab = torch.zeros(B, 8, dtype=torch.int32, device=DEV)
+    lens = torch.full((B,), 128, dtype=torch.int32, device=DEV)
     out = torch.zeros_like(q)
     with pytest.raises(pa.PaError) as e:
-        pa.pa_decode_attention_static(out, q, kp, kp, tab, lens, 16, 0.0625)
+        pa.pa_decode_attention_static(out, q, kp, kp, tab, lens, 128, 0.0625)
     assert e.value.status == pa.PA_ERR_WORKSPACE
