@@ -155,6 +155,16 @@ __device__ __forceinline__ void store16(__nv_bfloat16 *dst, const float *x)
     *reinterpret_cast<uint4 *>(dst) = u;
 }
 
+// Four consecutive outputs (16-byte aligned for fp32, 8-byte for bf16).
+__device__ __forceinline__ void store4(float *dst, float4 v)
+{
+    *reinterpret_cast<float4 *>(dst) = v;
+}
+__device__ __forceinline__ void store4(__nv_bfloat16 *dst, float4 v)
+{
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(ptx::pack_bf16x2(v.x, v.y), ptx::pack_bf16x2(v.z, v.w));
+}
+
 // =====================================================================
 // Tile enumeration
 // =====================================================================
@@ -541,24 +551,25 @@ struct MmaMath {
     }
 
     // Writes acc / sum (zeros where `zero` or the sum is 0) to o[head * D + d]
-    // for the heads this lane holds: one reciprocal per head, no division.
-    template <typename T>
-    __device__ __forceinline__ void store_final(T *o, bool zero, int lane) const
+    // as bf16: one reciprocal per head; each 8 x 8 block (d x head) of the
+    // normalised accumulators is packed to bf16 pairs and transposed across
+    // the warp (movmatrix), so lane (r, c) then holds head r at d = 2c, 2c + 1
+    // and stores them as one 4-byte word.
+    __device__ __forceinline__ void store_final(__nv_bfloat16 *o, bool zero, int lane) const
     {
         const int r = lane >> 2, c = lane & 3;
-        const int h0 = 2 * c, h1 = 2 * c + 1;
         const float i0 = (zero || !(l[0] > 0.f)) ? 0.f : __frcp_rn(l[0]);
         const float i1 = (zero || !(l[1] > 0.f)) ? 0.f : __frcp_rn(l[1]);
+        uint32_t *row = reinterpret_cast<uint32_t *>(o + r * D) + c;
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
-            const int d0 = 16 * k + r;
-            if (h0 < G) {
-                store_out<T>(o + h0 * D + d0, acc[k][0] * i0);
-                store_out<T>(o + h0 * D + d0 + 8, acc[k][2] * i0);
-            }
-            if (h1 < G) {
-                store_out<T>(o + h1 * D + d0, acc[k][1] * i1);
-                store_out<T>(o + h1 * D + d0 + 8, acc[k][3] * i1);
+            const uint32_t lo =
+                ptx::movmatrix_trans(ptx::pack_bf16x2(acc[k][0] * i0, acc[k][1] * i1));
+            const uint32_t hi =
+                ptx::movmatrix_trans(ptx::pack_bf16x2(acc[k][2] * i0, acc[k][3] * i1));
+            if (r < G) {
+                row[8 * k] = lo;
+                row[8 * k + 4] = hi;
             }
         }
     }
@@ -825,38 +836,39 @@ __device__ __forceinline__ int piece_slot(int x, bool first, int hpc, int hl)
 }
 
 // Bytes of per-warp shared scratch a cut-segment merge over np pieces needs:
-// np x G maxima (then weights) and np slices of at most G*D/np + 1 floats.
+// np slices of at most G*D/np + 4 floats, then np x G maxima (then weights).
 __host__ __device__ constexpr int64_t merge_scratch_bytes(int G, int D, int64_t np)
 {
-    return 4 * (np * G + (int64_t)G * D + np);
+    return 4 * ((int64_t)G * D + 4 * np + np * G);
 }
 
 // Merge of a segment cut across the CTAs x0..xl (mode 0), run by one warp
 // of every one of those CTAs for its head of the group, after all of the
 // CTA's own pieces are published.  Participant q = blockIdx.x - x0 of np
-// writes the outputs [q G D / np, (q + 1) G D / np) of that head's G query
-// heads (flattened [G][D]).  The result is the log-sum-exp combination of
-// the pieces' partial softmax states (max m_i, sum l_i, accumulator a_i, in
-// the log2 domain):
+// writes the outputs [4 lo4, 4 hi4) of that head's G query heads (flattened
+// [G][D]; lo4 = q (G D / 4) / np, hi4 likewise for q + 1).  The result is the
+// log-sum-exp combination of the pieces' partial softmax states (max m_i, sum
+// l_i, accumulator a_i, in the log2 domain):
 //     M = max_i m_i,   L = sum_i l_i 2^(m_i - M),   o = sum_i a_i 2^(m_i - M) / L,
 // the same identity the split-K reduction uses, with the pieces summed in
 // piece order so that the result does not depend on timing.  Round trips to
-// L2: one for the flags, one for the (max, sum) pairs, one for all slices.
+// L2: one for the flags, one for the (max, sum) pairs, one for all slices
+// (16-byte asynchronous copies into shared memory).
 template <typename T, int D, int G>
 __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, int total, int segS,
-                                               int ns, int64_t bh0, int hl, float *buf, int lane)
+                                                  int ns, int64_t bh0, int hl, float *buf,
+                                                  int lane)
 {
-    constexpr int GD = G * D;
-    constexpr int NL = GD / 32 + 1 < 33 ? GD / 32 + 1 : 33;   // loads in flight per lane
+    constexpr int GD4 = G * D / 4;
     const int hpc = p.geo.hpc;
     const int x0 = cta_of(segS, C, total);
     const int np = cta_of(segS + ns - 1, C, total) - x0 + 1;
     const int q = (int)blockIdx.x - x0;
-    const int lo = (int)((int64_t)q * GD / np);
-    const int S = (int)((int64_t)(q + 1) * GD / np) - lo;
-    float *wbuf = buf;            // [np][G]
-    float *raw = buf + np * G;    // [np][S]
-    T *out = static_cast<T *>(p.out);
+    const int lo4 = (int)((int64_t)q * GD4 / np);
+    const int S4 = (int)((int64_t)(q + 1) * GD4 / np) - lo4;
+    float *raw = buf;                      // [np][S4] float4
+    float *wbuf = buf + 4 * np * S4;       // [np][G]
+    T *out = static_cast<T *>(p.out) + bh0 * D;
 
     // 1. every piece's flag (lane i waits for pieces i, i + 32, ...), its bad
     //    mark and its (max, sum) per query head, merged per lane
@@ -874,10 +886,10 @@ __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, 
             continue;
         }
         const float *ps = p.wpart + (int64_t)slot * p.slot_floats;
-        bad |= __ldcg(ps + GD + 2 * G) != 0.f;
+        bad |= __ldcg(ps + 4 * GD4 + 2 * G) != 0.f;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const float m = __ldcg(ps + GD + g), l = __ldcg(ps + GD + G + g);
+            const float m = __ldcg(ps + 4 * GD4 + g), l = __ldcg(ps + 4 * GD4 + G + g);
             wbuf[i * G + g] = m;
             const float Mn = fmaxf(M[g], m);
             if (Mn != -INFINITY) {
@@ -888,7 +900,30 @@ __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, 
     }
     late = __any_sync(kFull, late);
     bad = __any_sync(kFull, bad);
-    // butterfly: the merge is symmetric, so every lane ends with equal values
+    // the warp barrier orders the lanes' reads below after the acquiring
+    // loads of the flags (the reads bypass L1)
+    __syncwarp();
+    if (late || bad) {
+        if (lane == 0)
+            report(p.dev_status, late ? PA_DEV_WAIT_TIMEOUT : PA_DEV_BAD_BLOCK);
+        for (int e = lane; e < 4 * S4; e += 32)
+            store_out<T>(out + 4 * lo4 + e, 0.f);
+        return;
+    }
+
+    // 2. this participant's slice of every piece, all copies in flight at once
+    const int items = np * S4;
+    const uint32_t raw_s = ptx::smem_u32(raw);
+    for (int f = lane; f < items; f += 32) {
+        const int i = f / S4;
+        const int slot = piece_slot(x0 + i, i == 0, hpc, hl);
+        ptx::cp_async16(raw_s + 16u * (uint32_t)f,
+                        p.wpart + (int64_t)slot * p.slot_floats + 4 * (lo4 + f - i * S4));
+    }
+
+    // 3. meanwhile: butterfly over the lanes (the merge is symmetric, so
+    //    every lane ends with equal values), then weights 2^(m_i - M) / L in
+    //    place of the maxima
 #pragma unroll
     for (int g = 0; g < G; ++g) {
 #pragma unroll
@@ -902,18 +937,6 @@ __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, 
             }
         }
     }
-    // the warp barrier orders the lanes' loads below after the acquiring
-    // loads of the flags (those loads bypass L1)
-    __syncwarp();
-    if (late || bad) {
-        if (lane == 0)
-            report(p.dev_status, late ? PA_DEV_WAIT_TIMEOUT : PA_DEV_BAD_BLOCK);
-        for (int e = lane; e < S; e += 32)
-            store_out<T>(out + (bh0 + (lo + e) / D) * D + (lo + e) % D, 0.f);
-        return;
-    }
-
-    // 2. weights 2^(m_i - M) / L in place of the maxima
     for (int i = lane; i < np; i += 32) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -921,43 +944,24 @@ __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, 
             wbuf[i * G + g] = (m == -INFINITY || !(L[g] > 0.f)) ? 0.f : ptx::ex2(m - M[g]) / L[g];
         }
     }
-
-    // 3. this participant's slice of every piece, all loads in flight at once
-    const int items = np * S;
-    // item f is element f mod S of piece f / S; the quotient comes from a
-    // float reciprocal: (f + 1/2) / S lies at least 1/(2S) from an integer and
-    // the two roundings move it by less than 2^-23 f / S, so it truncates
-    // exactly for f < 2^22 (f < G*D + np here)
-    const float invS = S > 0 ? 1.f / (float)S : 0.f;
-    for (int f0 = 0; f0 < items; f0 += 32 * NL) {
-        float v[NL];
-#pragma unroll
-        for (int k = 0; k < NL; ++k) {
-            const int f = f0 + lane + 32 * k;
-            v[k] = 0.f;
-            if (f < items) {
-                const int i = __float2int_rz(((float)f + 0.5f) * invS);
-                const int slot = piece_slot(x0 + i, i == 0, hpc, hl);
-                v[k] = __ldcg(p.wpart + (int64_t)slot * p.slot_floats + lo + (f - i * S));
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < NL; ++k) {
-            const int f = f0 + lane + 32 * k;
-            if (f < items)
-                raw[f] = v[k];
-        }
-    }
+    ptx::cp_async_wait_all();
     __syncwarp();
 
-    // 4. weighted sums in piece order
-    for (int e = lane; e < S; e += 32) {
-        const int idx = lo + e;
+    // 4. weighted sums in piece order, four consecutive outputs per lane step
+    const float4 *raw4 = reinterpret_cast<const float4 *>(raw);
+    for (int e = lane; e < S4; e += 32) {
+        const int idx = 4 * (lo4 + e);
         const int g = idx / D;
-        float o = 0.f;
-        for (int i = 0; i < np; ++i)
-            o = fmaf(wbuf[i * G + g], raw[i * S + e], o);
-        store_out<T>(out + (bh0 + g) * D + idx % D, o);
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < np; ++i) {
+            const float w = wbuf[i * G + g];
+            const float4 v = raw4[i * S4 + e];
+            o.x = fmaf(w, v.x, o.x);
+            o.y = fmaf(w, v.y, o.y);
+            o.z = fmaf(w, v.z, o.z);
+            o.w = fmaf(w, v.w, o.w);
+        }
+        store4(out + idx, o);
     }
     __syncwarp();
 }

@@ -128,6 +128,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     return false;
 }
 
+// ------------------------------------------- per-thread async copies (L2 only)
+// 16-byte global -> shared copy that bypasses L1; both addresses 16-byte
+// aligned.  Complete after cp_async_wait_all().
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // ------------------------------------------------------------- bulk copies
 // Global -> shared copy of `bytes` (multiple of 16, both addresses 16-byte
 // aligned) by the bulk-copy engine; completion adds `bytes` to the
