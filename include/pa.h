@@ -211,9 +211,10 @@ pa_status pa_splitk_reduce(void *out, const float *tmp_out, const float *max_log
  *   capture.  All calls share the one array: calls whose kernels overlap on
  *   the GPU (other streams, other threads) race and corrupt each other's
  *   results, so serialise them.  The array keeps the last call's contents
- *   and no word of it needs to start at zero: a call reads a partial result
- *   only after a flag word holds that call's own tag, which earlier calls
- *   never wrote.
+ *   and no word of it needs to start at zero: a call counts the partial
+ *   results of a split sequence in counter words tagged with that call's
+ *   own tag (a word with another tag counts as zero), and reads partial
+ *   results only once its own count is complete.
  */
 #define PA_STATIC_SCRATCH_BYTES (8u << 20)
 pa_status pa_decode_attention_static(void *out, const void *query, const void *k_pool,

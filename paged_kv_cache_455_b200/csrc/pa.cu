@@ -313,27 +313,29 @@ pa_status prepare_decode(DecodeLaunch &L, void *out, const void *query, const vo
     return PA_OK;
 }
 
-// Floats of one partial slot: acc [G][D], max [G], sum [G], bad mark.
+// Floats of one partial slot: the accumulator (G*D floats, the tensor-core
+// layout padding an odd group to an even one), max [G], sum [G], bad mark.
 int64_t slot_floats(int64_t group, int64_t head_dim)
 {
-    return round_up(group * head_dim + 2 * group + 1, 4);
+    return round_up(pa::piece_stats_off((int)head_dim, (int)group) + 2 * group + 1, 4);
 }
 
 // Stream-K workspace: two partial slots per CTA and head of the group (a CTA
 // holds at most two pieces of cut segments: one met at the start of its
-// range, one running past its end) and one publication flag per slot.
+// range, one running past its end), then one 64-bit arrival counter per CTA
+// and head (for the cut segment that starts in the CTA's range).
 size_t stream_k_bytes(int64_t num_seqs, int64_t num_kv_heads, int64_t group, int64_t head_dim,
                       int64_t ctas)
 {
     (void)num_seqs;
-    const int64_t slots = 2 * ctas * heads_per_cta((int)num_kv_heads);
-    return (size_t)(slots * slot_floats(group, head_dim) * 4 + round_up(slots * 4, 16));
+    const int64_t heads = ctas * heads_per_cta((int)num_kv_heads);
+    return (size_t)(2 * heads * slot_floats(group, head_dim) * 4 + round_up(heads * 8, 16));
 }
 
-// Epoch of a stream-K call: the value its published slots' flags hold.
-// Distinct for consecutive calls of this process and never 0; the sequence
-// starts at a clock-derived value, so flags another process left in reused
-// device memory are unlikely (about 2^-32 per flag) to match.
+// Epoch of a stream-K call: the tag its arrival counters carry.  Distinct
+// for consecutive calls of this process and never 0; the sequence starts at
+// a clock-derived value, so counters another process left in reused device
+// memory are unlikely (about 2^-32 per counter) to match.
 uint32_t epoch_seed()
 {
     uint64_t x = (uint64_t)std::chrono::high_resolution_clock::now().time_since_epoch().count();
@@ -651,8 +653,8 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
         p.mode = 0;
         p.slot_floats = (int)slot_floats(group, head_dim);
         p.wpart = static_cast<float *>(workspace);
-        p.flags = reinterpret_cast<uint32_t *>(p.wpart +
-                                               2 * (int64_t)grid * p.geo.hpc * p.slot_floats);
+        p.counters = reinterpret_cast<unsigned long long *>(
+            p.wpart + 2 * (int64_t)grid * p.geo.hpc * p.slot_floats);
         p.epoch = next_epoch();
     } else {
         p.mode = 1;

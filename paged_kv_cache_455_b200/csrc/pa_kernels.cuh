@@ -10,8 +10,9 @@
 //   that sequence:
 //     mode 0 (stream-K): equal ranges.  Every CTA holding a piece of a
 //       segment cut by range boundaries publishes the piece's partial softmax
-//       state, and after its range each of them merges an equal share of the
-//       segment's outputs from all pieces.  Balanced for any mix of lengths.
+//       state; the last one to do so merges all pieces after its range (all
+//       of them share the merge of a segment cut into many pieces).
+//       Balanced for any mix of lengths.
 //     mode 1: ranges snapped to segment starts, so one CTA finishes every
 //       segment it starts (no partials; used without a workspace and for the
 //       explicit fixed-partition split-K API).
@@ -90,7 +91,7 @@ struct DecodeParams {
     float *max_logits;       // [B, Hq, max_parts]
     float *exp_sums;         // [B, Hq, max_parts]
     float *wpart;            // mode 0: two partial slots per CTA and head
-    uint32_t *flags;         // mode 0: slot published (holds the call's epoch)
+    unsigned long long *counters;  // mode 0: arrivals per cut segment (owner CTA, head)
     int32_t *dev_status;
     int64_t num_blocks;
     int num_seqs;
@@ -106,7 +107,7 @@ struct DecodeParams {
     int public_partials;     // mode 1: write tmp_out / max_logits / exp_sums
     int slot_floats;         // floats per partial slot (mode 0)
     int head_groups;         // Hkv / hpc
-    uint32_t epoch;          // mode 0: value a published slot's flag holds (never 0)
+    uint32_t epoch;          // mode 0: tag of this call's counter values (never 0)
     float scale_log2;
     TileGeo geo;
 };
@@ -550,6 +551,45 @@ struct MmaMath {
         }
     }
 
+    // Published piece layout: the accumulator fragments of the lanes that hold
+    // real heads (c < CU), one float4 (acc[k][0..3]) per (k, lane) at unit
+    // k * 8 * CU + r * CU + c; then max and sum per head (publish_stats).
+    static constexpr int CU = (G + 1) / 2;
+    static constexpr int kUnits = KS * 8 * CU;
+
+    __device__ __forceinline__ void publish(float *ps, int lane) const
+    {
+        const int r = lane >> 2, c = lane & 3;
+        if (c < CU) {
+            float4 *p4 = reinterpret_cast<float4 *>(ps) + r * CU + c;
+#pragma unroll
+            for (int k = 0; k < KS; ++k)
+                p4[k * 8 * CU] = make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
+        }
+    }
+
+    __device__ __forceinline__ void publish_stats(float *st, int lane) const
+    {
+        const int r = lane >> 2, c = lane & 3;
+        if (r == 0 && 2 * c < G) {
+            st[2 * c] = m[0];
+            st[G + 2 * c] = l[0];
+            if (2 * c + 1 < G) {
+                st[2 * c + 1] = m[1];
+                st[G + 2 * c + 1] = l[1];
+            }
+        }
+    }
+
+    // (head, d) of element j of published unit u (head >= G: padding).
+    __device__ __forceinline__ static void unit_coords(int u, int j, int &g, int &d)
+    {
+        const int k = u / (8 * CU), rem = u - k * 8 * CU;
+        const int r = rem / CU, c = rem - r * CU;
+        g = 2 * c + (j & 1);
+        d = 16 * k + r + 8 * (j >> 1);
+    }
+
     // Writes acc / sum (zeros where `zero` or the sum is 0) to o[head * D + d]
     // as bf16: one reciprocal per head; each 8 x 8 block (d x head) of the
     // normalised accumulators is packed to bf16 pairs and transposed across
@@ -765,6 +805,43 @@ struct SimtMath {
         }
     }
 
+    // Published piece layout: acc in [G][D] order, float4 units; then max and
+    // sum per head (publish_stats).
+    static constexpr int kUnits = G * D / 4;
+
+    __device__ __forceinline__ void publish(float *ps, int lane) const
+    {
+        const int li = lane % LPR;
+        if (lane / LPR != 0)
+            return;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int c = 0; c < UPL; ++c)
+#pragma unroll
+                for (int q = 0; q < VEC / 4; ++q)
+                    *reinterpret_cast<float4 *>(ps + g * D + (c * LPR + li) * VEC + 4 * q) =
+                        make_float4(acc[g][c * VEC + 4 * q], acc[g][c * VEC + 4 * q + 1],
+                                    acc[g][c * VEC + 4 * q + 2], acc[g][c * VEC + 4 * q + 3]);
+    }
+
+    __device__ __forceinline__ void publish_stats(float *st, int lane) const
+    {
+        if (lane == 0) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                st[g] = m[g];
+                st[G + g] = l[g];
+            }
+        }
+    }
+
+    __device__ __forceinline__ static void unit_coords(int u, int j, int &g, int &d)
+    {
+        g = 4 * u / D;
+        d = 4 * u - g * D + j;
+    }
+
     // Writes acc / sum (zeros where `zero` or the sum is 0) to o[g * D + d],
     // VEC consecutive d per 16-byte store; lanes of row group 0 hold them.
     __device__ __forceinline__ void store_final(T *o, bool zero, int lane) const
@@ -835,133 +912,228 @@ __device__ __forceinline__ int piece_slot(int x, bool first, int hpc, int hl)
     return (2 * x + (first ? 1 : 0)) * hpc + hl;
 }
 
-// Bytes of per-warp shared scratch a cut-segment merge over np pieces needs:
-// np slices of at most G*D/np + 4 floats, then np x G maxima (then weights).
+// Offset (floats) of a published piece's max / sum / bad mark: after the
+// accumulator units of either tile math (the tensor-core layout pads an odd
+// group to an even one).
+__host__ __device__ constexpr int piece_stats_off(int D, int G) { return 2 * D * ((G + 1) / 2); }
+
+// A published piece's stats (max [G], sum [G], bad mark) in float4 units.
+__host__ __device__ constexpr int stats_units(int G) { return (2 * G + 1 + 3) / 4; }
+
+// Bytes of per-warp shared scratch a merge of a cut segment of up to np
+// pieces needs: np stats blocks, np x G weights, 2 G totals, and the units of
+// at least one piece (more pieces per copy round when the scratch allows).
 __host__ __device__ constexpr int64_t merge_scratch_bytes(int G, int D, int64_t np)
 {
-    return 4 * ((int64_t)G * D + 4 * np + np * G);
+    return 4 * ((int64_t)piece_stats_off(D, G) + 4 * np * stats_units(G) + np * G + 2 * G + 4);
 }
 
-// Merge of a segment cut across the CTAs x0..xl (mode 0), run by one warp
-// of every one of those CTAs for its head of the group, after all of the
-// CTA's own pieces are published.  Participant q = blockIdx.x - x0 of np
-// writes the outputs [4 lo4, 4 hi4) of that head's G query heads (flattened
-// [G][D]; lo4 = q (G D / 4) / np, hi4 likewise for q + 1).  The result is the
-// log-sum-exp combination of the pieces' partial softmax states (max m_i, sum
-// l_i, accumulator a_i, in the log2 domain):
+// Counts one more arrival at a cut segment's counter for this call.  The
+// high half of the counter holds a call's epoch: CTA x tags its own counters
+// (epoch, count 0) when it starts, before any piece is done.  An arrival
+// adds 1; if its add landed on a word that still carried an older epoch, the
+// owner's tag store (still to come) overwrites it, so the arrival waits
+// (bounded) for the tag and adds again.  The acquire-release add publishes
+// the caller's piece (stored before it) and, for the last arrival, makes
+// every earlier arrival's piece visible.  Returns the arrivals so far
+// including this one, or 0 if the tag never came.
+__device__ __forceinline__ int segment_arrive(unsigned long long *c, uint32_t epoch)
+{
+    unsigned long long old = ptx::atom_add_acq_rel_gpu(c, 1ull);
+    if ((uint32_t)(old >> 32) == epoch)
+        return (int)(old & 0xffffffffu) + 1;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t i = 0; i < (1u << 26); ++i) {
+        if ((uint32_t)(ptx::ld_relaxed_gpu_u64(c) >> 32) == epoch) {
+            old = ptx::atom_add_acq_rel_gpu(c, 1ull);
+            if ((uint32_t)(old >> 32) == epoch)
+                return (int)(old & 0xffffffffu) + 1;
+        }
+        __nanosleep(64);
+        if ((i & 15u) == 0 && ptx::globaltimer_ns() - t0 > kWaitLimitNs)
+            break;
+    }
+    return 0;
+}
+
+// Segments cut into more pieces than this are merged by all of their
+// CTAs together (each a slice of the outputs) rather than by the last one.
+constexpr int kLastMergesPieces = 8;
+
+// Merge of a segment cut across the CTAs x0..xl (mode 0, np pieces), for
+// this warp's head of the group, after the warp's range, over the published
+// units [lo, lo + S) of every piece:
+//   - np <= kLastMergesPieces: the warp whose arrival completed the count
+//     merges every unit (lo = 0, S = U), all pieces being published;
+//   - otherwise every participant q = blockIdx.x - x0 takes the units
+//     [q U / np, (q + 1) U / np), after waiting (bounded) for the count.
+// The result is the log-sum-exp combination of the pieces' partial softmax
+// states (max m_i, sum l_i, accumulator a_i, log2 domain):
 //     M = max_i m_i,   L = sum_i l_i 2^(m_i - M),   o = sum_i a_i 2^(m_i - M) / L,
-// the same identity the split-K reduction uses, with the pieces summed in
-// piece order so that the result does not depend on timing.  Round trips to
-// L2: one for the flags, one for the (max, sum) pairs, one for all slices
-// (16-byte asynchronous copies into shared memory).
-template <typename T, int D, int G>
+// the identity the split-K reduction uses, with every sum taken in piece
+// order so that the result does not depend on timing.  The stats and units
+// come into shared memory by 16-byte asynchronous copies, as many pieces per
+// round as `buf` holds.
+template <typename T, int D, int G, typename Math>
 __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, int total, int segS,
                                                   int ns, int64_t bh0, int hl, float *buf,
-                                                  int lane)
+                                                  int buf_floats, int lane)
 {
-    constexpr int GD4 = G * D / 4;
+    constexpr int U = Math::kUnits;
+    constexpr int UL = (U + 31) / 32;     // units per lane, at most
+    constexpr int SO = piece_stats_off(D, G);
+    constexpr int SU = stats_units(G);
     const int hpc = p.geo.hpc;
     const int x0 = cta_of(segS, C, total);
     const int np = cta_of(segS + ns - 1, C, total) - x0 + 1;
-    const int q = (int)blockIdx.x - x0;
-    const int lo4 = (int)((int64_t)q * GD4 / np);
-    const int S4 = (int)((int64_t)(q + 1) * GD4 / np) - lo4;
-    float *raw = buf;                      // [np][S4] float4
-    float *wbuf = buf + 4 * np * S4;       // [np][G]
+    int lo = 0, S = U;
     T *out = static_cast<T *>(p.out) + bh0 * D;
-
-    // 1. every piece's flag (lane i waits for pieces i, i + 32, ...), its bad
-    //    mark and its (max, sum) per query head, merged per lane
-    bool late = false, bad = false;
-    float M[G], L[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        M[g] = -INFINITY;
-        L[g] = 0.f;
-    }
-    for (int i = lane; i < np; i += 32) {
-        const int slot = piece_slot(x0 + i, i == 0, hpc, hl);
-        if (!ptx::flag_wait_bounded(p.flags + slot, p.epoch, kWaitLimitNs)) {
-            late = true;
-            continue;
-        }
-        const float *ps = p.wpart + (int64_t)slot * p.slot_floats;
-        bad |= __ldcg(ps + 4 * GD4 + 2 * G) != 0.f;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float m = __ldcg(ps + 4 * GD4 + g), l = __ldcg(ps + 4 * GD4 + G + g);
-            wbuf[i * G + g] = m;
-            const float Mn = fmaxf(M[g], m);
-            if (Mn != -INFINITY) {
-                L[g] = L[g] * ptx::ex2(M[g] - Mn) + l * ptx::ex2(m - Mn);
-                M[g] = Mn;
+    if (np > kLastMergesPieces) {
+        const int q = (int)blockIdx.x - x0;
+        lo = (int)((int64_t)q * U / np);
+        S = (int)((int64_t)(q + 1) * U / np) - lo;
+        bool done = false;
+        if (lane == 0) {
+            const unsigned long long want = ((unsigned long long)p.epoch << 32) | (unsigned)np;
+            unsigned long long *c = p.counters + (int64_t)x0 * hpc + hl;
+            const uint64_t t0 = ptx::globaltimer_ns();
+            for (uint32_t i = 0; i < (1u << 26); ++i) {
+                if (ptx::ld_acquire_gpu_u64(c) == want) {
+                    done = true;
+                    break;
+                }
+                __nanosleep(64);
+                if ((i & 15u) == 0 && ptx::globaltimer_ns() - t0 > kWaitLimitNs)
+                    break;
             }
+            if (!done)
+                report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
         }
-    }
-    late = __any_sync(kFull, late);
-    bad = __any_sync(kFull, bad);
-    // the warp barrier orders the lanes' reads below after the acquiring
-    // loads of the flags (the reads bypass L1)
-    __syncwarp();
-    if (late || bad) {
-        if (lane == 0)
-            report(p.dev_status, late ? PA_DEV_WAIT_TIMEOUT : PA_DEV_BAD_BLOCK);
-        for (int e = lane; e < 4 * S4; e += 32)
-            store_out<T>(out + 4 * lo4 + e, 0.f);
-        return;
-    }
-
-    // 2. this participant's slice of every piece, all copies in flight at once
-    const int items = np * S4;
-    const uint32_t raw_s = ptx::smem_u32(raw);
-    for (int f = lane; f < items; f += 32) {
-        const int i = f / S4;
-        const int slot = piece_slot(x0 + i, i == 0, hpc, hl);
-        ptx::cp_async16(raw_s + 16u * (uint32_t)f,
-                        p.wpart + (int64_t)slot * p.slot_floats + 4 * (lo4 + f - i * S4));
-    }
-
-    // 3. meanwhile: butterfly over the lanes (the merge is symmetric, so
-    //    every lane ends with equal values), then weights 2^(m_i - M) / L in
-    //    place of the maxima
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float M2 = __shfl_xor_sync(kFull, M[g], o);
-            const float L2 = __shfl_xor_sync(kFull, L[g], o);
-            const float Mn = fmaxf(M[g], M2);
-            if (Mn != -INFINITY) {
-                L[g] = L[g] * ptx::ex2(M[g] - Mn) + L2 * ptx::ex2(M2 - Mn);
-                M[g] = Mn;
+        done = __shfl_sync(kFull, done, 0);
+        // the warp barrier orders the lanes' copies below after lane 0's
+        // acquiring load (the copies bypass L1)
+        __syncwarp();
+        if (!done) {
+            for (int f = lane; f < 4 * S; f += 32) {
+                int g, d;
+                Math::unit_coords(lo + (f >> 2), f & 3, g, d);
+                if (g < G)
+                    store_out<T>(out + g * D + d, 0.f);
             }
+            return;
         }
     }
-    for (int i = lane; i < np; i += 32) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float m = wbuf[i * G + g];
-            wbuf[i * G + g] = (m == -INFINITY || !(L[g] > 0.f)) ? 0.f : ptx::ex2(m - M[g]) / L[g];
+    float *st = buf;                      // [np][SU] float4
+    float *w = st + 4 * np * SU;          // [np][G]
+    float *tot = w + np * G;              // [G] M, [G] L
+    float *raw = buf + ((4 * np * SU + np * G + 2 * G + 3) & ~3);   // [CP][S] float4
+    const int CP = max(1, (buf_floats - (int)(raw - buf)) / (4 * max(S, 1)));
+    auto src = [&](int i) {
+        return p.wpart + (int64_t)piece_slot(x0 + i, i == 0, hpc, hl) * p.slot_floats;
+    };
+    auto copy_units = [&](int i0, int i1) {
+        for (int f = lane; f < (i1 - i0) * S; f += 32) {
+            const int i = f / S;
+            ptx::cp_async16(ptx::smem_u32(raw + 4 * f), src(i0 + i) + 4 * (lo + f - i * S));
         }
+    };
+
+    // 1. every piece's stats and the first round of units
+    for (int f = lane; f < np * SU; f += 32) {
+        const int i = f / SU;
+        ptx::cp_async16(ptx::smem_u32(st + 4 * f), src(i) + SO + 4 * (f - i * SU));
     }
+    int i1 = min(np, CP);
+    copy_units(0, i1);
     ptx::cp_async_wait_all();
     __syncwarp();
 
-    // 4. weighted sums in piece order, four consecutive outputs per lane step
-    const float4 *raw4 = reinterpret_cast<const float4 *>(raw);
-    for (int e = lane; e < S4; e += 32) {
-        const int idx = 4 * (lo4 + e);
-        const int g = idx / D;
-        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int i = 0; i < np; ++i) {
-            const float w = wbuf[i * G + g];
-            const float4 v = raw4[i * S4 + e];
-            o.x = fmaf(w, v.x, o.x);
-            o.y = fmaf(w, v.y, o.y);
-            o.z = fmaf(w, v.z, o.z);
-            o.w = fmaf(w, v.w, o.w);
+    bool bad = false;
+    for (int i = lane; i < np; i += 32)
+        bad |= st[i * 4 * SU + 2 * G] != 0.f;
+    if (__any_sync(kFull, bad)) {
+        if (lane == 0)
+            report(p.dev_status, PA_DEV_BAD_BLOCK);
+        for (int f = lane; f < 4 * S; f += 32) {
+            int g, d;
+            Math::unit_coords(lo + (f >> 2), f & 3, g, d);
+            if (g < G)
+                store_out<T>(out + g * D + d, 0.f);
         }
-        store4(out + idx, o);
+        return;
+    }
+
+    // 2. per-head totals (lane g, pieces in order), then the weights
+    if (lane < G) {
+        float M = -INFINITY, L = 0.f;
+        for (int i = 0; i < np; ++i)
+            M = fmaxf(M, st[i * 4 * SU + lane]);
+        if (M != -INFINITY)
+            for (int i = 0; i < np; ++i) {
+                const float mi = st[i * 4 * SU + lane];
+                if (mi != -INFINITY)
+                    L = fmaf(st[i * 4 * SU + G + lane], ptx::ex2(mi - M), L);
+            }
+        tot[lane] = M;
+        tot[G + lane] = L;
+    }
+    __syncwarp();
+    for (int f = lane; f < np * G; f += 32) {
+        const int i = f / G, g = f - i * G;
+        const float mi = st[i * 4 * SU + g], M = tot[g], L = tot[G + g];
+        w[f] = (mi == -INFINITY || !(L > 0.f)) ? 0.f : ptx::ex2(mi - M) / L;
+    }
+    __syncwarp();
+
+    // 3. weighted sums in piece order: the lane holds units lo + lane + 32 t
+    float o[UL][4];
+#pragma unroll
+    for (int t = 0; t < UL; ++t)
+        o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+    const float4 *raw4 = reinterpret_cast<const float4 *>(raw);
+    for (int i0 = 0; i0 < np;) {
+#pragma unroll
+        for (int t = 0; t < UL; ++t) {
+            const int e = lane + 32 * t;
+            if (e < S) {
+                int gw[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    int d;
+                    Math::unit_coords(lo + e, j, gw[j], d);
+                    gw[j] = min(gw[j], G - 1);   // padding heads read a real weight
+                }
+                for (int i = i0; i < i1; ++i) {
+                    const float4 v = raw4[(i - i0) * S + e];
+                    const float *wi = w + i * G;
+                    o[t][0] = fmaf(wi[gw[0]], v.x, o[t][0]);
+                    o[t][1] = fmaf(wi[gw[1]], v.y, o[t][1]);
+                    o[t][2] = fmaf(wi[gw[2]], v.z, o[t][2]);
+                    o[t][3] = fmaf(wi[gw[3]], v.w, o[t][3]);
+                }
+            }
+        }
+        i0 = i1;
+        if (i0 < np) {
+            i1 = min(np, i0 + CP);
+            __syncwarp();
+            copy_units(i0, i1);
+            ptx::cp_async_wait_all();
+            __syncwarp();
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < UL; ++t) {
+        const int e = lane + 32 * t;
+        if (e < S) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                int g, d;
+                Math::unit_coords(lo + e, j, g, d);
+                if (g < G)
+                    store_out<T>(out + g * D + d, o[t][j]);
+            }
+        }
     }
     __syncwarp();
 }
@@ -977,12 +1149,14 @@ __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, 
 //
 // Mode 0 cuts segments at range borders and merges them inside the kernel.
 // Each CTA holding a piece of a cut segment publishes the piece's partial
-// state (acc [G][D], max [G], sum [G], bad) in its slot with a release store
-// of the call's epoch to the slot's flag, when it reaches the piece's end.
-// After its whole range, each such CTA merges its share of the segment's
-// outputs (merge_cut_segment).  A CTA waits only after all of its own pieces
-// are published and every CTA of the persistent grid is resident, so every
-// wait ends; each is bounded all the same.
+// state (acc, max, sum, bad) in its slot, then counts itself in at the
+// segment's counter with an acquire-release atomic add.  A segment of a few
+// pieces is merged, after its range, by the warp whose arrival completed the
+// count; everyone else moves on.  A segment of many pieces is merged by all
+// of its CTAs, each a slice, after waiting for the count (merge_cut_segment).
+// A CTA waits only after its range, when all of its own pieces are counted
+// in, and every CTA of the persistent grid is resident, so every wait ends;
+// each is bounded all the same.
 //
 // Nothing touches global memory before griddepcontrol.wait: the kernel is
 // launched as a programmatic dependent of the kernel before it on the stream.
@@ -1159,10 +1333,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     int segS = 0;          // global index of the current segment's first tile
     bool seg_bad = false;
     bool timed_out = false;
-    // cut segments this warp holds a piece of (mode 0): a later piece met at
-    // the start of the range, and the first piece of one that runs past its end
+    // cut segments this warp merges (mode 0): one met at the start of the
+    // range, one that runs past its end
     int laterS = -1, laterN = 0, laterB = 0, laterHG = 0;
     int firstS = -1, firstN = 0, firstB = 0, firstHG = 0;
+
+    // this CTA's arrival counters start the call at (epoch, 0)
+    if (p.mode == 0 && lane == 0)
+        ptx::st_relaxed_gpu_u64(p.counters + (int64_t)blockIdx.x * hpc + hl,
+                                (unsigned long long)p.epoch << 32);
 
     for (int i = R0; i < R1; ++i) {
         const int k = i - R0;
@@ -1227,19 +1406,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool first = segS >= R0;
                 const int slot = piece_slot(blockIdx.x, first, hpc, hl);
                 float *ps = p.wpart + (int64_t)slot * p.slot_floats;
-                math.for_each(
-                    lane, [&](int hh, int e, float v, float) { ps[hh * D + e] = v; },
-                    [&](int hh, float mm, float ll) {
-                        ps[G * D + hh] = mm;
-                        ps[G * D + G + hh] = ll;
-                    });
+                math.publish(ps, lane);
+                math.publish_stats(ps + piece_stats_off(D, G), lane);
                 if (lane == 0)
-                    ps[G * D + 2 * G] = seg_bad ? 1.f : 0.f;
+                    ps[piece_stats_off(D, G) + 2 * G] = seg_bad ? 1.f : 0.f;
                 // the warp barrier orders every lane's stores before lane 0's
-                // release of the flag
+                // release (the counter update)
                 __syncwarp();
+                const int x0 = cta_of(segS, C, total);
+                int arrived = 0;
                 if (lane == 0)
-                    ptx::st_release_gpu(p.flags + slot, p.epoch);
+                    arrived = segment_arrive(p.counters + (int64_t)x0 * hpc + hl, p.epoch);
+                arrived = __shfl_sync(kFull, arrived, 0);
+                __syncwarp();
+                if (arrived == 0) {
+                    if (lane == 0)
+                        report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+                    continue;
+                }
+                const int np = cta_of(segS + d.ns - 1, C, total) - x0 + 1;
+                if (np <= kLastMergesPieces && arrived != np)
+                    continue;   // a later arrival merges the segment
                 if (first) {
                     firstS = segS;
                     firstN = d.ns;
@@ -1288,14 +1475,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             return;
         float *buf = reinterpret_cast<float *>(
             sgen + (int64_t)hl * ((int64_t)stages_bytes / hpc & ~(int64_t)15));
+        const int buf_floats = (int)((int64_t)stages_bytes / hpc / 4) & ~3;
         if (laterS >= 0)
-            merge_cut_segment<T, D, G>(p, C, total, laterS, laterN,
-                                       (int64_t)laterB * Hq + (int64_t)(laterHG * hpc + hl) * G,
-                                       hl, buf, lane);
+            merge_cut_segment<T, D, G, Math>(
+                p, C, total, laterS, laterN,
+                (int64_t)laterB * Hq + (int64_t)(laterHG * hpc + hl) * G, hl, buf, buf_floats, lane);
         if (firstS >= 0)
-            merge_cut_segment<T, D, G>(p, C, total, firstS, firstN,
-                                       (int64_t)firstB * Hq + (int64_t)(firstHG * hpc + hl) * G,
-                                       hl, buf, lane);
+            merge_cut_segment<T, D, G, Math>(
+                p, C, total, firstS, firstN,
+                (int64_t)firstB * Hq + (int64_t)(firstHG * hpc + hl) * G, hl, buf, buf_floats, lane);
     }
 }
 

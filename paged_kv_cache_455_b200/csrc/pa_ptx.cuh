@@ -69,33 +69,36 @@ __device__ __forceinline__ void grid_wait_prerequisites()
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// ------------------------------------------------- cross-CTA flags (gpu scope)
-__device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v)
+// ------------------------------------------- cross-CTA counters (gpu scope)
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned long long *p)
 {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 
-// Waits until *p == v.  Gives up after limit_ns nanoseconds and returns false.
-__device__ __forceinline__ bool flag_wait_bounded(const uint32_t *p, uint32_t v, uint64_t limit_ns)
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long *p)
 {
-    if (ld_acquire_gpu(p) == v)
-        return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1; i < (1u << 26); ++i) {
-        __nanosleep(64);
-        if (ld_acquire_gpu(p) == v)
-            return true;
-        if ((i & 15u) == 0 && globaltimer_ns() - t0 > limit_ns)
-            return false;
-    }
-    return false;
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Atomic add with acquire-release semantics at gpu scope; returns the old value.
+__device__ __forceinline__ unsigned long long atom_add_acq_rel_gpu(unsigned long long *p,
+                                                                   unsigned long long v)
+{
+    unsigned long long old;
+    asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;"
+                 : "=l"(old)
+                 : "l"(p), "l"(v)
+                 : "memory");
+    return old;
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
