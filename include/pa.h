@@ -187,6 +187,27 @@ pa_status pa_splitk_reduce(void *out, const float *tmp_out, const float *max_log
                            int max_partitions, pa_dtype dtype, void *stream);
 
 /*
+ * pa_copy_blocks -- copy whole physical blocks of both pools, the copy that
+ * copy-on-write block sharing needs ("vLLM Architecture, Memory and
+ * Benchmarks Deep Dive", section 2, "Copy-on-Write (CoW) Branching": rollouts
+ * of one prompt share its blocks, and a block is cloned only when the
+ * sequences sharing it diverge).
+ *
+ * For every pair i: block block_mapping[2i + 1] of k_pool and of v_pool
+ * becomes a bit-exact copy of block block_mapping[2i].
+ *   block_mapping  device, [num_pairs][2] int64 (source, destination).
+ *                  Destinations must be distinct and must not be the source
+ *                  of another pair of the same call (the copies run
+ *                  concurrently).
+ *   k_pool,v_pool  device, [nb, bs, Hkv, d] in `dtype`.
+ * A source or destination outside [0, nb) sets PA_DEV_BAD_BLOCK and that
+ * pair is skipped.  num_pairs == 0 launches nothing.
+ */
+pa_status pa_copy_blocks(void *k_pool, void *v_pool, const int64_t *block_mapping, int num_pairs,
+                         int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                         pa_dtype dtype, int32_t *dev_status, void *stream);
+
+/*
  * pa_decode_attention_static -- pa_decode_attention for callers that cannot
  * allocate device memory.  The pages have no counterpart to this call; it is
  * an addition of this library.

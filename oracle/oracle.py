@@ -172,6 +172,23 @@ def reshape_and_cache_np(key, value, k_pool, v_pool, slot_mapping):
     return k_out, v_out
 
 
+def copy_blocks_np(k_pool, v_pool, block_mapping):
+    """Returns new (k_pool, v_pool) in which block dst of each (src, dst) pair
+    of block_mapping [P, 2] holds block src of the input pools, read before
+    any copy (the copy copy-on-write sharing needs: "vLLM Architecture, Memory
+    and Benchmarks Deep Dive", section 2, "Copy-on-Write (CoW) Branching").
+    Raises ValueError for a block id outside the pool."""
+    k_in, v_in = np.asarray(k_pool), np.asarray(v_pool)
+    k_out, v_out = np.array(k_in, copy=True), np.array(v_in, copy=True)
+    nb = k_in.shape[0]
+    for src, dst in np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2):
+        if not (0 <= src < nb and 0 <= dst < nb):
+            raise ValueError("block id outside the pool")
+        k_out[dst] = k_in[src]
+        v_out[dst] = v_in[src]
+    return k_out, v_out
+
+
 # --------------------------------------------------------------------------
 # Attention (C, fp64)
 # --------------------------------------------------------------------------

@@ -95,6 +95,40 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const CacheParams p)
         dst[c] = __ldg(src + c);
 }
 
+struct CopyParams {
+    void *k_pool;
+    void *v_pool;
+    const int64_t *block_mapping;   // [num_pairs][2]: source, destination
+    int32_t *dev_status;
+    int64_t num_blocks;
+    int64_t block_bytes;            // bs * Hkv * d * element size
+    int num_pairs;
+};
+
+// One CTA per (pair, pool, 8 KB chunk of the block): 16-byte copies, 512
+// bytes per warp instruction.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p, int chunks)
+{
+    const int pair = blockIdx.x / (2 * chunks);
+    const int rest = blockIdx.x - pair * 2 * chunks;
+    const int kv = rest / chunks;
+    const int chunk = rest - kv * chunks;
+    const int64_t src = p.block_mapping[2 * pair];
+    const int64_t dst = p.block_mapping[2 * pair + 1];
+    if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {
+        if (threadIdx.x == 0 && kv == 0 && chunk == 0)
+            pa::report(p.dev_status, PA_DEV_BAD_BLOCK);
+        return;
+    }
+    uint8_t *pool = static_cast<uint8_t *>(kv ? p.v_pool : p.k_pool);
+    const int4 *from = reinterpret_cast<const int4 *>(pool + src * p.block_bytes);
+    int4 *to = reinterpret_cast<int4 *>(pool + dst * p.block_bytes);
+    const int64_t n16 = p.block_bytes >> 4;
+    const int64_t end = min(n16, (int64_t)(chunk + 1) * 512);
+    for (int64_t c = (int64_t)chunk * 512 + threadIdx.x; c < end; c += 256)
+        to[c] = __ldcg(from + c);
+}
+
 // =====================================================================
 // Tensor maps
 // =====================================================================
@@ -529,6 +563,39 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_pool,
     if (blocks > INT32_MAX)
         return PA_ERR_INVALID_ARG;
     cache_write_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    ++g_launches;
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks(void *k_pool, void *v_pool, const int64_t *block_mapping, int num_pairs,
+                         int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                         pa_dtype dtype, int32_t *dev_status, void *stream)
+{
+    if (num_pairs < 0 || num_blocks <= 0 || num_kv_heads <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (dtype != PA_DTYPE_F32 && dtype != PA_DTYPE_BF16)
+        return PA_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+        return PA_ERR_UNSUPPORTED;
+    if (ilog2_exact(block_size) < 0 || block_size < 4 || block_size > 32)
+        return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0)
+        return PA_OK;
+    if (!k_pool || !v_pool || !block_mapping)
+        return PA_ERR_INVALID_ARG;
+    CopyParams p;
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.block_mapping = block_mapping;
+    p.dev_status = dev_status;
+    p.num_blocks = num_blocks;
+    p.block_bytes = (int64_t)block_size * num_kv_heads * head_dim * elem_size(dtype);
+    p.num_pairs = num_pairs;
+    const int chunks = (int)((p.block_bytes + 8191) / 8192);
+    const int64_t blocks = (int64_t)num_pairs * 2 * chunks;
+    if (blocks > INT32_MAX)
+        return PA_ERR_INVALID_ARG;
+    copy_blocks_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p, chunks);
     ++g_launches;
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

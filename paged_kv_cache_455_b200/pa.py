@@ -46,6 +46,7 @@ SIGNATURES = {
     "pa_splitk_reduce": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "pa_decode_attention_static": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                                         _I64, _F, _I, _P, _P]),
+    "pa_copy_blocks": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _I, _P, _P]),
     "pa_status_string": (ctypes.c_char_p, [_I]),
     "pa_launch_count": (ctypes.c_ulonglong, []),
 }
@@ -125,6 +126,20 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_pool: torch.T
     _check(lib.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_pool), _ptr(v_pool),
                                     _ptr(slot_mapping), T, hkv, d, bs, nb, _dtype_code(key),
                                     _ptr(dev_status), _stream(stream)), "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, block_mapping: torch.Tensor,
+                   dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """pools [nb, bs, Hkv, d]; block_mapping [P, 2] int64 (source, destination)."""
+    _cuda(k_pool, v_pool, block_mapping, dev_status)
+    nb, bs, hkv, d = k_pool.shape
+    if v_pool.shape != k_pool.shape or v_pool.dtype != k_pool.dtype:
+        raise ValueError("pool mismatch")
+    if block_mapping.dtype != torch.int64 or block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
+        raise ValueError("block_mapping must be int64 [P, 2]")
+    _check(lib.pa_copy_blocks(_ptr(k_pool), _ptr(v_pool), _ptr(block_mapping),
+                              block_mapping.shape[0], nb, bs, hkv, d, _dtype_code(k_pool),
+                              _ptr(dev_status), _stream(stream)), "pa_copy_blocks")
 
 
 def _attn_sizes(out, query, k_pool, v_pool, block_tables, context_lens):
@@ -218,7 +233,7 @@ def pa_splitk_reduce(out: torch.Tensor, tmp_out: torch.Tensor, max_logits: torch
 
 __all__ = [
     "lib", "LIB_PATH", "SIGNATURES", "PaError", "launch_count",
-    "pa_reshape_and_cache", "pa_decode_attention", "pa_decode_workspace_bytes",
+    "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode_attention", "pa_decode_workspace_bytes",
     "pa_decode_attention_static", "PA_STATIC_SCRATCH_BYTES",
     "pa_num_partitions", "pa_splitk_workspace_bytes", "pa_decode_splitk", "pa_splitk_reduce",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA", "PA_ERR_WORKSPACE",

@@ -130,6 +130,25 @@ def test_reshape_and_cache_host_validation(pa):
     assert call(T=0, key=None) == 0
 
 
+def test_copy_blocks_host_validation(pa):
+    L = pa.lib
+
+    def call(**kw):
+        a = dict(kp=A, vp=A, mapping=A, n=2, nb=16, bs=16, hkv=4, d=256, dt=1)
+        a.update(kw)
+        return L.pa_copy_blocks(a["kp"], a["vp"], a["mapping"], a["n"], a["nb"], a["bs"],
+                                a["hkv"], a["d"], a["dt"], None, None)
+    assert call(n=-1) == 1
+    assert call(nb=0) == 1
+    assert call(hkv=0) == 1
+    assert call(d=100) == 2
+    assert call(bs=12) == 2
+    assert call(dt=5) == 2
+    assert call(mapping=None) == 1
+    assert call(kp=None) == 1
+    assert call(n=0, kp=None, vp=None, mapping=None) == 0   # nothing to copy: no launch
+
+
 def test_binding_rejects_cpu_tensors(pa):
     import torch
     x = torch.zeros(3, 8, 64)
