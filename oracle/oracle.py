@@ -337,3 +337,48 @@ __all__ = [
     "paged_attention", "partition_attention", "merge_partitions", "threads", "to_f64",
     "gather_np", "paged_attention_np", "partition_attention_np",
 ]
+
+
+# --------------------------------------------------------------------------
+# Chunked prefill (numpy, fp64)
+# --------------------------------------------------------------------------
+
+def prefill_attention_np(q, k_pool, v_pool, block_tables, context_lens, cu_q_lens, scale: float,
+                         dtype: str) -> np.ndarray:
+    """Exact fp64 attention of a chunk of query tokens per sequence over its
+    paged cache, causal within the chunk; returns [total_q, Hq, d] float64.
+
+    Sequence b's chunk is query rows cu_q_lens[b] .. cu_q_lens[b + 1] - 1
+    (n_b rows); context_lens[b] counts every cached token including the
+    chunk, so chunk row j sits at position p = ctx_b - n_b + j and attends to
+    the keys at positions 0 .. p, reached through the block table ("vLLM
+    Architecture, Memory and Benchmarks Deep Dive", section 4, chunked
+    prefill; section 2, block table).  Query head hq uses KV head
+    hq // (Hq // Hkv).  A chunk longer than its context raises ValueError.
+    """
+    qf = to_f64(q, dtype)
+    kf = to_f64(k_pool, dtype)
+    vf = to_f64(v_pool, dtype)
+    hq, d = qf.shape[1], qf.shape[2]
+    hkv = kf.shape[2]
+    group = hq // hkv
+    out = np.zeros(qf.shape, dtype=np.float64)
+    cu = np.asarray(cu_q_lens, dtype=np.int64)
+    for b in range(len(context_lens)):
+        ctx, q0, n = int(context_lens[b]), int(cu[b]), int(cu[b + 1] - cu[b])
+        if n == 0:
+            continue
+        if n > ctx:
+            raise ValueError("chunk longer than its context")
+        kc = gather_np(kf, block_tables[b], ctx)          # [ctx, Hkv, d]
+        vc = gather_np(vf, block_tables[b], ctx)
+        pos = ctx - n + np.arange(n)                       # positions of the chunk rows
+        allowed = np.arange(ctx)[None, :] <= pos[:, None]  # [n, ctx] causal
+        for h in range(hq):
+            kh, vh = kc[:, h // group], vc[:, h // group]
+            s = scale * (qf[q0:q0 + n, h] @ kh.T)          # [n, ctx]
+            s = np.where(allowed, s, -np.inf)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            out[q0:q0 + n, h] = (p @ vh) / p.sum(axis=1, keepdims=True)
+    return out
+
