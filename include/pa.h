@@ -187,6 +187,36 @@ pa_status pa_splitk_reduce(void *out, const float *tmp_out, const float *max_log
                            int max_partitions, pa_dtype dtype, void *stream);
 
 /*
+ * pa_prefill_attention -- chunked prefill over the paged cache: a chunk of
+ * query tokens per sequence attends, causally, to everything the sequence
+ * has cached ("vLLM Architecture, Memory and Benchmarks Deep Dive",
+ * section 4, "Chunked Prefill": long prompts are cut into chunks, e.g. 512
+ * tokens, that run beside decode; section 2: the block table).
+ *
+ * Sequence b's chunk is query rows cu_q_lens[b] .. cu_q_lens[b + 1] - 1
+ * (n_b rows); context_lens[b] counts every cached token including the chunk
+ * (whose K/V pa_reshape_and_cache has already written), so chunk row j sits
+ * at position ctx_b - n_b + j and attends to the keys at positions 0 .. that
+ * position.  Query head hq uses KV head hq / (Hq / Hkv).
+ *   out            device, [total_q, Hq, d] bf16, written (rows of every chunk).
+ *   query          device, [total_q, Hq, d] bf16.
+ *   cu_q_lens      device, [num_seqs + 1] int32, non-decreasing from 0.
+ *   max_q_len      host hint, >= every n_b, <= max_context_len.
+ *   other arguments as in pa_decode_attention.
+ * bf16 only (fp32 returns PA_ERR_UNSUPPORTED); group 1, 2, 4 or 8; contexts
+ * up to 2048 blocks.  A chunk longer than its context, a context beyond the
+ * table, or rows outside [0, total_q) set PA_DEV_BAD_CONTEXT (its rows that
+ * exist are zeros); an invalid block id sets PA_DEV_BAD_BLOCK (zeros).
+ */
+pa_status pa_prefill_attention(void *out, const void *query, const int32_t *cu_q_lens, int total_q,
+                               int max_q_len, const void *k_pool, const void *v_pool,
+                               const int32_t *block_tables, int max_blocks_per_seq,
+                               const int32_t *context_lens, int num_seqs, int max_context_len,
+                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                               int64_t num_blocks, float scale, pa_dtype dtype,
+                               int32_t *dev_status, void *stream);
+
+/*
  * pa_copy_blocks -- copy whole physical blocks of both pools, the copy that
  * copy-on-write block sharing needs ("vLLM Architecture, Memory and
  * Benchmarks Deep Dive", section 2, "Copy-on-Write (CoW) Branching": rollouts

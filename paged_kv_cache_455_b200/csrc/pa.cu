@@ -21,6 +21,7 @@
 
 #include "pa.h"
 #include "pa_launch.cuh"
+#include "pa_prefill.cuh"
 
 namespace {
 
@@ -598,6 +599,78 @@ pa_status pa_copy_blocks(void *k_pool, void *v_pool, const int64_t *block_mappin
     copy_blocks_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p, chunks);
     ++g_launches;
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_prefill_attention(void *out, const void *query, const int32_t *cu_q_lens, int total_q,
+                               int max_q_len, const void *k_pool, const void *v_pool,
+                               const int32_t *block_tables, int max_blocks_per_seq,
+                               const int32_t *context_lens, int num_seqs, int max_context_len,
+                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                               int64_t num_blocks, float scale, pa_dtype dtype,
+                               int32_t *dev_status, void *stream)
+{
+    if (num_seqs < 0 || total_q < 0 || max_q_len < 0 || max_context_len < 0 ||
+        num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
+        num_q_heads % num_kv_heads != 0)
+        return PA_ERR_INVALID_ARG;
+    if (dtype != PA_DTYPE_BF16)
+        return PA_ERR_UNSUPPORTED;
+    const int group = num_q_heads / num_kv_heads;
+    const int bs_log2 = ilog2_exact(block_size);
+    if ((head_dim != 64 && head_dim != 128 && head_dim != 256) || bs_log2 < 2 || bs_log2 > 5 ||
+        (group != 1 && group != 2 && group != 4 && group != 8))
+        return PA_ERR_UNSUPPORTED;
+    if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size ||
+        max_q_len > std::max(max_context_len, 0))
+        return PA_ERR_INVALID_ARG;
+    if ((int64_t)max_context_len > (int64_t)pa::kPfMaxBlocks * block_size)
+        return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || total_q == 0 || max_q_len == 0)
+        return PA_OK;
+    if (!out || !query || !cu_q_lens || !k_pool || !v_pool || !block_tables || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(query) || !aligned16(k_pool) || !aligned16(v_pool))
+        return PA_ERR_INVALID_ARG;
+    pa::PrefillParams p;
+    p.out = out;
+    p.q = query;
+    p.cu_q_lens = cu_q_lens;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.dev_status = dev_status;
+    p.num_blocks = num_blocks;
+    p.total_q = total_q;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.max_blocks = max_blocks_per_seq;
+    p.block_size = block_size;
+    p.bs_log2 = bs_log2;
+    p.tr = std::min(16, block_size);
+    p.tr_log2 = ilog2_exact(p.tr);
+    p.ctx_cap = std::min(max_blocks_per_seq, pa::kPfMaxBlocks) * block_size;
+    const int tq = pa::kPfRows / group;
+    p.qblocks = (max_q_len + tq - 1) / tq;
+    p.box_stride = pa::prefill_box_stride(p.tr, head_dim);
+    const int stage = pa::prefill_stage_bytes(p.tr, head_dim);
+    const int fixed = pa::prefill_fixed_bytes(head_dim);
+    p.stages = std::min(pa::kPfMaxStages, (pa::kSmemBudget - fixed) / stage);
+    if (p.stages < 2)
+        return PA_ERR_UNSUPPORTED;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const int smem = fixed + p.stages * stage;
+    const int64_t grid = (int64_t)num_seqs * num_kv_heads * p.qblocks;
+    if (grid > INT32_MAX)
+        return PA_ERR_INVALID_ARG;
+    CUtensorMap tk, tv;
+    if (!encode_pool_map(&tk, k_pool, num_blocks, block_size, num_kv_heads, head_dim, dtype, p.tr,
+                         1) ||
+        !encode_pool_map(&tv, v_pool, num_blocks, block_size, num_kv_heads, head_dim, dtype, p.tr,
+                         1))
+        return PA_ERR_CUDA;
+    const pa_status st = pa::prefill_dispatch(head_dim, group, tk, tv, p, (int)grid, smem,
+                                              static_cast<cudaStream_t>(stream));
+    ++g_launches;
+    return st;
 }
 
 pa_status pa_decode_splitk(void *out, const void *query, const void *k_pool, const void *v_pool,

@@ -130,4 +130,9 @@ pa_status decode_f32(DecodeLaunch &L, int *grid, bool launch);
 pa_status decode_bf16_mma(DecodeLaunch &L, int *grid, bool launch);
 pa_status decode_bf16_simt(DecodeLaunch &L, int *grid, bool launch);
 
+// Chunked prefill (pa_inst_prefill.cu).
+struct PrefillParams;
+pa_status prefill_dispatch(int head_dim, int group, const CUtensorMap &tk, const CUtensorMap &tv,
+                           const PrefillParams &p, int grid, int smem, cudaStream_t stream);
+
 }  // namespace pa

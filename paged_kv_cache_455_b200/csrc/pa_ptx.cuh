@@ -204,6 +204,14 @@ __device__ __forceinline__ uint64_t policy_evict_first()
     return pol;
 }
 
+// Normal eviction priority (data other CTAs will read again soon).
+__device__ __forceinline__ uint64_t policy_evict_normal()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // ------------------------------------------------------ matrix fragments
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
 {

@@ -47,6 +47,8 @@ SIGNATURES = {
     "pa_decode_attention_static": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                                         _I64, _F, _I, _P, _P]),
     "pa_copy_blocks": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _I, _P, _P]),
+    "pa_prefill_attention": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
+                                  _I, _I64, _F, _I, _P, _P]),
     "pa_status_string": (ctypes.c_char_p, [_I]),
     "pa_launch_count": (ctypes.c_ulonglong, []),
 }
@@ -142,6 +144,35 @@ def pa_copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, block_mapping: to
                               _ptr(dev_status), _stream(stream)), "pa_copy_blocks")
 
 
+def pa_prefill_attention(out: torch.Tensor, query: torch.Tensor, cu_q_lens: torch.Tensor,
+                         max_q_len: int, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                         block_tables: torch.Tensor, context_lens: torch.Tensor,
+                         max_context_len: int, scale: float,
+                         dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """query/out [total_q, Hq, d] bf16; cu_q_lens [B + 1] int32; pools
+    [nb, bs, Hkv, d]; block_tables [B, max_blocks] int32; context_lens [B] int32."""
+    _cuda(out, query, cu_q_lens, k_pool, v_pool, block_tables, context_lens, dev_status)
+    total_q, hq, d = query.shape
+    nb, bs, hkv, d2 = k_pool.shape
+    B = context_lens.shape[0]
+    if out.shape != query.shape or v_pool.shape != k_pool.shape or d2 != d:
+        raise ValueError("shape mismatch")
+    if cu_q_lens.dtype != torch.int32 or cu_q_lens.shape != (B + 1,):
+        raise ValueError("cu_q_lens must be int32 [B + 1]")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("block_tables must be int32 [B, max_blocks]")
+    if context_lens.dtype != torch.int32:
+        raise ValueError("context_lens must be int32 [B]")
+    if not (out.dtype == query.dtype == k_pool.dtype == v_pool.dtype):
+        raise ValueError("dtype mismatch")
+    _check(lib.pa_prefill_attention(_ptr(out), _ptr(query), _ptr(cu_q_lens), total_q,
+                                    int(max_q_len), _ptr(k_pool), _ptr(v_pool),
+                                    _ptr(block_tables), block_tables.shape[1],
+                                    _ptr(context_lens), B, int(max_context_len), hq, hkv, d, bs,
+                                    nb, float(scale), _dtype_code(query), _ptr(dev_status),
+                                    _stream(stream)), "pa_prefill_attention")
+
+
 def _attn_sizes(out, query, k_pool, v_pool, block_tables, context_lens):
     _cuda(out, query, k_pool, v_pool, block_tables, context_lens)
     B, hq, d = query.shape
@@ -233,7 +264,7 @@ def pa_splitk_reduce(out: torch.Tensor, tmp_out: torch.Tensor, max_logits: torch
 
 __all__ = [
     "lib", "LIB_PATH", "SIGNATURES", "PaError", "launch_count",
-    "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode_attention", "pa_decode_workspace_bytes",
+    "pa_reshape_and_cache", "pa_copy_blocks", "pa_prefill_attention", "pa_decode_attention", "pa_decode_workspace_bytes",
     "pa_decode_attention_static", "PA_STATIC_SCRATCH_BYTES",
     "pa_num_partitions", "pa_splitk_workspace_bytes", "pa_decode_splitk", "pa_splitk_reduce",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA", "PA_ERR_WORKSPACE",

@@ -149,6 +149,31 @@ def test_copy_blocks_host_validation(pa):
     assert call(n=0, kp=None, vp=None, mapping=None) == 0   # nothing to copy: no launch
 
 
+def test_prefill_host_validation(pa):
+    L = pa.lib
+
+    def call(**kw):
+        a = dict(out=A, q=A, cu=A, total=10, maxq=8, kp=A, vp=A, tab=A, maxb=4, lens=A, B=2,
+                 maxctx=64, hq=16, hkv=4, d=256, bs=16, nb=32, dt=1)
+        a.update(kw)
+        return L.pa_prefill_attention(a["out"], a["q"], a["cu"], a["total"], a["maxq"], a["kp"],
+                                      a["vp"], a["tab"], a["maxb"], a["lens"], a["B"],
+                                      a["maxctx"], a["hq"], a["hkv"], a["d"], a["bs"], a["nb"],
+                                      0.0625, a["dt"], None, None)
+    assert call(dt=0) == 2                  # fp32: not built
+    assert call(hq=12) == 2                 # group 3
+    assert call(d=96) == 2
+    assert call(bs=12) == 2
+    assert call(hq=15) == 1                 # Hq % Hkv != 0
+    assert call(maxctx=65) == 1             # beyond the table
+    assert call(maxq=65, maxctx=64) == 1    # chunk longer than any context
+    assert call(maxb=4096, maxctx=40000) == 2   # more than 2048 blocks
+    assert call(cu=None) == 1
+    assert call(out=M) == 1
+    assert call(B=0, out=None) == 0         # nothing to do: no launch
+    assert call(maxq=0, out=None) == 0
+
+
 def test_binding_rejects_cpu_tensors(pa):
     import torch
     x = torch.zeros(3, 8, 64)
