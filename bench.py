@@ -486,6 +486,140 @@ def run_reference(args, rank, world, device):
 
 
 # ---------------------------------------------------------------------------
+# chunked prefill (--path prefill)
+# ---------------------------------------------------------------------------
+
+PREFILL_METRIC = "chunked-prefill paged attention TFLOP/s (causal flops)"
+
+
+def prefill_workload(device, layers: int, seed: int = 455 + 6):
+    """Qwen-shaped heads (Hq=16, Hkv=4, d=256, bs=16, bf16): B=16 sequences whose
+    contexts are uniform in [1024, 4096] tokens, each ending with a 512-token
+    chunk (the pages' example chunk size), one pool per layer."""
+    rng = np.random.default_rng(seed)
+    B, hq, hkv, d, bs, chunk = 16, 16, 4, 256, 16, 512
+    lens = rng.integers(1024, 4097, size=B).astype(np.int32)
+    need = -(-lens // bs)
+    nb = int(need.sum()) + 64
+    perm = rng.permutation(nb)
+    tables = np.full((B, int(need.max())), -1, np.int32)
+    pos = 0
+    for b in range(B):
+        tables[b, :need[b]] = perm[pos:pos + need[b]]
+        pos += need[b]
+    slots = np.concatenate([tables[b][np.arange(lens[b] - chunk, lens[b]) // bs] * bs +
+                            np.arange(lens[b] - chunk, lens[b]) % bs for b in range(B)])
+    cu = np.arange(B + 1, dtype=np.int32) * chunk
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    L = []
+    for _ in range(layers):
+        kp = torch.randn(nb, bs, hkv, d, generator=g, device=device).to(torch.bfloat16)
+        vp = torch.randn(nb, bs, hkv, d, generator=g, device=device).to(torch.bfloat16)
+        q = torch.randn(B * chunk, hq, d, generator=g, device=device).to(torch.bfloat16)
+        key = torch.randn(B * chunk, hkv, d, generator=g, device=device).to(torch.bfloat16)
+        val = torch.randn(B * chunk, hkv, d, generator=g, device=device).to(torch.bfloat16)
+        L.append((q, key, val, kp, vp, torch.empty_like(q)))
+    dev = dict(tables=torch.from_numpy(tables).to(device), lens=torch.from_numpy(lens).to(device),
+               slots=torch.from_numpy(slots.astype(np.int64)).to(device),
+               cu=torch.from_numpy(cu).to(device))
+    flops = 0
+    for b in range(B):
+        keys = np.arange(lens[b] - chunk, lens[b], dtype=np.int64) + 1   # keys per row (causal)
+        flops += 4 * d * hq * int(keys.sum())
+    nbytes = 2 * B * chunk * hq * d * 2 + int(lens.astype(np.int64).sum()) * 2 * hkv * d * 2
+    meta = dict(B=B, hq=hq, hkv=hkv, d=d, bs=bs, chunk=chunk, lens=lens, tables=tables, cu=cu,
+                flops=flops, bytes=nbytes, scale=1.0 / 16.0)
+    return L, dev, meta
+
+
+def run_prefill(args, device):
+    from paged_kv_cache_455_b200 import pa
+    layers = args.layers or 4
+    L, dev, meta = prefill_workload(device, layers)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    maxctx = int(meta["lens"].max())
+
+    def attend(i):
+        q, _, _, kp, vp, out = L[i]
+        pa.pa_prefill_attention(out, q, dev["cu"], meta["chunk"], kp, vp, dev["tables"],
+                                dev["lens"], maxctx, meta["scale"], status)
+
+    def step():
+        for i in range(layers):
+            q, key, val, kp, vp, _ = L[i]
+            pa.pa_reshape_and_cache(key, val, kp, vp, dev["slots"], status)
+            attend(i)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+    stream = torch.cuda.current_stream(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = pa.launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+    launches = pa.launch_count() - l0
+    ms_step = t0.elapsed_time(t1) / args.steps
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        for i in range(layers):
+            attend(i)
+    a1.record(stream)
+    torch.cuda.synchronize(device)
+    attn_ms = a0.elapsed_time(a1) / (args.steps * layers)
+    tflops = meta["flops"] / (attn_ms * 1e-3) / 1e12
+    step_tflops = meta["flops"] * layers / (ms_step * 1e-3) / 1e12
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, src = float(json.load(f)["bf16_tflops"]), "measured cuBLAS bf16 burst"
+    except Exception:
+        peak, src = 1590.0, "fallback"
+    line = {
+        "metric": PREFILL_METRIC, "value": round(step_tflops, 2), "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V, seeded lengths and block tables)",
+        "config": {"workload": "prefill: B=16 sequences, contexts U[1024,4096], each ending "
+                               "with a 512-token chunk, Hq=16, Hkv=4, d=256, block 16, bf16",
+                   "layers": layers, "l2": "no flush: each layer has its own pool"},
+        "attention_tflops": round(tflops, 2),
+        "attention_gbs": round(meta["bytes"] / (attn_ms * 1e-3) / 1e9, 1),
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
+                     "peak_source": src, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                     "traffic": None, "kernel": "pa_prefill_attention (prefill_kernel<256, 4>)",
+                     "algorithmic_flops_per_launch": meta["flops"],
+                     "launch_ms_mean": round(attn_ms, 5)},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline:
+        from oracle import oracle as O
+        q, _, _, kp, vp, _ = L[0]
+        b = 0
+        cu1 = np.array([0, meta["chunk"]])
+        qs = W.to_numpy_elems(q[:meta["chunk"]])
+        kp_h, vp_h = W.to_numpy_elems(kp), W.to_numpy_elems(vp)
+        tt = time.perf_counter()
+        O.prefill_attention_np(qs, kp_h, vp_h, meta["tables"][b:b + 1], meta["lens"][b:b + 1],
+                               cu1, meta["scale"], "bf16")
+        secs = time.perf_counter() - tt
+        keys = np.arange(meta["lens"][b] - meta["chunk"], meta["lens"][b], dtype=np.int64) + 1
+        f1 = 4 * meta["d"] * meta["hq"] * int(keys.sum())
+        line["cpu_baseline"] = {"value": round(f1 / secs / 1e12, 6), "unit": "TFLOP/s",
+                                "cores": os.cpu_count(), "kind": "oracle",
+                                "sample": f"layer 0, sequence 0 (one 512-token chunk over "
+                                          f"{int(meta['lens'][0])} tokens), numpy fp64 oracle, "
+                                          f"{secs:.2f} s"}
+    return line
+
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
@@ -499,6 +633,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=None,
                     help="layers per step (default: the workload's 16); fewer only for profiling")
+    ap.add_argument("--path", default="decode", choices=["decode", "prefill"],
+                    help="decode (the default measurement) or the chunked-prefill path")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -528,6 +664,11 @@ def main(argv=None):
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                  device_id=device)
         dist = tdist
+    if args.path == "prefill":
+        if world != 1:
+            raise SystemExit("--path prefill runs on one GPU")
+        print(json.dumps(run_prefill(args, device)), flush=True)
+        return 0
     try:
         line = run_ours(args, rank, world, device, dist)
         if rank == 0:
