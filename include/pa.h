@@ -238,6 +238,33 @@ pa_status pa_copy_blocks(void *k_pool, void *v_pool, const int64_t *block_mappin
                          pa_dtype dtype, int32_t *dev_status, void *stream);
 
 /*
+ * pa_swap_blocks -- copy whole blocks from one pair of pools to another, for
+ * paging blocks out to host memory and back ("Inside vLLM: Anatomy of a
+ * High-Throughput LLM Inference System", section "Memory-Efficient KV Cache
+ * Storage": blocks move between GPU and CPU memory, the less used ones paged
+ * out to the host when the cache outgrows the GPU).
+ *
+ * For every pair i: block block_mapping[2i + 1] of dst_k_pool / dst_v_pool
+ * becomes a bit-exact copy of block block_mapping[2i] of src_k_pool /
+ * src_v_pool.  Either pair of pools may be device memory or pinned host
+ * memory mapped into the device's address space (e.g. cudaHostAlloc on a
+ * unified-addressing system); the copy runs on the GPU, asynchronously on
+ * `stream`.
+ *   block_mapping  device (or mapped host), [num_pairs][2] int64.
+ *                  Destinations must be distinct.
+ *   pools          [nb, bs, Hkv, d] in `dtype`, nb given per side.
+ * A block id outside its pool sets PA_DEV_BAD_BLOCK and that pair is
+ * skipped.  The source and destination ranges must not overlap.  A pointer
+ * the GPU cannot address as it is (pageable host memory, for instance)
+ * returns PA_ERR_INVALID_ARG without a launch.
+ */
+pa_status pa_swap_blocks(void *dst_k_pool, void *dst_v_pool, int64_t dst_num_blocks,
+                         const void *src_k_pool, const void *src_v_pool, int64_t src_num_blocks,
+                         const int64_t *block_mapping, int num_pairs, int block_size,
+                         int num_kv_heads, int head_dim, pa_dtype dtype, int32_t *dev_status,
+                         void *stream);
+
+/*
  * pa_decode_attention_static -- pa_decode_attention for callers that cannot
  * allocate device memory.  The pages have no counterpart to this call; it is
  * an addition of this library.

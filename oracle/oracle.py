@@ -189,6 +189,22 @@ def copy_blocks_np(k_pool, v_pool, block_mapping):
     return k_out, v_out
 
 
+def swap_blocks_np(dst_k, dst_v, src_k, src_v, block_mapping):
+    """Returns new (dst_k, dst_v) in which block dst of each (src, dst) pair
+    holds block src of the source pools (paging blocks between GPU and host
+    memory: "Inside vLLM: Anatomy of a High-Throughput LLM Inference System",
+    section "Memory-Efficient KV Cache Storage").  Raises ValueError for a
+    block id outside its pool."""
+    k_out, v_out = np.array(dst_k, copy=True), np.array(dst_v, copy=True)
+    src_k, src_v = np.asarray(src_k), np.asarray(src_v)
+    for src, dst in np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2):
+        if not (0 <= src < src_k.shape[0] and 0 <= dst < k_out.shape[0]):
+            raise ValueError("block id outside the pool")
+        k_out[dst] = src_k[src]
+        v_out[dst] = src_v[src]
+    return k_out, v_out
+
+
 # --------------------------------------------------------------------------
 # Attention (C, fp64)
 # --------------------------------------------------------------------------

@@ -21,6 +21,14 @@ Readings taken where the page is silent:
 
 The manager only does bookkeeping; the device work is ``pa_copy_blocks`` for
 the returned pairs followed by ``pa_reshape_and_cache`` for the new tokens.
+
+Swapping ("Inside vLLM: Anatomy of a High-Throughput LLM Inference System",
+section "Memory-Efficient KV Cache Storage": blocks move between GPU and CPU
+memory, the less used ones paged out to the host when the cache outgrows the
+GPU): ``swap_out`` moves all of a sequence's (unshared) blocks to host
+blocks and frees the device ones, ``swap_in`` brings them back into fresh
+device blocks; each returns the (source, destination) pairs for
+``pa_swap_blocks``.
 """
 from __future__ import annotations
 
@@ -31,7 +39,8 @@ import numpy as np
 
 
 class BlockManager:
-    def __init__(self, num_blocks: int, block_size: int, free_order: Optional[Iterable[int]] = None):
+    def __init__(self, num_blocks: int, block_size: int, free_order: Optional[Iterable[int]] = None,
+                 num_host_blocks: int = 0):
         if num_blocks <= 0 or block_size <= 0:
             raise ValueError("num_blocks and block_size must be positive")
         self.num_blocks = num_blocks
@@ -43,6 +52,8 @@ class BlockManager:
         self.refs = np.zeros(num_blocks, dtype=np.int32)
         self.tables: Dict[int, List[int]] = {}
         self.lens: Dict[int, int] = {}
+        self.host_free = deque(range(num_host_blocks))
+        self.swapped: Dict[int, List[int]] = {}
 
     @property
     def num_free(self) -> int:
@@ -102,9 +113,39 @@ class BlockManager:
         self.lens[seq] = pos + 1
         return table[pos // self.block_size] * self.block_size + off, copy
 
+    def swap_out(self, seq: int) -> List[Tuple[int, int]]:
+        """(device block, host block) pairs that move seq to host memory; its
+        device blocks are freed.  Shared blocks cannot move (ValueError); too
+        few host blocks raise MemoryError; either way nothing changes."""
+        table = self.tables[seq]
+        if any(self.refs[b] > 1 for b in table):
+            raise ValueError(f"sequence {seq} shares blocks")
+        if len(table) > len(self.host_free):
+            raise MemoryError(f"need {len(table)} host blocks, {len(self.host_free)} free")
+        pairs = [(b, self.host_free.popleft()) for b in table]
+        for b in table:
+            self._drop(b)
+        self.swapped[seq] = [h for _, h in pairs]
+        self.tables[seq] = []
+        return pairs
+
+    def swap_in(self, seq: int) -> List[Tuple[int, int]]:
+        """(host block, device block) pairs that bring seq back into fresh
+        device blocks; its host blocks are freed.  MemoryError (nothing
+        changes) if the device has too few free blocks."""
+        host = self.swapped[seq]
+        if len(host) > len(self.free):
+            raise MemoryError(f"need {len(host)} blocks, {len(self.free)} free")
+        pairs = [(h, self._take()) for h in host]
+        self.host_free.extend(host)
+        self.tables[seq] = [d for _, d in pairs]
+        del self.swapped[seq]
+        return pairs
+
     def free_seq(self, seq: int) -> None:
         for b in self.tables.pop(seq):
             self._drop(b)
+        self.host_free.extend(self.swapped.pop(seq, []))
         del self.lens[seq]
 
     def block_tables(self, seqs: List[int], max_blocks: Optional[int] = None):

@@ -97,17 +97,21 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const CacheParams p)
 }
 
 struct CopyParams {
-    void *k_pool;
-    void *v_pool;
+    const void *src_k;
+    const void *src_v;
+    void *dst_k;
+    void *dst_v;
     const int64_t *block_mapping;   // [num_pairs][2]: source, destination
     int32_t *dev_status;
-    int64_t num_blocks;
+    int64_t src_blocks;
+    int64_t dst_blocks;
     int64_t block_bytes;            // bs * Hkv * d * element size
     int num_pairs;
 };
 
 // One CTA per (pair, pool, 8 KB chunk of the block): 16-byte copies, 512
-// bytes per warp instruction.
+// bytes per warp instruction.  Either side may be pinned host memory mapped
+// into the device's address space (swap).
 __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p, int chunks)
 {
     const int pair = blockIdx.x / (2 * chunks);
@@ -116,18 +120,64 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p, in
     const int chunk = rest - kv * chunks;
     const int64_t src = p.block_mapping[2 * pair];
     const int64_t dst = p.block_mapping[2 * pair + 1];
-    if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {
+    if (src < 0 || src >= p.src_blocks || dst < 0 || dst >= p.dst_blocks) {
         if (threadIdx.x == 0 && kv == 0 && chunk == 0)
             pa::report(p.dev_status, PA_DEV_BAD_BLOCK);
         return;
     }
-    uint8_t *pool = static_cast<uint8_t *>(kv ? p.v_pool : p.k_pool);
-    const int4 *from = reinterpret_cast<const int4 *>(pool + src * p.block_bytes);
-    int4 *to = reinterpret_cast<int4 *>(pool + dst * p.block_bytes);
+    const int4 *from = reinterpret_cast<const int4 *>(
+        static_cast<const uint8_t *>(kv ? p.src_v : p.src_k) + src * p.block_bytes);
+    int4 *to = reinterpret_cast<int4 *>(static_cast<uint8_t *>(kv ? p.dst_v : p.dst_k) +
+                                        dst * p.block_bytes);
     const int64_t n16 = p.block_bytes >> 4;
     const int64_t end = min(n16, (int64_t)(chunk + 1) * 512);
     for (int64_t c = (int64_t)chunk * 512 + threadIdx.x; c < end; c += 256)
         to[c] = __ldcg(from + c);
+}
+
+// True if the GPU can read and write `ptr` at that same address: device
+// memory, or pinned host memory mapped into the unified address space.
+bool device_addressable(const void *ptr)
+{
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+        cudaGetLastError();   // clear the error of an unknown pointer
+        return false;
+    }
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged)
+        return true;
+    return a.type == cudaMemoryTypeHost && a.devicePointer == ptr;
+}
+
+pa_status launch_copy(CopyParams &p, int block_size, int num_kv_heads, int head_dim,
+                      pa_dtype dtype, void *stream)
+{
+    if (p.num_pairs < 0 || p.src_blocks <= 0 || p.dst_blocks <= 0 || num_kv_heads <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (dtype != PA_DTYPE_F32 && dtype != PA_DTYPE_BF16)
+        return PA_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+        return PA_ERR_UNSUPPORTED;
+    if (ilog2_exact(block_size) < 0 || block_size < 4 || block_size > 32)
+        return PA_ERR_UNSUPPORTED;
+    if (p.num_pairs == 0)
+        return PA_OK;
+    if (!p.src_k || !p.src_v || !p.dst_k || !p.dst_v || !p.block_mapping)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(p.src_k) || !aligned16(p.src_v) || !aligned16(p.dst_k) || !aligned16(p.dst_v))
+        return PA_ERR_INVALID_ARG;
+    if (!device_addressable(p.src_k) || !device_addressable(p.src_v) ||
+        !device_addressable(p.dst_k) || !device_addressable(p.dst_v) ||
+        !device_addressable(p.block_mapping))
+        return PA_ERR_INVALID_ARG;   // e.g. pageable host memory
+    p.block_bytes = (int64_t)block_size * num_kv_heads * head_dim * elem_size(dtype);
+    const int chunks = (int)((p.block_bytes + 8191) / 8192);
+    const int64_t blocks = (int64_t)p.num_pairs * 2 * chunks;
+    if (blocks > INT32_MAX)
+        return PA_ERR_INVALID_ARG;
+    copy_blocks_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p, chunks);
+    ++g_launches;
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 // =====================================================================
@@ -572,33 +622,36 @@ pa_status pa_copy_blocks(void *k_pool, void *v_pool, const int64_t *block_mappin
                          int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
                          pa_dtype dtype, int32_t *dev_status, void *stream)
 {
-    if (num_pairs < 0 || num_blocks <= 0 || num_kv_heads <= 0)
-        return PA_ERR_INVALID_ARG;
-    if (dtype != PA_DTYPE_F32 && dtype != PA_DTYPE_BF16)
-        return PA_ERR_UNSUPPORTED;
-    if (head_dim != 64 && head_dim != 128 && head_dim != 256)
-        return PA_ERR_UNSUPPORTED;
-    if (ilog2_exact(block_size) < 0 || block_size < 4 || block_size > 32)
-        return PA_ERR_UNSUPPORTED;
-    if (num_pairs == 0)
-        return PA_OK;
-    if (!k_pool || !v_pool || !block_mapping)
-        return PA_ERR_INVALID_ARG;
     CopyParams p;
-    p.k_pool = k_pool;
-    p.v_pool = v_pool;
+    p.src_k = k_pool;
+    p.src_v = v_pool;
+    p.dst_k = k_pool;
+    p.dst_v = v_pool;
     p.block_mapping = block_mapping;
     p.dev_status = dev_status;
-    p.num_blocks = num_blocks;
-    p.block_bytes = (int64_t)block_size * num_kv_heads * head_dim * elem_size(dtype);
+    p.src_blocks = num_blocks;
+    p.dst_blocks = num_blocks;
     p.num_pairs = num_pairs;
-    const int chunks = (int)((p.block_bytes + 8191) / 8192);
-    const int64_t blocks = (int64_t)num_pairs * 2 * chunks;
-    if (blocks > INT32_MAX)
-        return PA_ERR_INVALID_ARG;
-    copy_blocks_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p, chunks);
-    ++g_launches;
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return launch_copy(p, block_size, num_kv_heads, head_dim, dtype, stream);
+}
+
+pa_status pa_swap_blocks(void *dst_k_pool, void *dst_v_pool, int64_t dst_num_blocks,
+                         const void *src_k_pool, const void *src_v_pool, int64_t src_num_blocks,
+                         const int64_t *block_mapping, int num_pairs, int block_size,
+                         int num_kv_heads, int head_dim, pa_dtype dtype, int32_t *dev_status,
+                         void *stream)
+{
+    CopyParams p;
+    p.src_k = src_k_pool;
+    p.src_v = src_v_pool;
+    p.dst_k = dst_k_pool;
+    p.dst_v = dst_v_pool;
+    p.block_mapping = block_mapping;
+    p.dev_status = dev_status;
+    p.src_blocks = src_num_blocks;
+    p.dst_blocks = dst_num_blocks;
+    p.num_pairs = num_pairs;
+    return launch_copy(p, block_size, num_kv_heads, head_dim, dtype, stream);
 }
 
 pa_status pa_prefill_attention(void *out, const void *query, const int32_t *cu_q_lens, int total_q,

@@ -47,6 +47,7 @@ SIGNATURES = {
     "pa_decode_attention_static": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                                         _I64, _F, _I, _P, _P]),
     "pa_copy_blocks": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _I, _P, _P]),
+    "pa_swap_blocks": (_I, [_P, _P, _I64, _P, _P, _I64, _P, _I, _I, _I, _I, _I, _P, _P]),
     "pa_prefill_attention": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
                                   _I, _I64, _F, _I, _P, _P]),
     "pa_status_string": (ctypes.c_char_p, [_I]),
@@ -142,6 +143,29 @@ def pa_copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, block_mapping: to
     _check(lib.pa_copy_blocks(_ptr(k_pool), _ptr(v_pool), _ptr(block_mapping),
                               block_mapping.shape[0], nb, bs, hkv, d, _dtype_code(k_pool),
                               _ptr(dev_status), _stream(stream)), "pa_copy_blocks")
+
+
+def pa_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor,
+                   src_v: torch.Tensor, block_mapping: torch.Tensor,
+                   dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Copies block src -> dst for each (src, dst) row of block_mapping [P, 2]
+    int64 from the source pools to the destination pools [nb, bs, Hkv, d];
+    one side may be pinned host memory (paging blocks out and back in)."""
+    for t in (dst_k, dst_v, src_k, src_v):
+        if not t.is_contiguous() or not (t.is_cuda or t.is_pinned()):
+            raise ValueError("pools must be contiguous CUDA or pinned host tensors")
+    _cuda(block_mapping, dev_status)
+    if dst_k.shape[1:] != src_k.shape[1:] or dst_v.shape != dst_k.shape or src_v.shape != src_k.shape:
+        raise ValueError("pool shape mismatch")
+    if not (dst_k.dtype == dst_v.dtype == src_k.dtype == src_v.dtype):
+        raise ValueError("dtype mismatch")
+    if block_mapping.dtype != torch.int64 or block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
+        raise ValueError("block_mapping must be int64 [P, 2]")
+    _, bs, hkv, d = dst_k.shape
+    _check(lib.pa_swap_blocks(_ptr(dst_k), _ptr(dst_v), dst_k.shape[0], _ptr(src_k), _ptr(src_v),
+                              src_k.shape[0], _ptr(block_mapping), block_mapping.shape[0], bs,
+                              hkv, d, _dtype_code(dst_k), _ptr(dev_status), _stream(stream)),
+           "pa_swap_blocks")
 
 
 def pa_prefill_attention(out: torch.Tensor, query: torch.Tensor, cu_q_lens: torch.Tensor,
@@ -264,7 +288,7 @@ def pa_splitk_reduce(out: torch.Tensor, tmp_out: torch.Tensor, max_logits: torch
 
 __all__ = [
     "lib", "LIB_PATH", "SIGNATURES", "PaError", "launch_count",
-    "pa_reshape_and_cache", "pa_copy_blocks", "pa_prefill_attention", "pa_decode_attention", "pa_decode_workspace_bytes",
+    "pa_reshape_and_cache", "pa_copy_blocks", "pa_swap_blocks", "pa_prefill_attention", "pa_decode_attention", "pa_decode_workspace_bytes",
     "pa_decode_attention_static", "PA_STATIC_SCRATCH_BYTES",
     "pa_num_partitions", "pa_splitk_workspace_bytes", "pa_decode_splitk", "pa_splitk_reduce",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA", "PA_ERR_WORKSPACE",

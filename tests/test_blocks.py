@@ -148,3 +148,44 @@ def test_attention_over_shared_blocks_equals_attention_over_private_copies():
     private = O.paged_attention_np(q, kp, vp, priv, lens, 0.25, "f32")
     assert np.abs(shared - private).max() == 0.0
     assert len(set(tab[:, 0])) == 1        # the prompt's first block really is shared
+
+
+def test_swap_out_and_in_moves_every_block_and_restores_the_table():
+    m = BlockManager(8, 4, num_host_blocks=4)
+    m.allocate(0, 10)                       # 3 blocks
+    m.allocate(1, 4)
+    before = list(m.tables[0])
+    out = m.swap_out(0)
+    assert [d for d, _ in out] == before and m.tables[0] == []
+    assert m.num_free == 8 - 1 and len(m.host_free) == 1
+    m.allocate(2, 8)                        # the freed device blocks are reused
+    back = m.swap_in(0)
+    assert [h for h, _ in back] == [h for _, h in out]
+    assert len(m.tables[0]) == 3 and m.lens[0] == 10 and len(m.host_free) == 4
+    slot, copy = m.append_slot(0)           # appends after the swap as before
+    assert copy is None and slot == m.tables[0][2] * 4 + 2
+
+
+def test_swap_refuses_shared_blocks_and_short_pools():
+    m = BlockManager(8, 4, num_host_blocks=2)
+    m.allocate(0, 6)
+    m.fork(0, 1)
+    with pytest.raises(ValueError):
+        m.swap_out(0)
+    m.allocate(2, 12)                       # 3 blocks > 2 host blocks
+    with pytest.raises(MemoryError):
+        m.swap_out(2)
+    assert len(m.tables[2]) == 3 and len(m.host_free) == 2
+
+
+def test_oracle_swap_copies_between_pools():
+    rng = np.random.default_rng(3)
+    dev_k = rng.standard_normal((6, 4, 2, 8)).astype(np.float32)
+    dev_v = rng.standard_normal((6, 4, 2, 8)).astype(np.float32)
+    host_k = np.zeros((3, 4, 2, 8), np.float32)
+    host_v = np.zeros((3, 4, 2, 8), np.float32)
+    hk, hv = O.swap_blocks_np(host_k, host_v, dev_k, dev_v, np.array([[5, 0], [2, 2]]))
+    assert hk[0].tobytes() == dev_k[5].tobytes() and hv[2].tobytes() == dev_v[2].tobytes()
+    assert not hk[1].any() and not hv[1].any()
+    with pytest.raises(ValueError):
+        O.swap_blocks_np(host_k, host_v, dev_k, dev_v, np.array([[6, 0]]))

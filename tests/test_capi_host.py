@@ -149,6 +149,26 @@ def test_copy_blocks_host_validation(pa):
     assert call(n=0, kp=None, vp=None, mapping=None) == 0   # nothing to copy: no launch
 
 
+def test_swap_blocks_host_validation(pa):
+    L = pa.lib
+
+    def call(**kw):
+        a = dict(dk=A, dv=A, dnb=8, sk=A, sv=A, snb=16, mapping=A, n=2, bs=16, hkv=4, d=256,
+                 dt=1)
+        a.update(kw)
+        return L.pa_swap_blocks(a["dk"], a["dv"], a["dnb"], a["sk"], a["sv"], a["snb"],
+                                a["mapping"], a["n"], a["bs"], a["hkv"], a["d"], a["dt"],
+                                None, None)
+    assert call(n=-1) == 1
+    assert call(dnb=0) == 1
+    assert call(snb=0) == 1
+    assert call(d=100) == 2
+    assert call(dt=7) == 2
+    assert call(sk=None) == 1
+    assert call(dv=M) == 1
+    assert call(n=0, dk=None, dv=None, sk=None, sv=None, mapping=None) == 0
+
+
 def test_prefill_host_validation(pa):
     L = pa.lib
 

@@ -1,6 +1,7 @@
-"""Copy-on-write block sharing on the GPU, through the C ABI ("vLLM
-Architecture, Memory and Benchmarks Deep Dive", section 2, "Copy-on-Write
-(CoW) Branching").
+"""Copy-on-write block sharing and host swap on the GPU, through the C ABI
+("vLLM Architecture, Memory and Benchmarks Deep Dive", section 2,
+"Copy-on-Write (CoW) Branching"; "Inside vLLM: Anatomy of a High-Throughput
+LLM Inference System", section "Memory-Efficient KV Cache Storage").
 
 pa_copy_blocks must be bit-exact against the oracle's copy over the whole
 pools.  A GRPO-shaped run (one prompt, 8 rollouts sharing its blocks, each
@@ -122,3 +123,47 @@ def test_grpo_rollouts_share_the_prompt_and_decode_exactly(pa):
     assert int(status.item()) == 0
     ref = O.paged_attention(W.to_numpy_elems(q), k_host, v_host, tab, lens, scale, dtype)
     assert np.abs(out.double().cpu().numpy() - ref).max() <= TOL[dtype]
+
+
+def test_swap_out_and_back_in_is_exact_and_decodes_identically(pa):
+    bs, hq, hkv, d, nb, host_nb = 16, 16, 4, 256, 48, 24
+    k, v = _pools(nb, bs, hkv, d, "bf16", 12)
+    m = BlockManager(nb, bs, free_order=np.random.default_rng(2).permutation(nb),
+                     num_host_blocks=host_nb)
+    m.allocate(0, 200)
+    m.allocate(1, 150)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(13)
+    q = torch.randn(2, hq, d, generator=g, device=DEV).to(torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+
+    def decode():
+        tab, lens = m.block_tables([0, 1])
+        out = torch.empty_like(q)
+        ws = torch.empty(pa.pa_decode_workspace_bytes(2, hq, hkv, d, int(lens.max())),
+                         dtype=torch.uint8, device=DEV)
+        pa.pa_decode_attention(out, q, k, v, torch.from_numpy(tab).to(DEV),
+                               torch.from_numpy(lens).to(DEV), int(lens.max()), 1 / 16, ws, status)
+        torch.cuda.synchronize()
+        return out
+
+    before = decode()
+    host_k = torch.zeros(host_nb, bs, hkv, d, dtype=torch.bfloat16).pin_memory()
+    host_v = torch.zeros(host_nb, bs, hkv, d, dtype=torch.bfloat16).pin_memory()
+    out_pairs = np.array(m.swap_out(0), dtype=np.int64)
+    pa.pa_swap_blocks(host_k, host_v, k, v, torch.from_numpy(out_pairs).to(DEV), status)
+    torch.cuda.synchronize()
+    zeros = np.zeros_like(W.to_numpy_elems(host_k))
+    ref_k, ref_v = O.swap_blocks_np(zeros, zeros, W.to_numpy_elems(k), W.to_numpy_elems(v),
+                                    out_pairs)
+    assert W.to_numpy_elems(host_k).tobytes() == ref_k.tobytes()
+    assert W.to_numpy_elems(host_v).tobytes() == ref_v.tobytes()
+    k[torch.from_numpy(out_pairs[:, 0]).to(DEV)] = 0          # the freed blocks get reused
+    v[torch.from_numpy(out_pairs[:, 0]).to(DEV)] = 0
+    m.allocate(2, 40)
+    in_pairs = np.array(m.swap_in(0), dtype=np.int64)
+    assert set(in_pairs[:, 1]).isdisjoint(m.tables[2])
+    pa.pa_swap_blocks(k, v, host_k, host_v, torch.from_numpy(in_pairs).to(DEV), status)
+    after = decode()
+    assert int(status.item()) == 0
+    assert torch.equal(before, after)       # same data, same tiles: bit-identical
