@@ -594,7 +594,7 @@ def run_prefill(args, device):
         "attention_gbs": round(meta["bytes"] / (attn_ms * 1e-3) / 1e9, 1),
         "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                      "peak_source": src, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
-                     "traffic": None, "kernel": "pa_prefill_attention (prefill_kernel<256, 4>)",
+                     "traffic": None, "kernel": "pa_prefill_attention (prefill_tc_kernel<256, 4>: tcgen05.mma, TMEM accumulators)",
                      "algorithmic_flops_per_launch": meta["flops"],
                      "launch_ms_mean": round(attn_ms, 5)},
         "gpu_launches": launches,

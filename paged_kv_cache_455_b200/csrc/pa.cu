@@ -720,8 +720,32 @@ pa_status pa_prefill_attention(void *out, const void *query, const int32_t *cu_q
         !encode_pool_map(&tv, v_pool, num_blocks, block_size, num_kv_heads, head_dim, dtype, p.tr,
                          1))
         return PA_ERR_CUDA;
-    const pa_status st = pa::prefill_dispatch(head_dim, group, tk, tv, p, (int)grid, smem,
-                                              static_cast<cudaStream_t>(stream));
+    pa_status st;
+    if (block_size >= 16) {
+        // 5th-generation tensor cores: the query rows of the CTA come by TMA
+        // through a 3-D map over [total_q, Hq, d] (box: 64 elements, the
+        // group's heads, the CTA's tokens)
+        EncodeTiledFn enc = encode_fn();
+        if (!enc)
+            return PA_ERR_CUDA;
+        alignas(64) CUtensorMap qmap;
+        const cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads,
+                                    (cuuint64_t)total_q};
+        const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2,
+                                       (cuuint64_t)num_q_heads * head_dim * 2};
+        const cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)tq};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(query), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return PA_ERR_CUDA;
+        st = pa::prefill_tc_dispatch(head_dim, group, qmap, tk, tv, p, (int)grid,
+                                     static_cast<cudaStream_t>(stream));
+    } else {
+        st = pa::prefill_dispatch(head_dim, group, tk, tv, p, (int)grid, smem,
+                                  static_cast<cudaStream_t>(stream));
+    }
     ++g_launches;
     return st;
 }

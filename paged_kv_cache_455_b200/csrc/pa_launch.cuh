@@ -134,5 +134,8 @@ pa_status decode_bf16_simt(DecodeLaunch &L, int *grid, bool launch);
 struct PrefillParams;
 pa_status prefill_dispatch(int head_dim, int group, const CUtensorMap &tk, const CUtensorMap &tv,
                            const PrefillParams &p, int grid, int smem, cudaStream_t stream);
+pa_status prefill_tc_dispatch(int head_dim, int group, const CUtensorMap &tq,
+                              const CUtensorMap &tk, const CUtensorMap &tv,
+                              const PrefillParams &p, int grid, cudaStream_t stream);
 
 }  // namespace pa
