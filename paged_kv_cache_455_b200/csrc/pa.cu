@@ -206,11 +206,11 @@ EncodeTiledFn encode_fn()
 struct MapKey {
     const void *base;
     int64_t rows;
-    int hkv, d, es, tr, hpc;
+    int hkv, d, es, tr, hpc, cpb;
     bool operator==(const MapKey &o) const
     {
         return base == o.base && rows == o.rows && hkv == o.hkv && d == o.d && es == o.es &&
-               tr == o.tr && hpc == o.hpc;
+               tr == o.tr && hpc == o.hpc && cpb == o.cpb;
     }
 };
 
@@ -227,11 +227,16 @@ int g_nmaps = 0, g_next_map = 0;
 // column, token row, column, head) -- the row stride precedes the column
 // stride, so a box lands in shared memory as [head][column][row] -- and a box
 // of `tr` token rows x d of `hpc` heads, 128-byte swizzled.
+// Box: `tr` rows of `hpc` heads, landing in shared memory as
+// [head][128-byte column][row][128 bytes].  With `grouped`, the rows are
+// split into groups of 8 (a fifth dimension) and a box of `tr` rows of one
+// head lands as [8-row group][column][row][128 bytes], so that 8-row groups
+// are a fixed stride apart whatever the number of columns.
 bool encode_pool_map(CUtensorMap *out, const void *base, int64_t nb, int bs, int hkv, int d,
-                     pa_dtype dt, int tr, int hpc)
+                     pa_dtype dt, int tr, int hpc, bool grouped = false)
 {
     const int es = elem_size(dt);
-    const MapKey key{base, nb * bs, hkv, d, es, tr, hpc};
+    const MapKey key{base, nb * bs, hkv, d, es, tr, hpc, grouped ? 1 : 0};
     {
         std::lock_guard<std::mutex> lock(g_map_mu);
         for (int i = 0; i < g_nmaps; ++i)
@@ -249,13 +254,26 @@ bool encode_pool_map(CUtensorMap *out, const void *base, int64_t nb, int bs, int
     const cuuint64_t rowb = (cuuint64_t)d * es;
     const cuuint32_t nch = (cuuint32_t)(rowb / 128);
     alignas(64) CUtensorMap map;
-    const cuuint64_t dims[4] = {epc, (cuuint64_t)(nb * bs), nch, (cuuint64_t)hkv};
-    const cuuint64_t strides[3] = {(cuuint64_t)hkv * rowb, 128, rowb};
-    const cuuint32_t box[4] = {epc, (cuuint32_t)tr, nch, (cuuint32_t)hpc};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUresult r = enc(&map, type, 4, const_cast<void *>(base), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r;
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    if (!grouped) {
+        const cuuint64_t dims[4] = {epc, (cuuint64_t)(nb * bs), nch, (cuuint64_t)hkv};
+        const cuuint64_t strides[3] = {(cuuint64_t)hkv * rowb, 128, rowb};
+        const cuuint32_t box[4] = {epc, (cuuint32_t)tr, nch, (cuuint32_t)hpc};
+        r = enc(&map, type, 4, const_cast<void *>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        if (bs % 8 != 0 || tr % 8 != 0 || hpc != 1)
+            return false;
+        const cuuint64_t dims[5] = {epc, 8, nch, (cuuint64_t)(nb * bs / 8), (cuuint64_t)hkv};
+        const cuuint64_t strides[4] = {(cuuint64_t)hkv * rowb, 128, 8 * (cuuint64_t)hkv * rowb,
+                                       rowb};
+        const cuuint32_t box[5] = {epc, 8, nch, (cuuint32_t)(tr / 8), 1};
+        r = enc(&map, type, 5, const_cast<void *>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
     if (r != CUDA_SUCCESS)
         return false;
     *out = map;
@@ -714,11 +732,13 @@ pa_status pa_prefill_attention(void *out, const void *query, const int32_t *cu_q
     const int64_t grid = (int64_t)num_seqs * num_kv_heads * p.qblocks;
     if (grid > INT32_MAX)
         return PA_ERR_INVALID_ARG;
+    // the tensor-core kernel takes 16-row boxes as [8-row group][column][row]
+    const bool grouped = block_size >= 16;
     CUtensorMap tk, tv;
     if (!encode_pool_map(&tk, k_pool, num_blocks, block_size, num_kv_heads, head_dim, dtype, p.tr,
-                         1) ||
+                         1, grouped) ||
         !encode_pool_map(&tv, v_pool, num_blocks, block_size, num_kv_heads, head_dim, dtype, p.tr,
-                         1))
+                         1, grouped))
         return PA_ERR_CUDA;
     pa_status st;
     if (block_size >= 16) {

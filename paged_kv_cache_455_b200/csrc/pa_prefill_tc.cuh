@@ -6,25 +6,37 @@
 //
 // One CTA per (sequence, KV head, 128 query rows); row r is (token r / G,
 // query head r % G of the group), so one K/V tile serves the whole group.
-// Warps 0-3 own one query row per thread; warp 4 is the control warp.
+// Warps 0-3 own one query row per thread; warp 4 issues the MMAs, warps 5
+// and 6 the TMA copies of K and V.
 //
-//   control (one thread)            TMA: Q once; K and V of 64-token tiles
-//                                   into two stages (16-row boxes of one KV
-//                                   head, 128-byte swizzle)
-//                                   S_j = Q K_j^T: 4 x 16 MMAs of M=128,N=16,
-//                                   K=16 into S buffer j % 2 (TMEM, fp32)
-//                                   O += P_j V_j: 4 MMAs of M=128, N=d, K=16,
-//                                   V read MN-major straight from its boxes
-//   softmax (128 threads)           S row from TMEM (tcgen05.ld), causal
-//                                   mask, running max; O rescaled in TMEM
-//                                   only when the max grew by more than 2^8;
-//                                   P = 2^(s - m) to shared memory (bf16,
-//                                   swizzled K-major), row sum in fp32
+//   producers (5, 6)    TMA: Q once; K tiles into three stages, V tiles into
+//                       four (two of them in the space Q held before it moved
+//                       to tensor memory), one box per 16 tokens (lane k
+//                       issues box k of a tile); through a 5-D map a box
+//                       lands as [8-token group][128-byte column][token]
+//                       [128 bytes] with 128-byte swizzle, so 8-token groups
+//                       are a fixed d * 16 bytes apart across the whole tile
+//   MMA (one thread)    S_j = Q K_j^T (M=128, N=64, K=16 steps) with Q read
+//                       from tensor memory and K from its stage; O += P_j V_j
+//                       (M=128, N=d, K=16 per block) with P_j read from
+//                       tensor memory and V MN-major straight from its stage;
+//                       whichever is ready first is issued.  A K stage is
+//                       free when its S is done, a V stage and a P buffer
+//                       when their P V is (tcgen05.commit)
+//   softmax (warps 0-3) first move the CTA's Q rows from shared to tensor
+//                       memory; then per tile: S row from tensor memory (the
+//                       S buffer is released as soon as it is read), causal
+//                       mask on diagonal tiles, running max; O rescaled in
+//                       tensor memory only when the max grew by more than
+//                       2^8; P = 2^(s - m) as bf16 into P buffer j % 2 of
+//                       tensor memory; row sum in fp32 of the rounded values
 //
-// Completion is tracked by mbarriers: TMA tx counts for the stages, and
-// tcgen05.commit for the MMAs.  Every wait is bounded; a timeout stops all
-// warps through a shared flag, and the tensor memory is released on every
-// path.
+// Tensor memory columns: S [0, 64), O [64, 64 + d), Q (d / 2 columns: two
+// bf16 per column) at 64 + d, P buffers (32 columns) after it.  With Q in
+// tensor memory an S MMA reads only K from shared memory.  S_{j+1} and
+// P_{j-1} V_{j-1} run while the softmax of tile j computes.
+// Every wait is bounded; a timeout stops all warps through a shared flag,
+// and the tensor memory is released on every path.
 #pragma once
 
 #include "pa_prefill.cuh"
@@ -33,18 +45,34 @@ namespace pa {
 
 constexpr int kTcRows = 128;            // query rows per CTA (MMA M)
 constexpr int kTcTile = 64;             // KV tokens per stage
-constexpr int kTcBoxes = kTcTile / 16;  // 16-row boxes per K or V tile
-constexpr int kTcThreads = 160;         // 4 softmax warps + 1 control warp
+constexpr int kTcBoxes = kTcTile / 16;  // 16-token blocks per tile
+constexpr int kTcKStages = 3;
+constexpr int kTcVStages = 4;           // two after the K stages, two where Q was
+constexpr int kTcThreads = 224;         // 4 softmax warps, MMA warp, 2 TMA warps
 
-// Shared memory layout (bytes from the 1024-aligned base), per head dim.
+// Shared memory layout (bytes from the 1024-aligned base), per head dim:
+// Q (then V stages 2, 3) | K stages | V stages 0, 1 | barriers.  The Q region
+// holds exactly two stages.  In a stage, column c of token t is at
+// (t / 8) * (d * 16) + c * 1024 + (t % 8) * 128.
+__host__ __device__ constexpr int tc_group_bytes(int D) { return 8 * D * 2; }
 __host__ __device__ constexpr int tc_box_bytes(int D) { return 16 * D * 2; }
 __host__ __device__ constexpr int tc_q_bytes(int D) { return kTcRows * D * 2; }
-__host__ __device__ constexpr int tc_stage_bytes(int D) { return 2 * kTcBoxes * tc_box_bytes(D); }
-__host__ __device__ constexpr int tc_p_off(int D) { return tc_q_bytes(D) + 2 * tc_stage_bytes(D); }
-__host__ __device__ constexpr int tc_blk_off(int D) { return tc_p_off(D) + kTcRows * 128; }
-__host__ __device__ constexpr int tc_bar_off(int D) { return tc_blk_off(D) + 4 * kPfMaxBlocks; }
-__host__ __device__ constexpr int tc_smem_bytes(int D) { return 1024 + tc_bar_off(D) + 128; }
-__host__ __device__ constexpr uint32_t tc_tmem_cols(int D) { return 128 + D <= 256 ? 256u : 512u; }
+__host__ __device__ constexpr int tc_kv_bytes(int D) { return kTcBoxes * tc_box_bytes(D); }
+__host__ __device__ constexpr int tc_bar_off(int D)
+{
+    return tc_q_bytes(D) + (kTcKStages + 2) * tc_kv_bytes(D);
+}
+__host__ __device__ constexpr int tc_smem_bytes(int D) { return 1024 + tc_bar_off(D) + 256; }
+__host__ __device__ constexpr uint32_t tc_tmem_cols(int D)
+{
+    return 64 + D + D / 2 + 64 <= 256 ? 256u : 512u;
+}
+
+// 16-token blocks of tile j that hold tokens of a context of ctx tokens.
+__device__ __forceinline__ int tc_boxes(int j, int ctx)
+{
+    return min(kTcBoxes, (ctx - j * kTcTile + 15) >> 4);
+}
 
 template <int D, int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -54,11 +82,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 {
     static_assert(D % 64 == 0 && D <= 256, "head dim of 64, 128 or 256");
     static_assert(G >= 1 && 128 % G == 0, "whole tokens per CTA");
+    static_assert(tc_smem_bytes(D) <= 232448, "shared memory per CTA");
     constexpr int TQ = kTcRows / G;
     constexpr int NCH = D / 64;                   // 128-byte columns per row
     constexpr int BOX = tc_box_bytes(D);
+    constexpr int KV = tc_kv_bytes(D);
     constexpr uint32_t TCOLS = tc_tmem_cols(D);
-    constexpr uint32_t IDESC_S = ptx::umma_idesc_bf16(128, 16, false, false);
+    constexpr uint32_t IDESC_S = ptx::umma_idesc_bf16(128, kTcTile, false, false);
     constexpr uint32_t IDESC_O = ptx::umma_idesc_bf16(128, D, false, true);
 
     extern __shared__ uint8_t smem_raw[];
@@ -67,15 +97,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
     const uint32_t q_s = base;
-    const uint32_t stage_s = base + tc_q_bytes(D);
-    const uint32_t p_s = base + tc_p_off(D);
-    int *sblk = reinterpret_cast<int *>(gbase + tc_blk_off(D));
+    const uint32_t k_s = base + tc_q_bytes(D);            // K stage s at k_s + s * KV
+    const uint32_t v_s = k_s + kTcKStages * KV;
+    auto vstage = [&](int s) {                            // V stage s
+        return s < 2 ? v_s + (uint32_t)(s * KV) : q_s + (uint32_t)((s - 2) * KV);
+    };
     const uint32_t bars = base + tc_bar_off(D);
-    // barriers: full[2], empty[2], sfull[2], pready, odone, qfull
-    const uint32_t full0 = bars, empty0 = bars + 16, sfull0 = bars + 32, pready = bars + 48,
-                   odone = bars + 56, qfull = bars + 64;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(gbase + tc_bar_off(D) + 72);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + tc_bar_off(D) + 76);
+    // kfull[3], kempty[3], vfull[4], vempty[4], pready[2], pfree[2], sfull, sfree,
+    // qfull, qready
+    const uint32_t kfull = bars, kempty = bars + 24, vfull = bars + 48, vempty = bars + 80,
+                   pready = bars + 112, pfree = bars + 128, sfull = bars + 144,
+                   sfree = bars + 152, qfull = bars + 160, qready = bars + 168;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(gbase + tc_bar_off(D) + 176);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + tc_bar_off(D) + 180);
 
     const int qb = blockIdx.x % p.qblocks;
     const int rest = blockIdx.x / p.qblocks;
@@ -109,17 +143,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int ntiles = (pos0 + ntok - 1) / kTcTile + 1;
     const int nblk = (min(ntiles * kTcTile, ctx) - 1) / p.block_size + 1;
 
-    // ---- set-up: barriers, block ids, tensor memory
+    // ---- set-up: barriers, block-id check, tensor memory
     if (tid == 0) {
-        ptx::mbar_init(full0, 1);
-        ptx::mbar_init(full0 + 8, 1);
-        ptx::mbar_init(empty0, 1);
-        ptx::mbar_init(empty0 + 8, 1);
-        ptx::mbar_init(sfull0, 1);
-        ptx::mbar_init(sfull0 + 8, 1);
-        ptx::mbar_init(pready, 4);
-        ptx::mbar_init(odone, 1);
+        for (int i = 0; i < kTcKStages; ++i) {
+            ptx::mbar_init(kfull + 8u * i, 1);
+            ptx::mbar_init(kempty + 8u * i, 1);
+        }
+        for (int i = 0; i < kTcVStages; ++i) {
+            ptx::mbar_init(vfull + 8u * i, 1);
+            ptx::mbar_init(vempty + 8u * i, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(pready + 8u * i, 4);
+            ptx::mbar_init(pfree + 8u * i, 1);
+        }
+        ptx::mbar_init(sfull, 1);
+        ptx::mbar_init(sfree, 4);
         ptx::mbar_init(qfull, 1);
+        ptx::mbar_init(qready, 4);
         *abort_flag = 0;
     }
     ptx::fence_mbar_init();
@@ -128,7 +169,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int i = tid; i < nblk; i += kTcThreads) {
         const int id = trow[i];
         bad |= id < 0 || (int64_t)id >= p.num_blocks;
-        sblk[i] = id;
     }
     if (warp == 0) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_holder), TCOLS);
@@ -138,149 +178,260 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bad = __syncthreads_or(bad);
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const uint32_t s_tm = tmem;            // S buffers: columns [0, 64) and [64, 128)
-    const uint32_t o_tm = tmem + 128;      // O: columns [128, 128 + D)
+    const uint32_t s_tm = tmem;
+    const uint32_t o_tm = tmem + 64;
+    const uint32_t q_tm = tmem + 64 + (uint32_t)D;
+    const uint32_t p_tm = q_tm + (uint32_t)(D / 2);  // P buffer s at p_tm + 32 s
 
     if (bad) {
         if (tid == 0)
             report(p.dev_status, PA_DEV_BAD_BLOCK);
-    } else if (warp == 4) {
-        // ================================================ control warp
+    } else if (warp >= 5) {
+        // ================================================ TMA producers
+        // warp 5 copies K (and Q), warp 6 copies V; lane x issues box x
+        // (tokens 16 x .. 16 x + 15) of each tile
+        const bool is_k = warp == 5;
+        const int xb = lane;
+        const uint32_t full = is_k ? kfull : vfull, empty = is_k ? kempty : vempty;
+        const int nst = is_k ? kTcKStages : kTcVStages;
+        const void *tmap = is_k ? static_cast<const void *>(&tmap_k)
+                                : static_cast<const void *>(&tmap_v);
+        bool ok = true;
         if (lane == 0) {
-            auto issue_kv = [&](int j) {
-                const int s = j & 1;
-                const uint32_t kst = stage_s + (uint32_t)(s * tc_stage_bytes(D));
-                const uint32_t vst = kst + (uint32_t)(kTcBoxes * BOX);
-                int nbox = 0;
-                while (nbox < kTcBoxes && j * kTcTile + nbox * 16 < ctx)
-                    ++nbox;
-                ptx::mbar_arrive_expect_tx(full0 + 8u * s, (uint32_t)(2 * nbox * BOX));
-                for (int k = 0; k < nbox; ++k) {
-                    const int t = j * kTcTile + k * 16;
-                    const int row = sblk[t >> p.bs_log2] * p.block_size + (t & (p.block_size - 1));
-                    ptx::tma_load_4d(kst + (uint32_t)(k * BOX), &tmap_k, 0, row, 0, h, full0 + 8u * s,
-                                     ptx::policy_evict_normal());
-                    ptx::tma_load_4d(vst + (uint32_t)(k * BOX), &tmap_v, 0, row, 0, h, full0 + 8u * s,
-                                     ptx::policy_evict_normal());
-                }
-            };
-            auto issue_s = [&](int j) {        // S_j = Q K_j^T into buffer j & 1
-                const uint32_t kst = stage_s + (uint32_t)((j & 1) * tc_stage_bytes(D));
-                for (int box = 0; box < kTcBoxes; ++box)
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t a = ptx::umma_desc_sw128(
-                            q_s + (uint32_t)((kk >> 2) * kTcRows * 128 + (kk & 3) * 32), 16, 1024);
-                        const uint64_t bd = ptx::umma_desc_sw128(
-                            kst + (uint32_t)(box * BOX + (kk >> 2) * 2048 + (kk & 3) * 32), 16,
-                            1024);
-                        ptx::umma_bf16_ss(s_tm + (uint32_t)((j & 1) * 64 + box * 16), a, bd,
-                                          IDESC_S, kk > 0);
-                    }
-                ptx::umma_commit(sfull0 + 8u * (j & 1));
-            };
-            bool ok = true;
-            ptx::prefetch_tensormap(&tmap_q);
-            ptx::prefetch_tensormap(&tmap_k);
-            ptx::prefetch_tensormap(&tmap_v);
-            ptx::mbar_arrive_expect_tx(qfull, (uint32_t)tc_q_bytes(D));
-            for (int c = 0; c < NCH; ++c)
-                ptx::tma_load_3d_nohint(q_s + (uint32_t)(c * kTcRows * 128), &tmap_q, c * 64,
-                                        h * G, q0 + tok0, qfull);
-            issue_kv(0);
-            if (ntiles > 1)
-                issue_kv(1);
-            ok = ptx::mbar_wait_bounded(qfull, 0, kWaitLimitNs) &&
-                 ptx::mbar_wait_bounded(full0, 0, kWaitLimitNs);
-            if (ok) {
-                ptx::tc_fence_after();
-                issue_s(0);
+            ptx::prefetch_tensormap(tmap);
+            if (is_k) {
+                ptx::prefetch_tensormap(&tmap_q);
+                ptx::mbar_arrive_expect_tx(qfull, (uint32_t)tc_q_bytes(D));
+                for (int c = 0; c < NCH; ++c)
+                    ptx::tma_load_3d_nohint(q_s + (uint32_t)(c * kTcRows * 128), &tmap_q, c * 64,
+                                            h * G, q0 + tok0, qfull);
             }
-            for (int j = 0; ok && j < ntiles; ++j) {
-                if (*abort_flag)
-                    break;
-                if (j + 1 < ntiles) {
-                    ok = ptx::mbar_wait_bounded(full0 + 8u * ((j + 1) & 1),
-                                                (uint32_t)(((j + 1) >> 1) & 1), kWaitLimitNs);
-                    if (!ok)
-                        break;
-                    ptx::tc_fence_after();
-                    issue_s(j + 1);
-                }
-                ok = ptx::mbar_wait_bounded(pready, (uint32_t)(j & 1), kWaitLimitNs);
-                if (!ok)
-                    break;
-                ptx::tc_fence_after();
-                const uint32_t vst =
-                    stage_s + (uint32_t)((j & 1) * tc_stage_bytes(D) + kTcBoxes * BOX);
-                for (int box = 0; box < kTcBoxes; ++box) {
-                    const uint64_t a = ptx::umma_desc_sw128(p_s + (uint32_t)(box * 32), 16, 1024);
-                    const uint64_t bd =
-                        ptx::umma_desc_sw128(vst + (uint32_t)(box * BOX), 2048, 1024);
-                    ptx::umma_bf16_ss(o_tm, a, bd, IDESC_O, j > 0 || box > 0);
-                }
-                ptx::umma_commit(empty0 + 8u * (j & 1));
-                ptx::umma_commit(odone);
-                if (j + 2 < ntiles) {
-                    ok = ptx::mbar_wait_bounded(empty0 + 8u * (j & 1), (uint32_t)((j >> 1) & 1),
-                                                kWaitLimitNs);
-                    if (!ok)
-                        break;
-                    issue_kv(j + 2);
-                }
+        }
+        // block ids come 32 at a time, lane l holding entry 32 * batch + l,
+        // one batch ahead, so that no copy waits for the table; a tile's
+        // blocks lie in one batch (a batch is 32 blocks >= 512 tokens)
+        auto batch_ids = [&](int bt) {
+            const int i = bt * 32 + lane;
+            return i < nblk ? __ldg(trow + i) : -1;
+        };
+        int ids_cur = batch_ids(0), ids_next = batch_ids(1), cur_batch = 0;
+        int issued = 0;
+        for (int i = 0; i < ntiles; ++i) {
+            if (__any_sync(kFull, *abort_flag != 0))
+                break;
+            const int bt = (i * kTcTile) >> (p.bs_log2 + 5);   // same for all lanes
+            if (bt != cur_batch) {
+                cur_batch = bt;
+                ids_cur = ids_next;
+                ids_next = batch_ids(bt + 1);
             }
+            const int id = __shfl_sync(kFull, ids_cur, ((i * kTcTile + xb * 16) >> p.bs_log2) & 31);
+            const int s = i % nst, nbox = tc_boxes(i, ctx);
+            const int row = id * p.block_size + ((i * kTcTile + xb * 16) & (p.block_size - 1));
+            if (i >= nst) {
+                ok = __all_sync(kFull, ptx::mbar_wait_bounded(empty + 8u * s,
+                                                              (uint32_t)((i / nst - 1) & 1),
+                                                              kWaitLimitNs));
+            } else if (!is_k && s >= 2) {
+                // V stages 2 and 3 are where Q was: wait until Q is in
+                // tensor memory
+                ok = __all_sync(kFull, ptx::mbar_wait_bounded(qready, 0, kWaitLimitNs));
+            }
+            if (!ok)
+                break;
+            const uint32_t dst = is_k ? k_s + (uint32_t)(s * KV) : vstage(s);
+            if (lane == 0)
+                ptx::mbar_arrive_expect_tx(full + 8u * s, (uint32_t)(nbox * BOX));
+            __syncwarp();
+            if (xb < nbox)
+                ptx::tma_load_5d(dst + (uint32_t)(xb * BOX), tmap, 0, 0, 0, row >> 3, h,
+                                 full + 8u * s, ptx::policy_evict_normal());
+            issued = i + 1;
+        }
+        if (lane == 0) {
             if (!ok) {
                 report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
                 *abort_flag = 1;
             }
+            // no copy may land after the CTA is gone: wait (bounded) for the
+            // last ones issued to each stage; on the normal path the MMA
+            // thread has already seen them all
+            if (is_k)
+                ptx::mbar_wait_bounded(qfull, 0, kWaitLimitNs);
+            for (int i = max(0, issued - nst); i < issued; ++i)
+                ptx::mbar_wait_bounded(full + 8u * (i % nst), (uint32_t)((i / nst) & 1),
+                                       kWaitLimitNs);
+        }
+        __syncwarp();
+    } else if (warp == 4) {
+        // ================================================ MMA issue
+        // Order: S_0, then per tile j: S_{j+1} (ready once the softmax has
+        // read S_j out of tensor memory and K_{j+1} has landed), P_j V_j
+        // (ready once the softmax has written P_j and V_j has landed).  The
+        // whole warp waits (suspending, so it takes no issue slots from the
+        // softmax warps); one elected lane, always lane 0, issues the MMAs
+        // and their commits.
+        // descriptors: K is K-major, 8-token groups d * 16 bytes apart; V is
+        // MN-major, 64-element columns 1024 bytes apart, 8-token groups
+        // d * 16 bytes apart
+        const uint64_t k_desc = ptx::umma_desc_sw128(k_s, 16, tc_group_bytes(D));
+        auto wait = [&](uint32_t bar, uint32_t parity) {
+            return __all_sync(kFull, ptx::mbar_wait_bounded(bar, parity, kWaitLimitNs));
+        };
+        auto issue_s = [&](int j) {
+            ptx::tc_fence_after();
+            // (columns of blocks past the context come out of stale rows;
+            // the causal mask drops them)
+            const uint64_t kd = k_desc + (uint64_t)(((j % kTcKStages) * KV) >> 4);
+            if (ptx::elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    ptx::umma_bf16_ts(s_tm, q_tm + (uint32_t)(kk * 8),
+                                      kd + (uint64_t)(((kk >> 2) * 1024 + (kk & 3) * 32) >> 4),
+                                      IDESC_S, kk > 0);
+                ptx::umma_commit(sfull);
+                ptx::umma_commit(kempty + 8u * (j % kTcKStages));
+            }
+            __syncwarp();
+        };
+        bool ok = wait(qready, 0) && wait(kfull, 0);
+        if (ok)
+            issue_s(0);
+        for (int j = 0; ok && j < ntiles; ++j) {
+            if (__any_sync(kFull, *abort_flag != 0))
+                break;
+            if (j + 1 < ntiles) {
+                if (!(ok = wait(sfree, (uint32_t)(j & 1)) &&
+                           wait(kfull + 8u * ((j + 1) % kTcKStages),
+                                (uint32_t)(((j + 1) / kTcKStages) & 1))))
+                    break;
+                issue_s(j + 1);
+            }
+            const int s = j & 1, vs = j % kTcVStages;
+            if (!(ok = wait(pready + 8u * s, (uint32_t)((j >> 1) & 1)) &&
+                       wait(vfull + 8u * vs, (uint32_t)((j / kTcVStages) & 1))))
+                break;
+            ptx::tc_fence_after();
+            const int nbox = tc_boxes(j, ctx);
+            const uint64_t vd = ptx::umma_desc_sw128(vstage(vs), 1024, tc_group_bytes(D));
+            if (ptx::elect_one()) {
+                for (int box = 0; box < nbox; ++box)
+                    ptx::umma_bf16_ts(o_tm, p_tm + (uint32_t)(s * 32 + box * 8),
+                                      vd + (uint64_t)((box * BOX) >> 4), IDESC_O,
+                                      j > 0 || box > 0);
+                ptx::umma_commit(vempty + 8u * vs);
+                ptx::umma_commit(pfree + 8u * s);
+            }
+            __syncwarp();
+        }
+        if (!ok && lane == 0) {
+            report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+            *abort_flag = 1;
         }
         __syncwarp();
     } else {
         // ================================================ softmax warps
         const int r = tid;                          // query row = TMEM lane
-        const int pos = pos0 + r / G;
+        // rows past the chunk (not stored) are clamped to the last position
+        const int pos = min(pos0 + r / G, ctx - 1);
         const uint32_t lane_tm = (uint32_t)(warp * 32) << 16;
+        // with a positive scale the max of the raw logits scales to the max
+        // of the scaled ones (rounding is monotone); otherwise scale first
+        const bool pos_scale = p.scale_log2 > 0.f;
+        const float sc = pos_scale ? p.scale_log2 : 1.f;
         float m_ref = -INFINITY, l = 0.f;
-        bool ok = true;
+        bool ok = __all_sync(kFull, ptx::mbar_wait_bounded(qfull, 0, kWaitLimitNs));
         // tcgen05.ld / st / wait are .sync.aligned: every decision that
         // guards one is made for the whole warp
-        for (int j = 0; j < ntiles; ++j) {
+        if (ok) {
+            // this row of Q, from the swizzled shared copy (column c, 16-byte
+            // unit u at c * 16384 + r * 128 + ((u ^ (r & 7)) << 4)) into
+            // tensor memory, two bf16 per column
+#pragma unroll
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+                uint32_t w[16];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int u = (c4 & 1) * 4 + k;
+                    const uint32_t a = q_s + (uint32_t)((c4 >> 1) * kTcRows * 128 + r * 128) +
+                                       ((uint32_t)(u ^ (r & 7)) << 4);
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w[4 * k]), "=r"(w[4 * k + 1]), "=r"(w[4 * k + 2]),
+                                   "=r"(w[4 * k + 3])
+                                 : "r"(a));
+                }
+                ptx::tmem_st16(q_tm + lane_tm + (uint32_t)(c4 * 16), w);
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            // the Q region is reused by V copies (async proxy)
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                ptx::mbar_arrive(qready);
+        }
+        for (int j = 0; ok && j < ntiles; ++j) {
+            const int s = j & 1;
             if (__any_sync(kFull, *abort_flag != 0)) {
                 ok = false;
                 break;
             }
-            if (!__all_sync(kFull, ptx::mbar_wait_bounded(sfull0 + 8u * (j & 1),
-                                                          (uint32_t)((j >> 1) & 1),
+            if (!__all_sync(kFull, ptx::mbar_wait_bounded(sfull, (uint32_t)(j & 1),
                                                           kWaitLimitNs))) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
             float sv[kTcTile];
-#pragma unroll
-            for (int c = 0; c < kTcTile / 16; ++c) {
-                uint32_t u[16];
-                ptx::tmem_ld16(s_tm + lane_tm + (uint32_t)((j & 1) * 64 + c * 16), u);
+            {
+                uint32_t u0[16], u1[16], u2[16], u3[16];
+                const uint32_t sa = s_tm + lane_tm;
+                ptx::tmem_ld16(sa, u0);
+                ptx::tmem_ld16(sa + 16, u1);
+                ptx::tmem_ld16(sa + 32, u2);
+                ptx::tmem_ld16(sa + 48, u3);
                 ptx::tmem_wait_ld();
+                // S is in registers: the MMA may overwrite it
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    ptx::mbar_arrive(sfree);
+                // (the values are taken only after the arrive, so that no
+                // arithmetic on them is scheduled ahead of it)
+                ptx::tmem_hold16(u0);
+                ptx::tmem_hold16(u1);
+                ptx::tmem_hold16(u2);
+                ptx::tmem_hold16(u3);
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    sv[c * 16 + e] = __uint_as_float(u[e]);
+                for (int e = 0; e < 16; ++e) {
+                    sv[e] = __uint_as_float(u0[e]);
+                    sv[16 + e] = __uint_as_float(u1[e]);
+                    sv[32 + e] = __uint_as_float(u2[e]);
+                    sv[48 + e] = __uint_as_float(u3[e]);
+                }
+            }
+            if (!pos_scale) {
+#pragma unroll
+                for (int c = 0; c < kTcTile; ++c)
+                    sv[c] *= p.scale_log2;
             }
             const int tstart = j * kTcTile;
-            float mx = -INFINITY;
+            if (tstart + kTcTile - 1 > pos0) {
+                // a column past some row's position (or past the context)
 #pragma unroll
-            for (int c = 0; c < kTcTile; ++c) {
-                sv[c] = tstart + c <= pos ? sv[c] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, sv[c]);
+                for (int c = 0; c < kTcTile; ++c)
+                    sv[c] = tstart + c <= pos ? sv[c] : -INFINITY;
             }
-            if (j > 0) {
-                // the previous P V is done: P may be overwritten, O is stable
-                if (!__all_sync(kFull, ptx::mbar_wait_bounded(odone, (uint32_t)((j - 1) & 1),
-                                                              kWaitLimitNs))) {
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-            }
+            float m8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                m8[e] = sv[e];
+#pragma unroll
+            for (int c = 8; c < kTcTile; ++c)
+                m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
+                             sc;
             bool grow = false;
             float alpha = 1.f;
             if (m_ref == -INFINITY) {
@@ -290,12 +441,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 alpha = ptx::ex2(m_ref - mx);
             }
             if (__any_sync(kFull, grow)) {
+                // O must be stable: P_{j-1} V_{j-1} (and all before) done
+                if (!__all_sync(kFull, ptx::mbar_wait_bounded(pfree + 8u * (s ^ 1),
+                                                              (uint32_t)(((j - 1) >> 1) & 1),
+                                                              kWaitLimitNs))) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
                 // the whole warp rescales its rows of O (alpha = 1 for rows
                 // whose max did not grow)
                 for (int c = 0; c < D / 16; ++c) {
                     uint32_t u[16];
                     ptx::tmem_ld16(o_tm + lane_tm + (uint32_t)(c * 16), u);
                     ptx::tmem_wait_ld();
+                    ptx::tmem_hold16(u);
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
@@ -307,52 +467,63 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 l *= alpha;
                 m_ref = mx;
             }
-            const float ref = m_ref == -INFINITY ? 0.f : m_ref;
-            // P row: 64 bf16 = 8 16-byte units, unit u at ((u ^ (r & 7)) << 4)
+            const float nref = m_ref == -INFINITY ? 0.f : -m_ref;
+            // P row as 32 columns of bf16 pairs
+            uint32_t w0[16], w1[16];
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                uint32_t w[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t pk = ptx::pack_bf16x2(ptx::ex2(sv[8 * u + 2 * k] - ref),
-                                                         ptx::ex2(sv[8 * u + 2 * k + 1] - ref));
-                    l += ptx::bf16lo_to_f32(pk) + ptx::bf16hi_to_f32(pk);
-                    w[k] = pk;
-                }
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                                 p_s + (uint32_t)(r * 128) + ((uint32_t)(u ^ (r & 7)) << 4)),
-                             "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
-                             : "memory");
+            for (int k = 0; k < 16; ++k) {
+                w0[k] = ptx::pack_bf16x2(ptx::ex2(fmaf(sv[2 * k], sc, nref)),
+                                         ptx::ex2(fmaf(sv[2 * k + 1], sc, nref)));
+                w1[k] = ptx::pack_bf16x2(ptx::ex2(fmaf(sv[32 + 2 * k], sc, nref)),
+                                         ptx::ex2(fmaf(sv[32 + 2 * k + 1], sc, nref)));
+                l4[k & 3] += (ptx::bf16lo_to_f32(w0[k]) + ptx::bf16hi_to_f32(w0[k])) +
+                             (ptx::bf16lo_to_f32(w1[k]) + ptx::bf16hi_to_f32(w1[k]));
             }
-            if (tstart + kTcTile > ctx) {
-                // V rows past the context: whatever the pool or an older tile
-                // left there; their weight is 0, but 0 * NaN is NaN.  (The
-                // stage's copies are complete: S_j, which follows them, is.)
-                if (!__all_sync(kFull, ptx::mbar_wait_bounded(full0 + 8u * (j & 1),
-                                                              (uint32_t)((j >> 1) & 1),
+            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            if (j >= 2) {
+                // P buffer s is free once P_{j-2} V_{j-2} is done
+                if (!__all_sync(kFull, ptx::mbar_wait_bounded(pfree + 8u * s,
+                                                              (uint32_t)(((j - 2) >> 1) & 1),
                                                               kWaitLimitNs))) {
                     ok = false;
                     break;
                 }
-                const uint32_t vst =
-                    stage_s + (uint32_t)((j & 1) * tc_stage_bytes(D) + kTcBoxes * BOX);
+                ptx::tc_fence_after();
+            }
+            ptx::tmem_st16(p_tm + lane_tm + (uint32_t)(s * 32), w0);
+            ptx::tmem_st16(p_tm + lane_tm + (uint32_t)(s * 32 + 16), w1);
+            if (tstart + kTcTile > ctx && ((ctx - tstart) & 15) != 0) {
+                // V rows of the last block past the context: whatever the
+                // pool holds there; their weight is 0, but 0 * NaN is NaN
+                if (!__all_sync(kFull, ptx::mbar_wait_bounded(
+                                           vfull + 8u * (j % kTcVStages),
+                                           (uint32_t)((j / kTcVStages) & 1), kWaitLimitNs))) {
+                    ok = false;
+                    break;
+                }
                 const int from = ctx - tstart;
-                for (int idx = r; idx < (kTcTile - from) * NCH * 8; idx += kTcRows) {
+                const int to = (from + 15) & ~15;
+                const uint32_t vst = vstage(j % kTcVStages);
+                for (int idx = r; idx < (to - from) * NCH * 8; idx += kTcRows) {
                     const int t = from + idx / (NCH * 8), rem = idx % (NCH * 8);
-                    const uint32_t a = vst + (uint32_t)((t >> 4) * BOX + (rem >> 3) * 2048 +
-                                                        (t & 15) * 128 + (rem & 7) * 16);
+                    const uint32_t a = vst + (uint32_t)((t >> 3) * tc_group_bytes(D) +
+                                                        (rem >> 3) * 1024 + (t & 7) * 128 +
+                                                        (rem & 7) * 16);
                     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0)
                                  : "memory");
                 }
+                // the MMA reads V through the async proxy
+                ptx::fence_proxy_async_smem();
             }
-            // the MMA reads P and V through the async proxy
-            ptx::fence_proxy_async_smem();
+            ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                ptx::mbar_arrive(pready);
+                ptx::mbar_arrive(pready + 8u * s);
         }
-        if (ok && !__all_sync(kFull, ptx::mbar_wait_bounded(odone, (uint32_t)((ntiles - 1) & 1),
+        if (ok && !__all_sync(kFull, ptx::mbar_wait_bounded(pfree + 8u * ((ntiles - 1) & 1),
+                                                            (uint32_t)(((ntiles - 1) >> 1) & 1),
                                                             kWaitLimitNs)))
             ok = false;
         if (!ok) {
@@ -371,6 +542,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 uint32_t u[16];
                 ptx::tmem_ld16(o_tm + lane_tm + (uint32_t)(c * 16), u);
                 ptx::tmem_wait_ld();
+                ptx::tmem_hold16(u);
                 uint4 a, b2;
                 a.x = ptx::pack_bf16x2(__uint_as_float(u[0]) * inv, __uint_as_float(u[1]) * inv);
                 a.y = ptx::pack_bf16x2(__uint_as_float(u[2]) * inv, __uint_as_float(u[3]) * inv);
