@@ -44,6 +44,7 @@ METRIC = "paged decode attention achieved HBM GB/s (% of 8 TB/s); decode tokens/
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_qwen.md")
+PREFILL_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "prefill_tc_kernel_chunk512.md")
 CSRC = os.path.join(ROOT, "paged_kv_cache_455_b200", "csrc")
 
 
@@ -76,11 +77,11 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the decode kernel from the committed ncu summary,
-    scaled to the benchmark's launch, or None if the kernel changed since."""
+def profiled_traffic(summary=None):
+    """DRAM bytes per launch of a kernel from its committed ncu summary (the
+    decode kernel's by default), or None if the kernel sources changed since."""
     try:
-        text = open(PROFILE_SUMMARY).read()
+        text = open(summary or PROFILE_SUMMARY).read()
     except OSError:
         return None
     m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
@@ -594,7 +595,10 @@ def run_prefill(args, device):
         "attention_gbs": round(meta["bytes"] / (attn_ms * 1e-3) / 1e9, 1),
         "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                      "peak_source": src, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
-                     "traffic": None, "kernel": "pa_prefill_attention (prefill_tc_kernel<256, 4>: tcgen05.mma, TMEM accumulators)",
+                     "traffic": profiled_traffic(PREFILL_PROFILE_SUMMARY),
+                     "kernel": "pa_prefill_attention (prefill_tc_kernel<256, 4>: tcgen05.mma, "
+                               "TMEM accumulators)",
+                     "algorithmic_bytes_per_launch": meta["bytes"],
                      "algorithmic_flops_per_launch": meta["flops"],
                      "launch_ms_mean": round(attn_ms, 5)},
         "gpu_launches": launches,

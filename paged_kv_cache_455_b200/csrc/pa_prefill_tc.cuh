@@ -9,9 +9,9 @@
 // Warps 0-3 own one query row per thread; warp 4 issues the MMAs, warps 5
 // and 6 the TMA copies of K and V.
 //
-//   producers (5, 6)    TMA: Q once; K tiles into three stages, V tiles into
-//                       four (two of them in the space Q held before it moved
-//                       to tensor memory), one box per 16 tokens (lane k
+//   producers (5, 6)    TMA: Q once; K tiles into four stages, V tiles into
+//                       three (one of each in the space Q held before it
+//                       moved to tensor memory), one box per 16 tokens (lane k
 //                       issues box k of a tile); through a 5-D map a box
 //                       lands as [8-token group][128-byte column][token]
 //                       [128 bytes] with 128-byte swizzle, so 8-token groups
@@ -46,13 +46,14 @@ namespace pa {
 constexpr int kTcRows = 128;            // query rows per CTA (MMA M)
 constexpr int kTcTile = 64;             // KV tokens per stage
 constexpr int kTcBoxes = kTcTile / 16;  // 16-token blocks per tile
-constexpr int kTcKStages = 3;
-constexpr int kTcVStages = 4;           // two after the K stages, two where Q was
+constexpr int kTcKStages = 4;           // three after Q, one where Q was
+constexpr int kTcVStages = 3;           // two after the K stages, one where Q was
 constexpr int kTcThreads = 224;         // 4 softmax warps, MMA warp, 2 TMA warps
 
 // Shared memory layout (bytes from the 1024-aligned base), per head dim:
-// Q (then V stages 2, 3) | K stages | V stages 0, 1 | barriers.  The Q region
-// holds exactly two stages.  In a stage, column c of token t is at
+// Q (then K stage 3, V stage 2) | K stages 0-2 | V stages 0, 1 | barriers.
+// The Q region holds exactly two stages.  In a stage, column c of token t is
+// at
 // (t / 8) * (d * 16) + c * 1024 + (t % 8) * 128.
 __host__ __device__ constexpr int tc_group_bytes(int D) { return 8 * D * 2; }
 __host__ __device__ constexpr int tc_box_bytes(int D) { return 16 * D * 2; }
@@ -60,7 +61,7 @@ __host__ __device__ constexpr int tc_q_bytes(int D) { return kTcRows * D * 2; }
 __host__ __device__ constexpr int tc_kv_bytes(int D) { return kTcBoxes * tc_box_bytes(D); }
 __host__ __device__ constexpr int tc_bar_off(int D)
 {
-    return tc_q_bytes(D) + (kTcKStages + 2) * tc_kv_bytes(D);
+    return tc_q_bytes(D) + 5 * tc_kv_bytes(D);
 }
 __host__ __device__ constexpr int tc_smem_bytes(int D) { return 1024 + tc_bar_off(D) + 256; }
 __host__ __device__ constexpr uint32_t tc_tmem_cols(int D)
@@ -97,15 +98,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
     const uint32_t q_s = base;
-    const uint32_t k_s = base + tc_q_bytes(D);            // K stage s at k_s + s * KV
-    const uint32_t v_s = k_s + kTcKStages * KV;
-    auto vstage = [&](int s) {                            // V stage s
-        return s < 2 ? v_s + (uint32_t)(s * KV) : q_s + (uint32_t)((s - 2) * KV);
+    const uint32_t n_s = base + tc_q_bytes(D);            // the five stages after Q
+    auto kstage = [&](int s) {                            // K stage s (3: where Q was)
+        return s < 3 ? n_s + (uint32_t)(s * KV) : q_s;
+    };
+    auto vstage = [&](int s) {                            // V stage s (2: where Q was)
+        return s < 2 ? n_s + (uint32_t)((3 + s) * KV) : q_s + (uint32_t)KV;
     };
     const uint32_t bars = base + tc_bar_off(D);
-    // kfull[3], kempty[3], vfull[4], vempty[4], pready[2], pfree[2], sfull, sfree,
+    // kfull[4], kempty[4], vfull[3], vempty[3], pready[2], pfree[2], sfull, sfree,
     // qfull, qready
-    const uint32_t kfull = bars, kempty = bars + 24, vfull = bars + 48, vempty = bars + 80,
+    const uint32_t kfull = bars, kempty = bars + 32, vfull = bars + 64, vempty = bars + 88,
                    pready = bars + 112, pfree = bars + 128, sfull = bars + 144,
                    sfree = bars + 152, qfull = bars + 160, qready = bars + 168;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(gbase + tc_bar_off(D) + 176);
@@ -232,14 +235,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 ok = __all_sync(kFull, ptx::mbar_wait_bounded(empty + 8u * s,
                                                               (uint32_t)((i / nst - 1) & 1),
                                                               kWaitLimitNs));
-            } else if (!is_k && s >= 2) {
-                // V stages 2 and 3 are where Q was: wait until Q is in
-                // tensor memory
+            } else if (s == (is_k ? 3 : 2)) {
+                // the stage where Q was: wait until Q is in tensor memory
                 ok = __all_sync(kFull, ptx::mbar_wait_bounded(qready, 0, kWaitLimitNs));
             }
             if (!ok)
                 break;
-            const uint32_t dst = is_k ? k_s + (uint32_t)(s * KV) : vstage(s);
+            const uint32_t dst = is_k ? kstage(s) : vstage(s);
             if (lane == 0)
                 ptx::mbar_arrive_expect_tx(full + 8u * s, (uint32_t)(nbox * BOX));
             __syncwarp();
@@ -274,15 +276,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // descriptors: K is K-major, 8-token groups d * 16 bytes apart; V is
         // MN-major, 64-element columns 1024 bytes apart, 8-token groups
         // d * 16 bytes apart
-        const uint64_t k_desc = ptx::umma_desc_sw128(k_s, 16, tc_group_bytes(D));
-        auto wait = [&](uint32_t bar, uint32_t parity) {
-            return __all_sync(kFull, ptx::mbar_wait_bounded(bar, parity, kWaitLimitNs));
+        // both phases complete?  One non-blocking test and one vote when
+        // they are (the usual case); else suspending waits, unless another
+        // warp has given up
+        auto ready = [&](uint32_t b1, uint32_t p1, uint32_t b2, uint32_t p2) -> bool {
+            if (__all_sync(kFull, ptx::mbar_test_wait(b1, p1) && ptx::mbar_test_wait(b2, p2)))
+                return true;
+            if (__any_sync(kFull, *abort_flag != 0))
+                return false;
+            return __all_sync(kFull, ptx::mbar_wait_bounded(b1, p1, kWaitLimitNs)) &&
+                   __all_sync(kFull, ptx::mbar_wait_bounded(b2, p2, kWaitLimitNs));
         };
         auto issue_s = [&](int j) {
             ptx::tc_fence_after();
             // (columns of blocks past the context come out of stale rows;
             // the causal mask drops them)
-            const uint64_t kd = k_desc + (uint64_t)(((j % kTcKStages) * KV) >> 4);
+            const uint64_t kd = ptx::umma_desc_sw128(kstage(j % kTcKStages), 16,
+                                                     tc_group_bytes(D));
             if (ptx::elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
@@ -294,22 +304,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             __syncwarp();
         };
-        bool ok = wait(qready, 0) && wait(kfull, 0);
+        bool ok = ready(qready, 0, kfull, 0);
         if (ok)
             issue_s(0);
         for (int j = 0; ok && j < ntiles; ++j) {
-            if (__any_sync(kFull, *abort_flag != 0))
-                break;
             if (j + 1 < ntiles) {
-                if (!(ok = wait(sfree, (uint32_t)(j & 1)) &&
-                           wait(kfull + 8u * ((j + 1) % kTcKStages),
-                                (uint32_t)(((j + 1) / kTcKStages) & 1))))
+                if (!(ok = ready(sfree, (uint32_t)(j & 1), kfull + 8u * ((j + 1) % kTcKStages),
+                                 (uint32_t)(((j + 1) / kTcKStages) & 1))))
                     break;
                 issue_s(j + 1);
             }
             const int s = j & 1, vs = j % kTcVStages;
-            if (!(ok = wait(pready + 8u * s, (uint32_t)((j >> 1) & 1)) &&
-                       wait(vfull + 8u * vs, (uint32_t)((j / kTcVStages) & 1))))
+            if (!(ok = ready(pready + 8u * s, (uint32_t)((j >> 1) & 1), vfull + 8u * vs,
+                             (uint32_t)((j / kTcVStages) & 1))))
                 break;
             ptx::tc_fence_after();
             const int nbox = tc_boxes(j, ctx);
