@@ -61,9 +61,15 @@ def attention_bytes(layout: W.BatchLayout) -> int:
     return qo + kv
 
 
-def kernel_source_hash() -> str:
+# the sources each profiled kernel is built and launched from
+DECODE_SOURCES = ("pa.cu", "pa_inst_bf16.cu", "pa_kernels.cuh", "pa_launch.cuh", "pa_ptx.cuh")
+PREFILL_SOURCES = ("pa.cu", "pa_inst_prefill.cu", "pa_launch.cuh", "pa_prefill.cuh",
+                   "pa_prefill_tc.cuh", "pa_ptx.cuh")
+
+
+def kernel_source_hash(sources=DECODE_SOURCES) -> str:
     h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
+    for f in sorted(sources):
         with open(os.path.join(CSRC, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -77,16 +83,16 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic(summary=None):
+def profiled_traffic(summary=PROFILE_SUMMARY, sources=DECODE_SOURCES):
     """DRAM bytes per launch of a kernel from its committed ncu summary (the
-    decode kernel's by default), or None if the kernel sources changed since."""
+    decode kernel's by default), or None if its sources changed since."""
     try:
-        text = open(summary or PROFILE_SUMMARY).read()
+        text = open(summary).read()
     except OSError:
         return None
     m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
     m_bytes = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash(sources):
         return None
     return float(m_bytes.group(1))
 
@@ -595,7 +601,7 @@ def run_prefill(args, device):
         "attention_gbs": round(meta["bytes"] / (attn_ms * 1e-3) / 1e9, 1),
         "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                      "peak_source": src, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
-                     "traffic": profiled_traffic(PREFILL_PROFILE_SUMMARY),
+                     "traffic": profiled_traffic(PREFILL_PROFILE_SUMMARY, PREFILL_SOURCES),
                      "kernel": "pa_prefill_attention (prefill_tc_kernel<256, 4>: tcgen05.mma, "
                                "TMEM accumulators)",
                      "algorithmic_bytes_per_launch": meta["bytes"],

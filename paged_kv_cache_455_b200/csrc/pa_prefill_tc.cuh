@@ -6,8 +6,8 @@
 //
 // One CTA per (sequence, KV head, 128 query rows); row r is (token r / G,
 // query head r % G of the group), so one K/V tile serves the whole group.
-// Warps 0-3 own one query row per thread; warp 4 issues the MMAs, warps 5
-// and 6 the TMA copies of K and V.
+// Warps 0-3 own one query row per thread; warp 4 issues the S MMAs, warp 7
+// the P V MMAs, warps 5 and 6 the TMA copies of K and V.
 //
 //   producers (5, 6)    TMA: Q once; K tiles into four stages, V tiles into
 //                       three (one of each in the space Q held before it
@@ -16,13 +16,15 @@
 //                       lands as [8-token group][128-byte column][token]
 //                       [128 bytes] with 128-byte swizzle, so 8-token groups
 //                       are a fixed d * 16 bytes apart across the whole tile
-//   MMA (one thread)    S_j = Q K_j^T (M=128, N=64, K=16 steps) with Q read
-//                       from tensor memory and K from its stage; O += P_j V_j
-//                       (M=128, N=d, K=16 per block) with P_j read from
-//                       tensor memory and V MN-major straight from its stage;
-//                       whichever is ready first is issued.  A K stage is
-//                       free when its S is done, a V stage and a P buffer
-//                       when their P V is (tcgen05.commit)
+//   MMA (warps 4, 7)    S_j = Q K_j^T (M=128, N=64, K=16 steps) with Q read
+//                       from tensor memory and K from its stage (warp 4);
+//                       O += P_j V_j (M=128, N=d, K=16 per block) with P_j
+//                       read from tensor memory and V MN-major straight from
+//                       its stage (warp 7).  The two write disjoint tensor
+//                       memory and every reuse is guarded by a barrier, so
+//                       their waits overlap.  A K stage is free when its S is
+//                       done, a V stage and a P buffer when their P V is
+//                       (tcgen05.commit)
 //   softmax (warps 0-3) first move the CTA's Q rows from shared to tensor
 //                       memory; then per tile: S row from tensor memory (the
 //                       S buffer is released as soon as it is read), causal
@@ -48,7 +50,7 @@ constexpr int kTcTile = 64;             // KV tokens per stage
 constexpr int kTcBoxes = kTcTile / 16;  // 16-token blocks per tile
 constexpr int kTcKStages = 4;           // three after Q, one where Q was
 constexpr int kTcVStages = 3;           // two after the K stages, one where Q was
-constexpr int kTcThreads = 224;         // 4 softmax warps, MMA warp, 2 TMA warps
+constexpr int kTcThreads = 256;         // 4 softmax warps, 2 MMA warps, 2 TMA warps
 
 // Shared memory layout (bytes from the 1024-aligned base), per head dim:
 // Q (then K stage 3, V stage 2) | K stages 0-2 | V stages 0, 1 | barriers.
@@ -189,7 +191,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (bad) {
         if (tid == 0)
             report(p.dev_status, PA_DEV_BAD_BLOCK);
-    } else if (warp >= 5) {
+    } else if (warp == 5 || warp == 6) {
         // ================================================ TMA producers
         // warp 5 copies K (and Q), warp 6 copies V; lane x issues box x
         // (tokens 16 x .. 16 x + 15) of each tile
@@ -265,14 +267,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                        kWaitLimitNs);
         }
         __syncwarp();
-    } else if (warp == 4) {
+    } else if (warp == 4 || warp == 7) {
         // ================================================ MMA issue
-        // Order: S_0, then per tile j: S_{j+1} (ready once the softmax has
-        // read S_j out of tensor memory and K_{j+1} has landed), P_j V_j
-        // (ready once the softmax has written P_j and V_j has landed).  The
-        // whole warp waits (suspending, so it takes no issue slots from the
-        // softmax warps); one elected lane, always lane 0, issues the MMAs
-        // and their commits.
+        // Warp 4: S_0, then S_{j+1} once the softmax has read S_j out of
+        // tensor memory and K_{j+1} has landed.  Warp 7: P_j V_j once the
+        // softmax has written P_j and V_j has landed.  Each whole warp waits
+        // (suspending, so it takes no issue slots from the softmax warps);
+        // one elected lane, always lane 0, issues the MMAs and their commits
+        // (a commit tracks the MMAs of its own thread).
         // descriptors: K is K-major, 8-token groups d * 16 bytes apart; V is
         // MN-major, 64-element columns 1024 bytes apart, 8-token groups
         // d * 16 bytes apart
@@ -304,16 +306,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             __syncwarp();
         };
-        bool ok = ready(qready, 0, kfull, 0);
-        if (ok)
-            issue_s(0);
-        for (int j = 0; ok && j < ntiles; ++j) {
-            if (j + 1 < ntiles) {
+        bool ok = true;
+        if (warp == 4) {
+            ok = ready(qready, 0, kfull, 0);
+            if (ok)
+                issue_s(0);
+            for (int j = 0; ok && j + 1 < ntiles; ++j) {
                 if (!(ok = ready(sfree, (uint32_t)(j & 1), kfull + 8u * ((j + 1) % kTcKStages),
                                  (uint32_t)(((j + 1) / kTcKStages) & 1))))
                     break;
                 issue_s(j + 1);
             }
+        }
+        for (int j = 0; warp == 7 && ok && j < ntiles; ++j) {
             const int s = j & 1, vs = j % kTcVStages;
             if (!(ok = ready(pready + 8u * s, (uint32_t)((j >> 1) & 1), vfull + 8u * vs,
                              (uint32_t)((j / kTcVStages) & 1))))
