@@ -31,7 +31,7 @@
 //                       mask on diagonal tiles, running max; O rescaled in
 //                       tensor memory only when the max grew by more than
 //                       2^8; P = 2^(s - m) as bf16 into P buffer j % 2 of
-//                       tensor memory; row sum in fp32 of the rounded values
+//                       tensor memory; row sum in fp32 of the fp32 weights
 //
 // Tensor memory columns: S [0, 64), O [64, 64 + d), Q (d / 2 columns: two
 // bf16 per column) at 64 + d, P buffers (32 columns) after it.  With Q in
@@ -485,12 +485,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                w0[k] = ptx::pack_bf16x2(ptx::ex2(fmaf(sv[2 * k], sc, nref)),
-                                         ptx::ex2(fmaf(sv[2 * k + 1], sc, nref)));
-                w1[k] = ptx::pack_bf16x2(ptx::ex2(fmaf(sv[32 + 2 * k], sc, nref)),
-                                         ptx::ex2(fmaf(sv[32 + 2 * k + 1], sc, nref)));
-                l4[k & 3] += (ptx::bf16lo_to_f32(w0[k]) + ptx::bf16hi_to_f32(w0[k])) +
-                             (ptx::bf16lo_to_f32(w1[k]) + ptx::bf16hi_to_f32(w1[k]));
+                const float e0 = ptx::ex2(fmaf(sv[2 * k], sc, nref));
+                const float e1 = ptx::ex2(fmaf(sv[2 * k + 1], sc, nref));
+                const float e2 = ptx::ex2(fmaf(sv[32 + 2 * k], sc, nref));
+                const float e3 = ptx::ex2(fmaf(sv[32 + 2 * k + 1], sc, nref));
+                w0[k] = ptx::pack_bf16x2(e0, e1);
+                w1[k] = ptx::pack_bf16x2(e2, e3);
+                l4[k & 3] += (e0 + e1) + (e2 + e3);
             }
             l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
             if (j >= 2) {
