@@ -60,7 +60,8 @@ def _oracle(q, kp, vp, tables, lens, cu, scale):
 
 
 @pytest.mark.parametrize("d,hq,hkv,bs", [(256, 16, 4, 16), (128, 8, 8, 32), (64, 16, 2, 4),
-                                         (128, 16, 8, 8), (256, 8, 4, 32)])
+                                         (128, 16, 8, 8), (256, 8, 4, 32), (64, 16, 2, 16),
+                                         (128, 32, 4, 32), (256, 8, 1, 16)])
 def test_random_chunks_match_oracle(pa, d, hq, hkv, bs):
     ctxs = [1, 40, 300, 97, 513, 64]
     chunks = [1, 40, 37, 1, 129, 33]           # whole prompts, prefix + chunk, single tokens
