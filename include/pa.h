@@ -206,7 +206,11 @@ pa_status pa_splitk_reduce(void *out, const float *tmp_out, const float *max_log
  * bf16 only (fp32 returns PA_ERR_UNSUPPORTED); group 1, 2, 4 or 8; contexts
  * up to 2048 blocks.  A chunk longer than its context, a context beyond the
  * table, or rows outside [0, total_q) set PA_DEV_BAD_CONTEXT (its rows that
- * exist are zeros); an invalid block id sets PA_DEV_BAD_BLOCK (zeros).
+ * exist are zeros); an invalid block id sets PA_DEV_BAD_BLOCK (zeros); a
+ * wait inside the kernel that runs out sets PA_DEV_WAIT_TIMEOUT.
+ * Arithmetic: scores and the softmax in fp32; the softmax weights are
+ * rounded to bf16 for the P.V product (their fp32 values make the row sum);
+ * P.V accumulates in fp32; the output is rounded to bf16.
  */
 pa_status pa_prefill_attention(void *out, const void *query, const int32_t *cu_q_lens, int total_q,
                                int max_q_len, const void *k_pool, const void *v_pool,
