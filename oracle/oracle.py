@@ -281,7 +281,10 @@ def threads(num_threads: int = 0) -> int:
 # --------------------------------------------------------------------------
 
 def to_f64(a: np.ndarray, dtype: str) -> np.ndarray:
-    """Exact conversion of f32 / raw-bf16 data to float64."""
+    """Exact conversion of f32 / raw-bf16 data to float64 ("f64" data is
+    returned as it is)."""
+    if dtype == "f64":
+        return np.asarray(a, dtype=np.float64)
     if dtype == "f32":
         return np.asarray(a, dtype=np.float32).astype(np.float64)
     bits = np.asarray(a, dtype=np.uint16).astype(np.uint32) << 16
@@ -398,3 +401,88 @@ def prefill_attention_np(q, k_pool, v_pool, block_tables, context_lens, cu_q_len
             out[q0:q0 + n, h] = (p @ vh) / p.sum(axis=1, keepdims=True)
     return out
 
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) KV cache (numpy, fp64)
+#
+# A quantised cache halves the bytes a bandwidth-bound decode step reads
+# ("vLLM Architecture, Memory and Benchmarks Deep Dive", section 4, FP8:
+# fewer bytes per value double the effective memory bandwidth; "Inside vLLM:
+# Anatomy of a High-Throughput LLM Inference System", FAQ: quantized KV
+# caches).  Reading taken where the pages give no format: each pool element
+# is one E4M3 byte with a per-tensor scale, K = code value * k_scale and
+# V = code value * v_scale; the cache write stores the E4M3 code of
+# x / scale, the division taken in binary32, rounded to nearest (ties to the
+# even code) and saturated to +-448.
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Value of each E4M3 byte: bit 7 is the sign, bits 6..3 the exponent
+    (bias 7), bits 2..0 the mantissa; exponent field 0 holds the subnormals
+    m * 2^-9; 0x7f and 0xff are NaN; there are no infinities."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return np.where((c & 0x80) != 0, -mag, mag)
+
+
+def f32_to_e4m3(x) -> np.ndarray:
+    """E4M3 code (uint8) of each binary32 value: the nearest of the 127
+    non-negative finite magnitudes (ties to the even code), magnitudes above
+    448 (infinities included) saturating to 448, the sign kept (also for
+    zero); NaN gives 0x7f."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    grid = e4m3_to_f64(np.arange(0x7F, dtype=np.uint8))      # codes 0..126, increasing
+    nan = np.isnan(x)
+    a = np.minimum(np.abs(np.where(nan, 0.0, x)), E4M3_MAX)
+    hi = np.clip(np.searchsorted(grid, a, side="left"), 0, 0x7E)
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - grid[lo], grid[hi] - a
+    tie_pick = np.where(lo % 2 == 0, lo, hi)
+    code = np.where(d_hi < d_lo, hi, np.where(d_lo < d_hi, lo, tie_pick))
+    code = np.where(np.signbit(x), code | 0x80, code)
+    return np.where(nan, 0x7F, code).astype(np.uint8)
+
+
+def quantize_e4m3(x, scale: float) -> np.ndarray:
+    """E4M3 codes of x / scale, the division taken in binary32."""
+    y = np.asarray(x, dtype=np.float32) / np.float32(scale)
+    return f32_to_e4m3(y)
+
+
+def dequantize_e4m3(codes, scale: float) -> np.ndarray:
+    """fp64 values code * scale (exact: a code has at most 4 significant bits,
+    a binary32 scale 24)."""
+    return e4m3_to_f64(codes) * float(np.float32(scale))
+
+
+def reshape_and_cache_fp8_np(key, value, k_pool, v_pool, slot_mapping, k_scale: float,
+                             v_scale: float):
+    """Cache write into E4M3 pools: key/value are raw bf16 [T, Hkv, d], pools
+    uint8 codes [nb, bs, Hkv, d]; each token's rows become the codes of
+    key / k_scale and value / v_scale (``quantize_e4m3``) at its slot.
+    Negative slots are skipped; a slot past the pool raises ValueError."""
+    kq = quantize_e4m3(to_f64(key, "bf16").astype(np.float32), k_scale)
+    vq = quantize_e4m3(to_f64(value, "bf16").astype(np.float32), v_scale)
+    return reshape_and_cache_np(kq, vq, np.asarray(k_pool, dtype=np.uint8),
+                                np.asarray(v_pool, dtype=np.uint8), slot_mapping)
+
+
+def paged_attention_fp8_np(q, k_pool, v_pool, block_tables, context_lens, scale: float,
+                           k_scale: float, v_scale: float) -> np.ndarray:
+    """Exact fp64 decode attention over an E4M3 cache: the query is raw bf16,
+    the pools' codes are dequantised exactly (``dequantize_e4m3``) and the
+    result is the definition of ``paged_attention_np`` on those values."""
+    return paged_attention_np(to_f64(q, "bf16"), dequantize_e4m3(k_pool, k_scale),
+                              dequantize_e4m3(v_pool, v_scale), block_tables, context_lens,
+                              scale, "f64")
+
+
+__all__ += ["E4M3_MAX", "e4m3_to_f64", "f32_to_e4m3", "quantize_e4m3", "dequantize_e4m3",
+            "reshape_and_cache_fp8_np", "paged_attention_fp8_np"]
