@@ -38,10 +38,16 @@
  *     output is zeros (attention) or left untouched (cache write).
  *   - Inputs and outputs must not overlap.
  *   - Every call is asynchronous on `stream` and keeps stream order.  The
- *     attention kernels are launched as programmatic dependents of the
- *     kernel before them on the stream, so their set-up overlaps its tail;
- *     they read and write no memory before that kernel has completed.  The
- *     cache write lets the attention that follows start its set-up early.
+ *     decode and cache-write kernels are launched as programmatic dependents
+ *     of the kernel before them on the stream (programmatic dependent
+ *     launch), and each lets the kernel after it start early, so that a
+ *     kernel's set-up overlaps the tail of the one ahead.  The cache write
+ *     touches no memory before the kernel ahead has completed.  The decode
+ *     kernels read context_lens and block_tables before it has completed
+ *     (everything else after): a kernel ahead of them that allows an early
+ *     start (griddepcontrol.launch_dependents) must not write those two
+ *     arrays.  Kernels that do not allow an early start, host copies and
+ *     this library's own kernels need no care.
  */
 #ifndef PA_H_
 #define PA_H_
@@ -63,7 +69,8 @@ typedef enum pa_status {
 
 typedef enum pa_dtype {
     PA_DTYPE_F32 = 0,
-    PA_DTYPE_BF16 = 1
+    PA_DTYPE_BF16 = 1,
+    PA_DTYPE_FP8_E4M3 = 2   /* pools only: pa_copy_blocks, pa_swap_blocks */
 } pa_dtype;
 
 /* Bits a kernel ORs into *dev_status. */
@@ -221,6 +228,53 @@ pa_status pa_prefill_attention(void *out, const void *query, const int32_t *cu_q
                                int32_t *dev_status, void *stream);
 
 /*
+ * FP8 cache ("vLLM Architecture, Memory and Benchmarks Deep Dive", section 4,
+ * FP8: fewer bytes per value double the effective memory bandwidth of a
+ * bandwidth-bound step; "Inside vLLM: Anatomy of a High-Throughput LLM
+ * Inference System", FAQ: quantized KV caches).  The pages fix no format;
+ * this library's reading: every pool element is one E4M3 byte (OCP FP8:
+ * sign, 4 exponent bits of bias 7, 3 mantissa bits, subnormals, no
+ * infinities, 0x7f / 0xff NaN), with one scale per tensor:
+ *   K = code * k_scale,  V = code * v_scale.
+ * Queries, new keys and values, and outputs stay bf16.  Supported: d 128 or
+ * 256, blocks of 16 or 32 tokens, Hq / Hkv in {1, 2, 4, 8}.  Pools are
+ * [nb, bs, Hkv, d] bytes.
+ *
+ * pa_reshape_and_cache_fp8 -- the cache write: each element x of a token's
+ * key (value) row is stored as the E4M3 code of x / k_scale (x / v_scale),
+ * the division rounded as binary32, then rounded to the nearest code (ties
+ * to the even code) with finite overflow saturating to +-448.  key, value:
+ * device [num_tokens, Hkv, d] bf16; other arguments and errors as in
+ * pa_reshape_and_cache; scales must be positive and finite
+ * (PA_ERR_INVALID_ARG otherwise).
+ */
+pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_pool, void *v_pool,
+                                   const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                                   int head_dim, int block_size, int64_t num_blocks,
+                                   float k_scale, float v_scale, int32_t *dev_status, void *stream);
+
+/*
+ * pa_decode_attention_fp8 -- pa_decode_attention over an E4M3 cache: the
+ * result is the definition of pa_decode_attention with K and V replaced by
+ * their dequantised values code * k_scale and code * v_scale.  query and out
+ * are bf16 [B, Hq, d]; other arguments, the workspace and the errors as in
+ * pa_decode_attention (pa_decode_workspace_bytes sizes the workspace).
+ * Arithmetic: codes convert exactly to f16; the query is rounded to f16
+ * (components must stay below 65504 in magnitude; those below 2^-14 keep
+ * f16's subnormal precision); logits, the softmax and the accumulators are
+ * fp32; the softmax weights are rounded to f16 for the P.V product (the same
+ * rounded weights make the row sum); the output is rounded to bf16.
+ */
+pa_status pa_decode_attention_fp8(void *out, const void *query, const void *k_pool,
+                                  const void *v_pool, const int32_t *block_tables,
+                                  int max_blocks_per_seq, const int32_t *context_lens,
+                                  int num_seqs, int max_context_len, int num_q_heads,
+                                  int num_kv_heads, int head_dim, int block_size,
+                                  int64_t num_blocks, float scale, float k_scale, float v_scale,
+                                  void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                                  void *stream);
+
+/*
  * pa_copy_blocks -- copy whole physical blocks of both pools, the copy that
  * copy-on-write block sharing needs ("vLLM Architecture, Memory and
  * Benchmarks Deep Dive", section 2, "Copy-on-Write (CoW) Branching": rollouts
@@ -233,7 +287,8 @@ pa_status pa_prefill_attention(void *out, const void *query, const int32_t *cu_q
  *                  Destinations must be distinct and must not be the source
  *                  of another pair of the same call (the copies run
  *                  concurrently).
- *   k_pool,v_pool  device, [nb, bs, Hkv, d] in `dtype`.
+ *   k_pool,v_pool  device, [nb, bs, Hkv, d] in `dtype` (PA_DTYPE_FP8_E4M3
+ *                  for an FP8 cache).
  * A source or destination outside [0, nb) sets PA_DEV_BAD_BLOCK and that
  * pair is skipped.  num_pairs == 0 launches nothing.
  */
@@ -256,7 +311,8 @@ pa_status pa_copy_blocks(void *k_pool, void *v_pool, const int64_t *block_mappin
  * `stream`.
  *   block_mapping  device (or mapped host), [num_pairs][2] int64.
  *                  Destinations must be distinct.
- *   pools          [nb, bs, Hkv, d] in `dtype`, nb given per side.
+ *   pools          [nb, bs, Hkv, d] in `dtype` (PA_DTYPE_FP8_E4M3 for an FP8
+ *                  cache), nb given per side.
  * A block id outside its pool sets PA_DEV_BAD_BLOCK and that pair is
  * skipped.  The source and destination ranges must not overlap.  A pointer
  * the GPU cannot address as it is (pageable host memory, for instance)
@@ -278,25 +334,34 @@ pa_status pa_swap_blocks(void *dst_k_pool, void *dst_v_pool, int64_t dst_num_blo
  * device memory is owned by another framework, and code paths where an
  * allocation (which may synchronise the device) is not allowed.  This call
  * computes the same result as pa_decode_attention with a sufficient
- * workspace, using instead a fixed scratch array of PA_STATIC_SCRATCH_BYTES
- * that every device holds in device memory from the moment it loads the
- * library until the process exits.  It never calls cudaMalloc, cudaFree or
- * any allocating routine.
+ * workspace (bit for bit: the same kernel, grid and merge order), using
+ * instead a fixed scratch array of PA_STATIC_SCRATCH_BYTES in device memory.
+ * The call itself never calls cudaMalloc, cudaFree or any allocating
+ * routine.
  *
  *   Arguments are those of pa_decode_attention without the workspace.
  *   Returns PA_ERR_WORKSPACE, launching nothing, when these sizes need more
  *   scratch than PA_STATIC_SCRATCH_BYTES: about 33 KB per SM for
  *   Hkv = 4, Hq / Hkv = 4, d = 256 (fits), 66 KB per SM for Hq / Hkv = 8,
- *   d = 256 (refused on a 148-SM GPU).
- *   The first call on a device looks up the array's device address (a CUDA
- *   runtime query, no allocation); make that first call before any stream
- *   capture.  All calls share the one array: calls whose kernels overlap on
- *   the GPU (other streams, other threads) race and corrupt each other's
- *   results, so serialise them.  The array keeps the last call's contents
- *   and no word of it needs to start at zero: a call counts the partial
- *   results of a split sequence in counter words tagged with that call's
- *   own tag (a word with another tag counts as zero), and reads partial
- *   results only once its own count is complete.
+ *   d = 256 (refused on a 148-SM GPU).  It refuses rather than falling back
+ *   to pa_decode_attention's workspace-free decomposition, which can be much
+ *   slower for long contexts: such a caller should pass a workspace.
+ *   The array lives in the library's device code.  Once that code is loaded
+ *   on a device, the device holds the array until the process exits.  The
+ *   CUDA runtime may load it lazily (the default since CUDA 12.2): then the
+ *   first call of this library on a device loads it, which places the
+ *   8 MiB array in device memory (an allocation made by the driver, not by
+ *   this call) and may synchronise the device.  The first call of this
+ *   entry point on a device also looks up the array's device address (a
+ *   CUDA runtime query).  So make a first call on each device at start-up,
+ *   outside any stream capture and any section that must not allocate.
+ *   All calls share the one array: calls whose kernels overlap on the GPU
+ *   (other streams, other threads) race and corrupt each other's results,
+ *   so serialise them.  The array keeps the last call's contents and no
+ *   word of it needs to start at zero: a call counts the partial results of
+ *   a split sequence in counter words tagged with that call's own tag (a
+ *   word with another tag counts as zero), and reads partial results only
+ *   once its own count is complete.
  */
 #define PA_STATIC_SCRATCH_BYTES (8u << 20)
 pa_status pa_decode_attention_static(void *out, const void *query, const void *k_pool,

@@ -19,9 +19,9 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpa.so")
 SOURCES = [os.path.join(CSRC, f) for f in
            ("pa.cu", "pa_inst_f32.cu", "pa_inst_bf16.cu", "pa_inst_bf16_simt.cu",
-            "pa_inst_prefill.cu")]
+            "pa_inst_fp8.cu", "pa_inst_prefill.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + \
-    [os.path.join(INCLUDE, "pa.h")]
+    [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
 OBJ_DIR = os.path.join(PKG, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -15,11 +15,15 @@
 #include <cstring>
 #include <mutex>
 
+#include <cmath>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "pa.h"
+#include "pa_testing.h"
 #include "pa_launch.cuh"
 #include "pa_prefill.cuh"
 
@@ -30,6 +34,11 @@ using pa::DecodeParams;
 using pa::TileGeo;
 
 std::atomic<unsigned long long> g_launches{0};
+
+// Test hooks (include/pa_testing.h): the bounded-wait limit of the decode
+// kernels and a CTA that withholds its cut pieces.
+std::atomic<unsigned long long> g_test_wait_ns{0};
+std::atomic<int> g_test_withhold{-1};
 
 // Bound on decode CTAs used to size the stream-K workspace (one per SM, up
 // to 256 SMs).
@@ -47,7 +56,7 @@ int ilog2_exact(int v)
 
 int64_t round_up(int64_t v, int64_t m) { return ((v + m - 1) / m) * m; }
 
-int elem_size(pa_dtype dt) { return dt == PA_DTYPE_F32 ? 4 : 2; }
+int elem_size(pa_dtype dt) { return dt == PA_DTYPE_F32 ? 4 : (dt == PA_DTYPE_FP8_E4M3 ? 1 : 2); }
 
 // =====================================================================
 // Cache write kernel: one warp per (token, KV head, K|V) row, 16-byte copies.
@@ -70,6 +79,9 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const CacheParams p)
     // the decode kernel that follows may start its set-up now; it waits for
     // this grid to finish before reading the pools
     pa::ptx::grid_launch_dependents();
+    // launched as a programmatic dependent of the kernel ahead: its inputs
+    // (and readers of the pools) must be done before anything is touched
+    pa::ptx::grid_wait_prerequisites();
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t nrows = (int64_t)p.num_tokens * p.num_kv_heads * 2;
@@ -94,6 +106,73 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const CacheParams p)
     const int n16 = p.row_bytes >> 4;
     for (int c = lane; c < n16; c += 32)
         dst[c] = __ldg(src + c);
+}
+
+struct CacheFp8Params {
+    const __nv_bfloat16 *key;
+    const __nv_bfloat16 *value;
+    uint8_t *k_pool;
+    uint8_t *v_pool;
+    const int64_t *slot_mapping;
+    int32_t *dev_status;
+    int64_t num_slots;      // nb * bs
+    int num_tokens;
+    int num_kv_heads;
+    int head_dim;
+    float k_scale;
+    float v_scale;
+};
+
+// Cache write into E4M3 pools: one warp per (token, KV head, K|V) row; a
+// lane turns 8 bf16 elements into the E4M3 codes of element / scale (the
+// division rounded as binary32, then to nearest E4M3, ties to even,
+// saturating at +-448) and stores them as one 8-byte word.
+__global__ void __launch_bounds__(256) cache_write_fp8_kernel(const CacheFp8Params p)
+{
+    pa::ptx::grid_launch_dependents();
+    pa::ptx::grid_wait_prerequisites();
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t nrows = (int64_t)p.num_tokens * p.num_kv_heads * 2;
+    if (row >= nrows)
+        return;
+    const int kv = (int)(row & 1);
+    const int64_t th = row >> 1;
+    const int64_t t = th / p.num_kv_heads;
+    const int64_t h = th - t * p.num_kv_heads;
+    const int64_t slot = p.slot_mapping[t];
+    if (slot < 0)
+        return;
+    if (slot >= p.num_slots) {
+        if (lane == 0 && h == 0 && kv == 0)
+            pa::report(p.dev_status, PA_DEV_BAD_SLOT);
+        return;
+    }
+    const float sc = kv ? p.v_scale : p.k_scale;
+    const uint4 *src = reinterpret_cast<const uint4 *>((kv ? p.value : p.key) +
+                                                       (t * p.num_kv_heads + h) * p.head_dim);
+    uint2 *dst = reinterpret_cast<uint2 *>((kv ? p.v_pool : p.k_pool) +
+                                           (slot * p.num_kv_heads + h) * p.head_dim);
+    for (int c = lane; c < (p.head_dim >> 3); c += 32) {
+        const uint4 in = __ldg(src + c);
+        const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+        uint32_t packed[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            uint32_t v = 0;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const uint32_t b = w[2 * i + j];
+                const float x0 = __fdiv_rn(pa::ptx::bf16lo_to_f32(b), sc);
+                const float x1 = __fdiv_rn(pa::ptx::bf16hi_to_f32(b), sc);
+                const uint32_t two = (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(x0, x1),
+                                                                        __NV_SATFINITE, __NV_E4M3);
+                v |= (two & 0xffffu) << (16 * j);
+            }
+            packed[i] = v;
+        }
+        dst[c] = make_uint2(packed[0], packed[1]);
+    }
 }
 
 struct CopyParams {
@@ -154,7 +233,7 @@ pa_status launch_copy(CopyParams &p, int block_size, int num_kv_heads, int head_
 {
     if (p.num_pairs < 0 || p.src_blocks <= 0 || p.dst_blocks <= 0 || num_kv_heads <= 0)
         return PA_ERR_INVALID_ARG;
-    if (dtype != PA_DTYPE_F32 && dtype != PA_DTYPE_BF16)
+    if (dtype != PA_DTYPE_F32 && dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP8_E4M3)
         return PA_ERR_UNSUPPORTED;
     if (head_dim != 64 && head_dim != 128 && head_dim != 256)
         return PA_ERR_UNSUPPORTED;
@@ -249,7 +328,9 @@ bool encode_pool_map(CUtensorMap *out, const void *base, int64_t nb, int bs, int
     if (!enc)
         return false;
     const CUtensorMapDataType type =
-        dt == PA_DTYPE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        dt == PA_DTYPE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                           : (dt == PA_DTYPE_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                      : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     const cuuint32_t epc = 128 / es;           // elements per 128-byte column
     const cuuint64_t rowb = (cuuint64_t)d * es;
     const cuuint32_t nch = (cuuint32_t)(rowb / 128);
@@ -290,7 +371,7 @@ bool encode_pool_map(CUtensorMap *out, const void *base, int64_t nb, int bs, int
 // KV heads per CTA tile: the largest of 4, 2, 1 dividing Hkv.
 int heads_per_cta(int hkv) { return hkv % 4 == 0 ? 4 : (hkv % 2 == 0 ? 2 : 1); }
 
-bool make_geo(TileGeo &g, int D, int es, int bs, int group, int hpc, int *smem)
+bool make_geo(TileGeo &g, int D, int es, int es_q, int bs, int group, int hpc, int *smem)
 {
     const int rowb = D * es;
     const int nch = rowb / 128;
@@ -301,7 +382,7 @@ bool make_geo(TileGeo &g, int D, int es, int bs, int group, int hpc, int *smem)
     g.head_lines = nch * g.tr;
     g.box_stride = (int)round_up((int64_t)hpc * g.head_lines * 128, 1024);
     g.kv_bytes = g.bpt * g.box_stride;
-    g.q_head_bytes = group * D * es;
+    g.q_head_bytes = group * D * es_q;
     g.q_bytes = hpc * g.q_head_bytes;
     g.q_off = 2 * g.kv_bytes;
     g.stage_bytes = (int)round_up((int64_t)g.q_off + g.q_bytes, 1024);
@@ -325,6 +406,8 @@ bool bf16_use_mma()
 
 pa_status decode_call(DecodeLaunch &L, pa_dtype dtype, int *grid, bool launch)
 {
+    if (L.kv8)
+        return pa::decode_fp8(L, grid, launch);
     if (dtype == PA_DTYPE_F32)
         return pa::decode_f32(L, grid, launch);
     if (bf16_use_mma())
@@ -381,7 +464,8 @@ pa_status prepare_decode(DecodeLaunch &L, void *out, const void *query, const vo
                          const int32_t *context_lens, int num_seqs, int num_q_heads,
                          int num_kv_heads, int head_dim, int block_size, int bs_log2,
                          int64_t num_blocks, float scale, pa_dtype dtype, int group,
-                         int32_t *dev_status, void *stream)
+                         int32_t *dev_status, void *stream, bool kv8 = false,
+                         float k_scale = 1.f, float v_scale = 1.f)
 {
     std::memset(&L.p, 0, sizeof(L.p));
     DecodeParams &p = L.p;
@@ -397,21 +481,28 @@ pa_status prepare_decode(DecodeLaunch &L, void *out, const void *query, const vo
     p.max_blocks = max_blocks;
     p.block_size = block_size;
     p.bs_log2 = bs_log2;
-    p.scale_log2 = scale * pa::kLog2e;
+    // an FP8 cache's K scale multiplies every logit, its V scale every output
+    p.scale_log2 = kv8 ? scale * k_scale * pa::kLog2e : scale * pa::kLog2e;
+    p.out_scale = kv8 ? v_scale : 1.f;
+    const unsigned long long wait_ns = g_test_wait_ns.load();
+    p.wait_ns = wait_ns ? wait_ns : pa::kWaitLimitNs;
+    p.withhold_cta = g_test_withhold.load();
     L.head_dim = head_dim;
     L.group = group;
     L.tr16 = block_size >= 16;
+    L.kv8 = kv8;
     L.stream = static_cast<cudaStream_t>(stream);
-    const int es = elem_size(dtype);
+    const pa_dtype pool_dtype = kv8 ? PA_DTYPE_FP8_E4M3 : dtype;
+    const int es = elem_size(pool_dtype);
     const int tr = std::min(16, block_size);
     const int hpc = heads_per_cta(num_kv_heads);
     p.head_groups = num_kv_heads / hpc;
-    if (!make_geo(p.geo, head_dim, es, block_size, group, hpc, &L.smem_bytes))
+    if (!make_geo(p.geo, head_dim, es, elem_size(dtype), block_size, group, hpc, &L.smem_bytes))
         return PA_ERR_UNSUPPORTED;
-    if (!encode_pool_map(&L.tmap_k, k_pool, num_blocks, block_size, num_kv_heads, head_dim, dtype,
-                         tr, hpc) ||
-        !encode_pool_map(&L.tmap_v, v_pool, num_blocks, block_size, num_kv_heads, head_dim, dtype,
-                         tr, hpc))
+    if (!encode_pool_map(&L.tmap_k, k_pool, num_blocks, block_size, num_kv_heads, head_dim,
+                         pool_dtype, tr, hpc) ||
+        !encode_pool_map(&L.tmap_v, v_pool, num_blocks, block_size, num_kv_heads, head_dim,
+                         pool_dtype, tr, hpc))
         return PA_ERR_CUDA;
     return PA_OK;
 }
@@ -572,6 +663,10 @@ const char *pa_status_string(pa_status status)
 
 unsigned long long pa_launch_count(void) { return g_launches.load(); }
 
+void pa_testing_set_wait_limit_ns(unsigned long long ns) { g_test_wait_ns.store(ns); }
+
+void pa_testing_withhold_pieces(int cta) { g_test_withhold.store(cta < 0 ? -1 : cta); }
+
 int pa_num_partitions(int max_context_len, int partition_size)
 {
     if (partition_size <= 0 || max_context_len <= 0)
@@ -631,9 +726,69 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_pool,
     const int64_t blocks = (rows + 7) / 8;   // 8 warps per CTA
     if (blocks > INT32_MAX)
         return PA_ERR_INVALID_ARG;
-    cache_write_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    // a programmatic dependent of the kernel ahead (its CTAs may be placed on
+    // SMs that kernel has left, and wait there for it to complete)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, cache_write_kernel, p);
     ++g_launches;
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_pool, void *v_pool,
+                                   const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                                   int head_dim, int block_size, int64_t num_blocks,
+                                   float k_scale, float v_scale, int32_t *dev_status, void *stream)
+{
+    if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+        return PA_ERR_INVALID_ARG;
+    if ((head_dim != 128 && head_dim != 256) || (block_size != 16 && block_size != 32))
+        return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0)
+        return PA_OK;
+    if (!key || !value || !k_pool || !v_pool || !slot_mapping)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_pool) || !aligned16(v_pool))
+        return PA_ERR_INVALID_ARG;
+    CacheFp8Params p;
+    p.key = static_cast<const __nv_bfloat16 *>(key);
+    p.value = static_cast<const __nv_bfloat16 *>(value);
+    p.k_pool = static_cast<uint8_t *>(k_pool);
+    p.v_pool = static_cast<uint8_t *>(v_pool);
+    p.slot_mapping = slot_mapping;
+    p.dev_status = dev_status;
+    p.num_slots = num_blocks * block_size;
+    p.num_tokens = num_tokens;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    const int64_t rows = (int64_t)num_tokens * num_kv_heads * 2;
+    const int64_t blocks = (rows + 7) / 8;   // 8 warps per CTA
+    if (blocks > INT32_MAX)
+        return PA_ERR_INVALID_ARG;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, cache_write_fp8_kernel, p);
+    ++g_launches;
+    return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_copy_blocks(void *k_pool, void *v_pool, const int64_t *block_mapping, int num_pairs,
@@ -844,13 +999,16 @@ pa_status pa_splitk_reduce(void *out, const float *tmp_out, const float *max_log
                          static_cast<cudaStream_t>(stream));
 }
 
-pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
+// pa_decode_attention and pa_decode_attention_fp8 (kv8: E4M3 pools with
+// scales, bf16 query and output).
+static pa_status decode_entry(void *out, const void *query, const void *k_pool,
                               const void *v_pool, const int32_t *block_tables,
                               int max_blocks_per_seq, const int32_t *context_lens, int num_seqs,
                               int max_context_len, int num_q_heads, int num_kv_heads,
                               int head_dim, int block_size, int64_t num_blocks, float scale,
                               pa_dtype dtype, void *workspace, size_t workspace_bytes,
-                              int32_t *dev_status, void *stream)
+                              int32_t *dev_status, void *stream, bool kv8, float k_scale,
+                              float v_scale)
 {
     int group = 0, bs_log2 = 0;
     pa_status st = check_attention_args(out, query, k_pool, v_pool, block_tables,
@@ -864,7 +1022,8 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
     DecodeLaunch L;
     st = prepare_decode(L, out, query, k_pool, v_pool, block_tables, max_blocks_per_seq,
                         context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                        bs_log2, num_blocks, scale, dtype, group, dev_status, stream);
+                        bs_log2, num_blocks, scale, dtype, group, dev_status, stream, kv8,
+                        k_scale, v_scale);
     if (st != PA_OK)
         return st;
     DecodeParams &p = L.p;
@@ -902,6 +1061,39 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
     if (st == PA_OK && stream_k && grid != want)
         return PA_ERR_CUDA;   // capacity changed between query and launch
     return st;
+}
+
+pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
+                              const void *v_pool, const int32_t *block_tables,
+                              int max_blocks_per_seq, const int32_t *context_lens, int num_seqs,
+                              int max_context_len, int num_q_heads, int num_kv_heads,
+                              int head_dim, int block_size, int64_t num_blocks, float scale,
+                              pa_dtype dtype, void *workspace, size_t workspace_bytes,
+                              int32_t *dev_status, void *stream)
+{
+    return decode_entry(out, query, k_pool, v_pool, block_tables, max_blocks_per_seq,
+                        context_lens, num_seqs, max_context_len, num_q_heads, num_kv_heads,
+                        head_dim, block_size, num_blocks, scale, dtype, workspace,
+                        workspace_bytes, dev_status, stream, false, 1.f, 1.f);
+}
+
+pa_status pa_decode_attention_fp8(void *out, const void *query, const void *k_pool,
+                                  const void *v_pool, const int32_t *block_tables,
+                                  int max_blocks_per_seq, const int32_t *context_lens,
+                                  int num_seqs, int max_context_len, int num_q_heads,
+                                  int num_kv_heads, int head_dim, int block_size,
+                                  int64_t num_blocks, float scale, float k_scale, float v_scale,
+                                  void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                                  void *stream)
+{
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+        return PA_ERR_INVALID_ARG;
+    if ((head_dim != 128 && head_dim != 256) || (block_size != 16 && block_size != 32))
+        return PA_ERR_UNSUPPORTED;
+    return decode_entry(out, query, k_pool, v_pool, block_tables, max_blocks_per_seq,
+                        context_lens, num_seqs, max_context_len, num_q_heads, num_kv_heads,
+                        head_dim, block_size, num_blocks, scale, PA_DTYPE_BF16, workspace,
+                        workspace_bytes, dev_status, stream, true, k_scale, v_scale);
 }
 
 pa_status pa_decode_attention_static(void *out, const void *query, const void *k_pool,

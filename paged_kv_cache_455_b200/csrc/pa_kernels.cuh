@@ -39,6 +39,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <type_traits>
 
@@ -109,6 +110,9 @@ struct DecodeParams {
     int head_groups;         // Hkv / hpc
     uint32_t epoch;          // mode 0: tag of this call's counter values (never 0)
     float scale_log2;
+    float out_scale;         // multiplies every output (the V scale of an FP8 cache; else 1)
+    uint64_t wait_ns;        // limit of every bounded wait (kWaitLimitNs unless a test sets it)
+    int withhold_cta;        // test hook: this CTA does not count its cut pieces in (-1: none)
     TileGeo geo;
 };
 
@@ -643,6 +647,234 @@ struct MmaMath {
 };
 
 // =====================================================================
+// Tile math over an E4M3 (FP8) cache: bf16 query and output, one byte per
+// K / V element with a per-tensor scale.  Codes convert exactly to f16
+// (cvt.f16x2.e4m3x2), and the tile products run on f16 tensor cores with
+// fp32 accumulation; the query is rounded to f16 and the softmax weights
+// are f16.  The K scale is folded into the logit scale, the V scale into
+// the output scale.
+//
+// One 16-byte unit of a row holds 16 elements.  ldmatrix reads 8 x 8
+// matrices of 16-bit elements, i.e. 8 rows x 16 bytes:
+//   S = K Q^T: lane (r, c) receives bytes 4c .. 4c+3 of row r of a unit.
+//     Bytes 4c, 4c+1 serve as the MMA's columns 2c, 2c+1 and bytes 4c+2,
+//     4c+3 as columns 2c+8, 2c+9 (a fixed permutation of the reduction
+//     index); the query fragment is built with the same permutation.
+//   O^T += V^T P^T (ldmatrix.trans): lane (r, c) receives tokens 2c, 2c+1
+//     of bytes 2r, 2r+1 of a unit; a byte permute pairs the two tokens of
+//     each byte, so MMA row r is element 2r of the unit and row r + 8 is
+//     element 2r + 1.  Accumulator acc[k][0..3] thus holds
+//     O[head 2c][16k + 2r], O[head 2c+1][16k + 2r], O[head 2c][16k + 2r + 1],
+//     O[head 2c+1][16k + 2r + 1].
+// =====================================================================
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes)
+{
+    const __half2_raw h =
+        __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(codes & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+template <int D, int G>
+struct MmaMath8 {
+    static_assert(G <= 8, "group must fit the N = 8 MMA");
+    static constexpr int KS = D / 16;   // 16-byte units per row
+
+    uint32_t qf[KS][2];
+    float acc[KS][4];
+    float m[2];
+    float l[2];
+
+    // Query fragments from the stage's query slot ([G][D] bf16).
+    __device__ __forceinline__ void begin(const uint8_t *qslot, int lane)
+    {
+        const int r = lane >> 2, c = lane & 3;
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            if (r < G) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(qslot + (r * D + 16 * k + 4 * c) * 2);
+                qf[k][0] = ptx::pack_f16x2(ptx::bf16lo_to_f32(w.x), ptx::bf16hi_to_f32(w.x));
+                qf[k][1] = ptx::pack_f16x2(ptx::bf16lo_to_f32(w.y), ptx::bf16hi_to_f32(w.y));
+            } else {
+                qf[k][0] = 0u;
+                qf[k][1] = 0u;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                acc[k][i] = 0.f;
+        }
+        m[0] = m[1] = -INFINITY;
+        l[0] = l[1] = 0.f;
+    }
+
+    __device__ __forceinline__ void tile(uint32_t ks, uint32_t vs, int hline, int n,
+                                         float scale_log2, const TileGeo &geo, int lane)
+    {
+        const int r = lane >> 2;
+        const int row = (lane & 7) + (((lane >> 3) & 1) << 3), half = lane >> 4;
+        // ---- S = K Q^T (two accumulation chains), two units per ldmatrix
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k2 = 0; k2 < KS / 2; ++k2) {
+            uint32_t a[4];
+            ptx::ldsm_x4(kv_addr16(ks, hline, row, 2 * k2 + half), a);
+            const uint32_t f0[4] = {e4m3x2_to_f16x2(a[0]), e4m3x2_to_f16x2(a[1]),
+                                    e4m3x2_to_f16x2(a[0] >> 16), e4m3x2_to_f16x2(a[1] >> 16)};
+            const uint32_t f1[4] = {e4m3x2_to_f16x2(a[2]), e4m3x2_to_f16x2(a[3]),
+                                    e4m3x2_to_f16x2(a[2] >> 16), e4m3x2_to_f16x2(a[3] >> 16)};
+            ptx::mma_f16_16816(sa, f0, qf[2 * k2][0], qf[2 * k2][1]);
+            ptx::mma_f16_16816(sb, f1, qf[2 * k2 + 1][0], qf[2 * k2 + 1][1]);
+        }
+        float s[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            s[i] = (sa[i] + sb[i]) * scale_log2;
+        if (r >= n) {
+            s[0] = -INFINITY;
+            s[1] = -INFINITY;
+        }
+        if (r + 8 >= n) {
+            s[2] = -INFINITY;
+            s[3] = -INFINITY;
+        }
+        // ---- online softmax for heads 2c, 2c+1
+        float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o));
+        }
+        const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+        const float al0 = mn0 == -INFINITY ? 1.f : ptx::ex2(m[0] - mn0);
+        const float al1 = mn1 == -INFINITY ? 1.f : ptx::ex2(m[1] - mn1);
+        const float rf0 = mn0 == -INFINITY ? 0.f : mn0;
+        const float rf1 = mn1 == -INFINITY ? 0.f : mn1;
+        m[0] = mn0;
+        m[1] = mn1;
+        const uint32_t p01 = ptx::pack_f16x2(ptx::ex2(s[0] - rf0), ptx::ex2(s[1] - rf1));
+        const uint32_t p23 = ptx::pack_f16x2(ptx::ex2(s[2] - rf0), ptx::ex2(s[3] - rf1));
+        // the sum uses the same rounded weights as the MMA
+        l[0] = l[0] * al0 + ptx::f16lo_to_f32(p01) + ptx::f16lo_to_f32(p23);
+        l[1] = l[1] * al1 + ptx::f16hi_to_f32(p01) + ptx::f16hi_to_f32(p23);
+        if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+            for (int k = 0; k < KS; ++k) {
+                acc[k][0] *= al0;
+                acc[k][1] *= al1;
+                acc[k][2] *= al0;
+                acc[k][3] *= al1;
+            }
+        }
+        const uint32_t b0 = ptx::movmatrix_trans(p01);
+        const uint32_t b1 = ptx::movmatrix_trans(p23);
+        // ---- O^T += V^T P^T, two units per ldmatrix
+#pragma unroll
+        for (int k2 = 0; k2 < KS / 2; ++k2) {
+            uint32_t a[4];
+            ptx::ldsm_x4_trans(kv_addr16(vs, hline, row, 2 * k2 + half), a);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t lo = ptx::prmt(a[2 * u], 0u, 0x3120u);       // tokens 0-7
+                const uint32_t hi = ptx::prmt(a[2 * u + 1], 0u, 0x3120u);   // tokens 8-15
+                const uint32_t f[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(lo >> 16),
+                                       e4m3x2_to_f16x2(hi), e4m3x2_to_f16x2(hi >> 16)};
+                ptx::mma_f16_16816(acc[2 * k2 + u], f, b0, b1);
+            }
+        }
+    }
+
+    __device__ __forceinline__ void finish()
+    {
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            l[0] += __shfl_xor_sync(kFull, l[0], o);
+            l[1] += __shfl_xor_sync(kFull, l[1], o);
+        }
+    }
+
+    // Published piece layout: as MmaMath (one float4 acc[k][0..3] per unit
+    // k * 8 * CU + r * CU + c), with this layout's element coordinates.
+    static constexpr int CU = (G + 1) / 2;
+    static constexpr int kUnits = KS * 8 * CU;
+
+    __device__ __forceinline__ void publish(float *ps, int lane) const
+    {
+        const int r = lane >> 2, c = lane & 3;
+        if (c < CU) {
+            float4 *p4 = reinterpret_cast<float4 *>(ps) + r * CU + c;
+#pragma unroll
+            for (int k = 0; k < KS; ++k)
+                p4[k * 8 * CU] = make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
+        }
+    }
+
+    __device__ __forceinline__ void publish_stats(float *st, int lane) const
+    {
+        const int r = lane >> 2, c = lane & 3;
+        if (r == 0 && 2 * c < G) {
+            st[2 * c] = m[0];
+            st[G + 2 * c] = l[0];
+            if (2 * c + 1 < G) {
+                st[2 * c + 1] = m[1];
+                st[G + 2 * c + 1] = l[1];
+            }
+        }
+    }
+
+    __device__ __forceinline__ static void unit_coords(int u, int j, int &g, int &d)
+    {
+        const int k = u / (8 * CU), rem = u - k * 8 * CU;
+        const int r = rem / CU, c = rem - r * CU;
+        g = 2 * c + (j & 1);
+        d = 16 * k + 2 * r + (j >> 1);
+    }
+
+    // Writes out_scale * acc / sum (zeros where `zero` or the sum is 0) to
+    // o[head * D + d] as bf16: lane (r, c) holds two consecutive d of heads
+    // 2c and 2c + 1 and stores each pair as one 4-byte word.
+    __device__ __forceinline__ void store_final(__nv_bfloat16 *o, bool zero, float out_scale,
+                                                int lane) const
+    {
+        const int r = lane >> 2, c = lane & 3;
+        const float i0 = (zero || !(l[0] > 0.f)) ? 0.f : out_scale * __frcp_rn(l[0]);
+        const float i1 = (zero || !(l[1] > 0.f)) ? 0.f : out_scale * __frcp_rn(l[1]);
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            if (2 * c < G)
+                *reinterpret_cast<uint32_t *>(o + (2 * c) * D + 16 * k + 2 * r) =
+                    ptx::pack_bf16x2(acc[k][0] * i0, acc[k][2] * i0);
+            if (2 * c + 1 < G)
+                *reinterpret_cast<uint32_t *>(o + (2 * c + 1) * D + 16 * k + 2 * r) =
+                    ptx::pack_bf16x2(acc[k][1] * i1, acc[k][3] * i1);
+        }
+    }
+
+    template <typename F, typename FM>
+    __device__ __forceinline__ void for_each(int lane, F f, FM fm) const
+    {
+        const int r = lane >> 2, c = lane & 3;
+        const int h0 = 2 * c, h1 = 2 * c + 1;
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            const int d0 = 16 * k + 2 * r;
+            if (h0 < G) {
+                f(h0, d0, acc[k][0], l[0]);
+                f(h0, d0 + 1, acc[k][2], l[0]);
+            }
+            if (h1 < G) {
+                f(h1, d0, acc[k][1], l[1]);
+                f(h1, d0 + 1, acc[k][3], l[1]);
+            }
+        }
+        if (r == 0) {
+            if (h0 < G)
+                fm(h0, m[0], l[0]);
+            if (h1 < G)
+                fm(h1, m[1], l[1]);
+        }
+    }
+};
+
+// =====================================================================
 // Tile math, CUDA cores
 // =====================================================================
 template <typename T, int D, int G, bool TR16>
@@ -928,30 +1160,44 @@ __host__ __device__ constexpr int64_t merge_scratch_bytes(int G, int D, int64_t 
     return 4 * ((int64_t)piece_stats_off(D, G) + 4 * np * stats_units(G) + np * G + 2 * G + 4);
 }
 
-// Counts one more arrival at a cut segment's counter for this call.  The
-// high half of the counter holds a call's epoch: CTA x tags its own counters
-// (epoch, count 0) when it starts, before any piece is done.  An arrival
-// adds 1; if its add landed on a word that still carried an older epoch, the
-// owner's tag store (still to come) overwrites it, so the arrival waits
-// (bounded) for the tag and adds again.  The acquire-release add publishes
-// the caller's piece (stored before it) and, for the last arrival, makes
-// every earlier arrival's piece visible.  Returns the arrivals so far
-// including this one, or 0 if the tag never came.
+// Counts one more arrival at a cut segment's counter for this call and
+// returns the arrivals so far including this one (0 if the count could not
+// be taken, which cannot happen while fewer than 2^20 pieces race).
+//
+// The high half of a counter word holds the epoch of the call that counts
+// in it; a word with another epoch counts as zero.  Nothing needs to be
+// initialised and no arrival waits for another CTA:
+//   - the CTA owning the counter raises it to (epoch, 0) with an atomic
+//     maximum when it starts, which leaves a count of this call untouched
+//     (epochs of one process increase);
+//   - an arrival adds 1 with an acquire-release atomic add; if the word it
+//     added to carried another epoch, it restarts the count as (epoch, 1)
+//     with a compare-and-swap on the value its add left.  A restart erases
+//     the adds other arrivals made to the stale word: each of them sees its
+//     own swap fail on a word of this epoch and adds again.
+// Every arrival is therefore counted once in this epoch.  The add (or the
+// swap) releases the caller's piece, stored before it, and the last arrival
+// acquires every earlier one.
 __device__ __forceinline__ int segment_arrive(unsigned long long *c, uint32_t epoch)
 {
     unsigned long long old = ptx::atom_add_acq_rel_gpu(c, 1ull);
     if ((uint32_t)(old >> 32) == epoch)
         return (int)(old & 0xffffffffu) + 1;
-    const uint64_t t0 = ptx::globaltimer_ns();
-    for (uint32_t i = 0; i < (1u << 26); ++i) {
-        if ((uint32_t)(ptx::ld_relaxed_gpu_u64(c) >> 32) == epoch) {
+    const unsigned long long mine = ((unsigned long long)epoch << 32) | 1ull;
+    unsigned long long cur = old + 1;
+    for (uint32_t i = 0; i < (1u << 20); ++i) {
+        const unsigned long long prev = ptx::atom_cas_acq_rel_gpu(c, cur, mine);
+        if (prev == cur)
+            return 1;
+        if ((uint32_t)(prev >> 32) == epoch) {
+            // another arrival restarted the count, erasing this one's add
             old = ptx::atom_add_acq_rel_gpu(c, 1ull);
             if ((uint32_t)(old >> 32) == epoch)
                 return (int)(old & 0xffffffffu) + 1;
+            cur = old + 1;
+        } else {
+            cur = prev;   // more adds to the stale word since: swap that value
         }
-        __nanosleep(64);
-        if ((i & 15u) == 0 && ptx::globaltimer_ns() - t0 > kWaitLimitNs)
-            break;
     }
     return 0;
 }
@@ -1003,7 +1249,7 @@ __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, 
                     break;
                 }
                 __nanosleep(64);
-                if ((i & 15u) == 0 && ptx::globaltimer_ns() - t0 > kWaitLimitNs)
+                if ((i & 15u) == 0 && ptx::globaltimer_ns() - t0 > p.wait_ns)
                     break;
             }
             if (!done)
@@ -1081,7 +1327,8 @@ __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, 
     for (int f = lane; f < np * G; f += 32) {
         const int i = f / G, g = f - i * G;
         const float mi = st[i * 4 * SU + g], M = tot[g], L = tot[G + g];
-        w[f] = (mi == -INFINITY || !(L > 0.f)) ? 0.f : ptx::ex2(mi - M) / L;
+        // out_scale (1 unless the cache is FP8) multiplies the weights exactly
+        w[f] = (mi == -INFINITY || !(L > 0.f)) ? 0.f : ptx::ex2(mi - M) / L * p.out_scale;
     }
     __syncwarp();
 
@@ -1158,10 +1405,13 @@ __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, 
 // in, and every CTA of the persistent grid is resident, so every wait ends;
 // each is bounded all the same.
 //
-// Nothing touches global memory before griddepcontrol.wait: the kernel is
-// launched as a programmatic dependent of the kernel before it on the stream.
+// The kernel is launched as a programmatic dependent of the kernel before it
+// on the stream.  Before griddepcontrol.wait it reads only the context
+// lengths and the block tables (the kernel ahead must not write them); the
+// query, the pools, the outputs and the workspace come after the wait.  It
+// lets the kernel after it start early in the same way.
 // =====================================================================
-template <typename T, int D, int G, bool MMA, bool TR16>
+template <typename T, int D, int G, bool MMA, bool TR16, bool KV8>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p)
@@ -1194,12 +1444,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     ptx::fence_mbar_init();
-    ptx::grid_wait_prerequisites();
+    // The lengths and block tables are read before the kernel ahead on the
+    // stream has completed (see the launch): the work decomposition and the
+    // first block-table batches overlap its tail.
     const int total = chunk_prefix(p, cbase);   // contains __syncthreads
     // C <= T CTAs take part, so that every participating range is non-empty
     const int C = min(total_ctas, max(total, 1));
     const int R0 = range_begin(blockIdx.x, C, total, p, cbase, lane);
     const int R1 = range_begin(blockIdx.x + 1, C, total, p, cbase, lane);
+    // the next kernel on the stream may start its own set-up on SMs this
+    // grid leaves; it waits for this grid to complete before using its results
+    if (threadIdx.x == 0)
+        ptx::grid_launch_dependents();
 
     if (warp == hpc) {
         // =================================================== producer warp
@@ -1216,6 +1472,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         TileDesc bat0, bat1;
         fill_batch(bat0, win, R0, R1, p, cbase, lane);
         fill_batch(bat1, win, R0 + 32, R1, p, cbase, lane);
+        // the pools and the query may be written by the kernel ahead
+        ptx::grid_wait_prerequisites();
         int filled = 2;
         int issued = R0;
         for (; issued < R1; ++issued) {
@@ -1224,7 +1482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = k % spw;
             const uint32_t bar = full0 + 8u * s;
             if (k >= spw && !ptx::mbar_wait_bounded(empty0 + 8u * s,
-                                                    (uint32_t)(((k / spw) - 1) & 1), kWaitLimitNs)) {
+                                                    (uint32_t)(((k / spw) - 1) & 1), p.wait_ns)) {
                 if (lane == 0)
                     report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
                 break;
@@ -1290,7 +1548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = max(R0, issued - spw); i < issued; ++i) {
                 const int k = i - R0;
                 ptx::mbar_wait_bounded(full0 + 8u * (k % spw), (uint32_t)((k / spw) & 1),
-                                       kWaitLimitNs);
+                                       p.wait_ns);
             }
         }
         return;
@@ -1300,6 +1558,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hl = warp;                        // head within the group
     const int hline = hl * geo.head_lines;      // its first 128-byte line in a box
     float *scores = scores_all + hl * kTile * G;
+    // outputs and the workspace may still be in use by the kernel ahead
+    ptx::grid_wait_prerequisites();
 
     // Sequences without tiles (length 0 or invalid) get a zero output.
     for (int b = blockIdx.x; b < p.num_seqs; b += total_ctas) {
@@ -1327,8 +1587,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
-    using Math =
-        typename std::conditional<MMA, MmaMath<D, G, TR16>, SimtMath<T, D, G, TR16>>::type;
+    static_assert(!KV8 || (MMA && TR16), "an FP8 cache uses the tensor-core math, blocks >= 16");
+    using Math = typename std::conditional<
+        KV8, MmaMath8<D, G>,
+        typename std::conditional<MMA, MmaMath<D, G, TR16>, SimtMath<T, D, G, TR16>>::type>::type;
     Math math;
     int segS = 0;          // global index of the current segment's first tile
     bool seg_bad = false;
@@ -1338,15 +1600,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     int laterS = -1, laterN = 0, laterB = 0, laterHG = 0;
     int firstS = -1, firstN = 0, firstB = 0, firstHG = 0;
 
-    // this CTA's arrival counters start the call at (epoch, 0)
+    // this CTA's arrival counters start the call at (epoch, 0) unless an
+    // arrival has already counted in them (see segment_arrive)
     if (p.mode == 0 && lane == 0)
-        ptx::st_relaxed_gpu_u64(p.counters + (int64_t)blockIdx.x * hpc + hl,
-                                (unsigned long long)p.epoch << 32);
+        ptx::red_max_relaxed_gpu_u64(p.counters + (int64_t)blockIdx.x * hpc + hl,
+                                     (unsigned long long)p.epoch << 32);
 
     for (int i = R0; i < R1; ++i) {
         const int k = i - R0;
         const int s = k % spw;
-        if (!ptx::mbar_wait_bounded(full0 + 8u * s, (uint32_t)((k / spw) & 1), kWaitLimitNs)) {
+        if (!ptx::mbar_wait_bounded(full0 + 8u * s, (uint32_t)((k / spw) & 1), p.wait_ns)) {
             if (lane == 0)
                 report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
             timed_out = true;
@@ -1371,7 +1634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (d.n < kTile) {
                 // rows past the sequence end hold whatever the pool has there:
                 // zero them in this head's V (their weight is 0, but 0 * NaN is NaN)
-                constexpr int NCH = D * (int)sizeof(T) / 128;
+                constexpr int NCH = D * (KV8 ? 1 : (int)sizeof(T)) / 128;
                 const int lines = (kTile - d.n) * NCH;
                 for (int idx = lane; idx < lines * 8; idx += 32) {
                     const int line = idx >> 3;
@@ -1415,6 +1678,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 const int x0 = cta_of(segS, C, total);
                 int arrived = 0;
+                if ((int)blockIdx.x == p.withhold_cta) {
+                    // test hook: the piece is never counted in, so the waits
+                    // of a cooperative merge run out; this CTA still takes
+                    // its share of such a merge
+                    const int npw = cta_of(segS + d.ns - 1, C, total) - x0 + 1;
+                    if (npw > kLastMergesPieces) {
+                        if (first) {
+                            firstS = segS; firstN = d.ns; firstB = d.b; firstHG = d.hg;
+                        } else {
+                            laterS = segS; laterN = d.ns; laterB = d.b; laterHG = d.hg;
+                        }
+                    }
+                    continue;
+                }
                 if (lane == 0)
                     arrived = segment_arrive(p.counters + (int64_t)x0 * hpc + hl, p.epoch);
                 arrived = __shfl_sync(kFull, arrived, 0);
@@ -1444,7 +1721,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 report(p.dev_status, PA_DEV_BAD_BLOCK);
             const bool single = num_parts(d.ctx, p.partition_size) == 1;
             if (single && !p.public_partials) {
-                math.store_final(static_cast<T *>(p.out) + bh0 * D, seg_bad, lane);
+                if constexpr (KV8)
+                    math.store_final(static_cast<T *>(p.out) + bh0 * D, seg_bad, p.out_scale, lane);
+                else
+                    math.store_final(static_cast<T *>(p.out) + bh0 * D, seg_bad, lane);
                 continue;
             }
             math.for_each(
@@ -1454,7 +1734,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (p.public_partials)
                         p.tmp_out[((bh0 + hh) * p.max_parts + d.part) * D + e] = res;
                     if (single)
-                        store_out<T>(static_cast<T *>(p.out) + (bh0 + hh) * D + e, res);
+                        store_out<T>(static_cast<T *>(p.out) + (bh0 + hh) * D + e,
+                                     res * p.out_scale);
                 },
                 [&](int hh, float mm, float ll) {
                     if (p.public_partials) {

@@ -15,6 +15,7 @@ struct DecodeLaunch {
     int head_dim;
     int group;
     bool tr16;          // block size >= 16: one 16-row box per tile
+    bool kv8;           // the pools hold E4M3 codes (query and output bf16)
     int smem_bytes;
     cudaStream_t stream;
 };
@@ -62,10 +63,10 @@ inline pa_status grid_capacity(const void *fn, int threads, int smem_bytes, int 
 
 // With launch == false, *grid receives the capacity; otherwise the kernel is
 // launched with min(*grid, capacity) CTAs and *grid receives that count.
-template <typename T, int D, int G, bool MMA, bool TR16>
+template <typename T, int D, int G, bool MMA, bool TR16, bool KV8 = false>
 pa_status decode_one(DecodeLaunch &L, int *grid, bool launch)
 {
-    auto fn = &decode_kernel<T, D, G, MMA, TR16>;
+    auto fn = &decode_kernel<T, D, G, MMA, TR16, KV8>;
     const int threads = 32 * (L.p.geo.hpc + 1);
     int cap = 0;
     pa_status st = grid_capacity(reinterpret_cast<const void *>(fn), threads, L.smem_bytes, &cap);
@@ -125,8 +126,34 @@ pa_status decode_dispatch(DecodeLaunch &L, int *grid, bool launch)
     }
 }
 
+// FP8 (E4M3) cache: bf16 query and output, blocks of 16 or 32, d 128 or 256.
+template <int D>
+pa_status decode_fp8_g(DecodeLaunch &L, int *grid, bool launch)
+{
+    using B = __nv_bfloat16;
+    switch (L.group) {
+    case 1: return decode_one<B, D, 1, true, true, true>(L, grid, launch);
+    case 2: return decode_one<B, D, 2, true, true, true>(L, grid, launch);
+    case 4: return decode_one<B, D, 4, true, true, true>(L, grid, launch);
+    case 8: return decode_one<B, D, 8, true, true, true>(L, grid, launch);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+inline pa_status decode_fp8_dispatch(DecodeLaunch &L, int *grid, bool launch)
+{
+    if (!L.tr16)
+        return PA_ERR_UNSUPPORTED;
+    switch (L.head_dim) {
+    case 128: return decode_fp8_g<128>(L, grid, launch);
+    case 256: return decode_fp8_g<256>(L, grid, launch);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
 // Entry points of the instantiation units.
 pa_status decode_f32(DecodeLaunch &L, int *grid, bool launch);
+pa_status decode_fp8(DecodeLaunch &L, int *grid, bool launch);
 pa_status decode_bf16_mma(DecodeLaunch &L, int *grid, bool launch);
 pa_status decode_bf16_simt(DecodeLaunch &L, int *grid, bool launch);
 

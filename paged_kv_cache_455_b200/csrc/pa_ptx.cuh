@@ -101,6 +101,26 @@ __device__ __forceinline__ unsigned long long atom_add_acq_rel_gpu(unsigned long
     return old;
 }
 
+// Atomic compare-and-swap with acquire-release semantics at gpu scope;
+// returns the old value (the swap happened iff it equals `expected`).
+__device__ __forceinline__ unsigned long long atom_cas_acq_rel_gpu(unsigned long long *p,
+                                                                   unsigned long long expected,
+                                                                   unsigned long long v)
+{
+    unsigned long long old;
+    asm volatile("atom.acq_rel.gpu.global.cas.b64 %0, [%1], %2, %3;"
+                 : "=l"(old)
+                 : "l"(p), "l"(expected), "l"(v)
+                 : "memory");
+    return old;
+}
+
+// Atomic maximum without a result (relaxed, gpu scope).
+__device__ __forceinline__ void red_max_relaxed_gpu_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t done;
@@ -289,6 +309,50 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     uint32_t d;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// D += A * B, A 16x16 f16 (row), B 16x8 f16 (col), D 16x8 fp32.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Packs two fp32 values into f16x2 (round to nearest even), `lo` in the low
+// half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+__device__ __forceinline__ float f16lo_to_f32(uint32_t x)
+{
+    float f;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, lo;\n\t}"
+        : "=f"(f) : "r"(x));
+    return f;
+}
+
+__device__ __forceinline__ float f16hi_to_f32(uint32_t x)
+{
+    float f;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, hi;\n\t}"
+        : "=f"(f) : "r"(x));
+    return f;
+}
+
+// Byte permute: byte i of the result is byte ((sel >> 4 i) & 7) of {b, a}.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
     return d;
 }
 

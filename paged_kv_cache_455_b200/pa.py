@@ -30,7 +30,7 @@ _SZ = ctypes.c_size_t
 _F = ctypes.c_float
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE = range(5)
-PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
+PA_DTYPE_F32, PA_DTYPE_BF16, PA_DTYPE_FP8_E4M3 = 0, 1, 2
 PA_DEV_BAD_SLOT, PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_WAIT_TIMEOUT = 1, 2, 4, 8
 
 # Every symbol include/pa.h declares, with its C signature.
@@ -50,8 +50,14 @@ SIGNATURES = {
     "pa_swap_blocks": (_I, [_P, _P, _I64, _P, _P, _I64, _P, _I, _I, _I, _I, _I, _P, _P]),
     "pa_prefill_attention": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
                                   _I, _I64, _F, _I, _P, _P]),
+    "pa_reshape_and_cache_fp8": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _F, _F, _P, _P]),
+    "pa_decode_attention_fp8": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F,
+                                     _F, _F, _P, _SZ, _P, _P]),
     "pa_status_string": (ctypes.c_char_p, [_I]),
     "pa_launch_count": (ctypes.c_ulonglong, []),
+    # include/pa_testing.h
+    "pa_testing_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
+    "pa_testing_withhold_pieces": (None, [_I]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _fn = getattr(lib, _name)
@@ -70,11 +76,16 @@ def _check(status: int, where: str) -> None:
         raise PaError(status, where)
 
 
+FP8_POOL_DTYPES = (torch.uint8, torch.float8_e4m3fn)
+
+
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return PA_DTYPE_F32
     if t.dtype == torch.bfloat16:
         return PA_DTYPE_BF16
+    if t.dtype in FP8_POOL_DTYPES:
+        return PA_DTYPE_FP8_E4M3
     raise ValueError(f"unsupported dtype {t.dtype}")
 
 
@@ -96,6 +107,16 @@ def _stream(stream) -> int:
 
 def launch_count() -> int:
     return int(lib.pa_launch_count())
+
+
+def testing_set_wait_limit_ns(ns: int) -> None:
+    """Test hook: limit of the decode kernels' bounded waits (0: the default)."""
+    lib.pa_testing_set_wait_limit_ns(int(ns))
+
+
+def testing_withhold_pieces(cta: int) -> None:
+    """Test hook: CTA `cta` of later decode launches withholds its pieces (-1: off)."""
+    lib.pa_testing_withhold_pieces(int(cta))
 
 
 def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int,
@@ -129,6 +150,59 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_pool: torch.T
     _check(lib.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_pool), _ptr(v_pool),
                                     _ptr(slot_mapping), T, hkv, d, bs, nb, _dtype_code(key),
                                     _ptr(dev_status), _stream(stream)), "pa_reshape_and_cache")
+
+
+def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, k_pool: torch.Tensor,
+                             v_pool: torch.Tensor, slot_mapping: torch.Tensor, k_scale: float,
+                             v_scale: float, dev_status: Optional[torch.Tensor] = None,
+                             stream=None) -> None:
+    """key/value [T, Hkv, d] bf16; pools [nb, bs, Hkv, d] of E4M3 codes (uint8 or
+    float8_e4m3fn); slot_mapping [T] int64; per-tensor scales."""
+    _cuda(key, value, k_pool, v_pool, slot_mapping, dev_status)
+    T, hkv, d = key.shape
+    nb, bs = k_pool.shape[:2]
+    if value.shape != key.shape or v_pool.shape != k_pool.shape or k_pool.shape[2:] != (hkv, d):
+        raise ValueError("shape mismatch")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (T,):
+        raise ValueError("slot_mapping must be int64 [T]")
+    if key.dtype != torch.bfloat16 or value.dtype != torch.bfloat16:
+        raise ValueError("key and value must be bf16")
+    if k_pool.dtype not in FP8_POOL_DTYPES or v_pool.dtype not in FP8_POOL_DTYPES:
+        raise ValueError("pools must hold E4M3 codes (uint8 or float8_e4m3fn)")
+    _check(lib.pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), _ptr(k_pool), _ptr(v_pool),
+                                        _ptr(slot_mapping), T, hkv, d, bs, nb, float(k_scale),
+                                        float(v_scale), _ptr(dev_status), _stream(stream)),
+           "pa_reshape_and_cache_fp8")
+
+
+def pa_decode_attention_fp8(out: torch.Tensor, query: torch.Tensor, k_pool: torch.Tensor,
+                            v_pool: torch.Tensor, block_tables: torch.Tensor,
+                            context_lens: torch.Tensor, max_context_len: int, scale: float,
+                            k_scale: float, v_scale: float,
+                            workspace: Optional[torch.Tensor] = None,
+                            dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out, query [B, Hq, d] bf16; pools [nb, bs, Hkv, d] of E4M3 codes;
+    block_tables [B, max_blocks] int32; context_lens [B] int32."""
+    _cuda(out, query, k_pool, v_pool, block_tables, context_lens, workspace, dev_status)
+    B, hq, d = query.shape
+    nb, bs, hkv, d2 = k_pool.shape
+    if out.shape != query.shape or v_pool.shape != k_pool.shape or d2 != d:
+        raise ValueError("shape mismatch")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("block_tables must be int32 [B, max_blocks]")
+    if context_lens.dtype != torch.int32 or context_lens.shape != (B,):
+        raise ValueError("context_lens must be int32 [B]")
+    if query.dtype != torch.bfloat16 or out.dtype != torch.bfloat16:
+        raise ValueError("query and out must be bf16")
+    if k_pool.dtype not in FP8_POOL_DTYPES or v_pool.dtype not in FP8_POOL_DTYPES:
+        raise ValueError("pools must hold E4M3 codes (uint8 or float8_e4m3fn)")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_attention_fp8(_ptr(out), _ptr(query), _ptr(k_pool), _ptr(v_pool),
+                                       _ptr(block_tables), block_tables.shape[1],
+                                       _ptr(context_lens), B, int(max_context_len), hq, hkv, d,
+                                       bs, nb, float(scale), float(k_scale), float(v_scale),
+                                       _ptr(workspace), ws_bytes, _ptr(dev_status),
+                                       _stream(stream)), "pa_decode_attention_fp8")
 
 
 def pa_copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, block_mapping: torch.Tensor,
@@ -288,10 +362,11 @@ def pa_splitk_reduce(out: torch.Tensor, tmp_out: torch.Tensor, max_logits: torch
 
 __all__ = [
     "lib", "LIB_PATH", "SIGNATURES", "PaError", "launch_count",
-    "pa_reshape_and_cache", "pa_copy_blocks", "pa_swap_blocks", "pa_prefill_attention", "pa_decode_attention", "pa_decode_workspace_bytes",
+    "pa_reshape_and_cache", "pa_reshape_and_cache_fp8", "pa_decode_attention_fp8",
+    "testing_set_wait_limit_ns", "testing_withhold_pieces", "pa_copy_blocks", "pa_swap_blocks", "pa_prefill_attention", "pa_decode_attention", "pa_decode_workspace_bytes",
     "pa_decode_attention_static", "PA_STATIC_SCRATCH_BYTES",
     "pa_num_partitions", "pa_splitk_workspace_bytes", "pa_decode_splitk", "pa_splitk_reduce",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA", "PA_ERR_WORKSPACE",
-    "PA_DTYPE_F32", "PA_DTYPE_BF16",
+    "PA_DTYPE_F32", "PA_DTYPE_BF16", "PA_DTYPE_FP8_E4M3",
     "PA_DEV_BAD_SLOT", "PA_DEV_BAD_BLOCK", "PA_DEV_BAD_CONTEXT", "PA_DEV_WAIT_TIMEOUT",
 ]

@@ -329,6 +329,50 @@ def make_layers(layout: BatchLayout, device, layers: Optional[int] = None,
     return out
 
 
+# FP8 (E4M3) cache contents: the per-tensor scales of the synthetic
+# workloads put 8 standard deviations at the format's largest value, 448.
+FP8_SCALE = 8.0 / 448.0
+FP8_NAN = 0x7F
+
+
+def fp8_codes(x: torch.Tensor, scale: float) -> torch.Tensor:
+    """E4M3 codes (uint8) of the draws x / scale, clamped to +-448, through
+    torch's own float8_e4m3fn conversion (input generation only)."""
+    y = (x.float() / scale).clamp_(-448.0, 448.0)
+    return y.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def make_layers_fp8(layout: BatchLayout, device, layers: Optional[int] = None,
+                    scale: float = FP8_SCALE, chunk_rows: int = 1 << 16) -> List[LayerTensors]:
+    """Like ``make_layers`` but with E4M3 pools (uint8 codes): pool rows in
+    ``valid_slots`` are codes of N(0,1) draws / ``scale``, every other row is
+    the NaN code; query and the new token's key / value are bf16 N(0,1)."""
+    cfg = layout.config
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(shard_seed(cfg, int(layout.notes.get("shard", 0))) + 104729)
+    nl = cfg.layers if layers is None else layers
+    slots = torch.from_numpy(valid_slots(layout)).to(device)
+    B, hq, hkv, d = cfg.num_seqs, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim
+    nb, bs = layout.num_blocks, cfg.block_size
+    out = []
+    for _ in range(nl):
+        q = _randn((B, hq, d), gen, device, torch.bfloat16)
+        k = _randn((B, hkv, d), gen, device, torch.bfloat16)
+        v = _randn((B, hkv, d), gen, device, torch.bfloat16)
+        pools = []
+        for _kv in range(2):
+            pool = torch.full((nb, bs, hkv, d), FP8_NAN, device=device, dtype=torch.uint8)
+            rows = pool.view(nb * bs, hkv, d)
+            for s0 in range(0, slots.numel(), chunk_rows):
+                idx = slots[s0:s0 + chunk_rows]
+                rows[idx] = fp8_codes(torch.randn((idx.numel(), hkv, d), generator=gen,
+                                                  device=device), scale)
+            pools.append(pool)
+        out.append(LayerTensors(q, k, v, pools[0], pools[1]))
+    return out
+
+
 def device_metadata(layout: BatchLayout, device):
     """(block_tables, context_lens, slot_mapping) as tensors on ``device``."""
     return (torch.from_numpy(layout.block_tables).to(device),
@@ -341,8 +385,11 @@ def device_metadata(layout: BatchLayout, device):
 # --------------------------------------------------------------------------
 
 def to_numpy_elems(t: torch.Tensor) -> np.ndarray:
-    """fp32 -> numpy float32; bf16 -> numpy uint16 holding the raw bits."""
+    """fp32 -> numpy float32; bf16 -> numpy uint16 holding the raw bits;
+    E4M3 codes (uint8) -> numpy uint8."""
     t = t.detach().contiguous().cpu()
+    if t.dtype == torch.uint8:
+        return t.numpy()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
     if t.dtype == torch.float32:

@@ -1,5 +1,6 @@
-"""libpa.so loads on a CPU-only machine, exports every symbol include/pa.h
-declares, and rejects bad arguments on the host without touching a device."""
+"""libpa.so loads on a CPU-only machine, exports every symbol the headers in
+include/ declare, and rejects bad arguments on the host without touching a
+device."""
 import ctypes
 import os
 import re
@@ -18,16 +19,20 @@ def pa():
 
 
 def _declared_functions():
-    text = open(os.path.join(ROOT, "include", "pa.h")).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_every_declared_symbol_is_exported(pa):
     names = _declared_functions()
     assert len(names) >= 9
     for n in names:
-        assert hasattr(pa.lib, n), f"{n} declared in pa.h but not exported"
+        assert hasattr(pa.lib, n), f"{n} declared in include/ but not exported"
         assert n in pa.SIGNATURES, f"{n} has no binding"
 
 
@@ -201,3 +206,38 @@ def test_binding_rejects_cpu_tensors(pa):
         pa.pa_decode_attention(x, x, torch.zeros(16, 4, 2, 64), torch.zeros(16, 4, 2, 64),
                                torch.zeros(3, 2, dtype=torch.int32),
                                torch.zeros(3, dtype=torch.int32), 8, 0.125)
+
+
+def test_fp8_host_validation(pa):
+    L = pa.lib
+
+    def cache(**kw):
+        a = dict(key=A, value=A, kp=A, vp=A, slots=A, T=3, hkv=2, d=128, bs=16, nb=16, ks=0.02,
+                 vs=0.02)
+        a.update(kw)
+        return L.pa_reshape_and_cache_fp8(a["key"], a["value"], a["kp"], a["vp"], a["slots"],
+                                          a["T"], a["hkv"], a["d"], a["bs"], a["nb"], a["ks"],
+                                          a["vs"], None, None)
+
+    def attn(**kw):
+        a = dict(out=A, query=A, kp=A, vp=A, tab=A, maxb=4, lens=A, B=3, max_ctx=64, hq=8, hkv=2,
+                 d=128, bs=16, nb=16, scale=0.1, ks=0.02, vs=0.02)
+        a.update(kw)
+        return L.pa_decode_attention_fp8(a["out"], a["query"], a["kp"], a["vp"], a["tab"],
+                                         a["maxb"], a["lens"], a["B"], a["max_ctx"], a["hq"],
+                                         a["hkv"], a["d"], a["bs"], a["nb"], a["scale"], a["ks"],
+                                         a["vs"], None, 0, None, None)
+    assert cache(key=None) == 1
+    assert cache(ks=0.0) == 1 and cache(vs=-1.0) == 1 and cache(ks=float("inf")) == 1
+    assert cache(d=64) == 2 and cache(bs=8) == 2
+    assert cache(kp=M) == 1
+    assert cache(T=0, key=None) == 0
+    assert attn(out=None) == 1
+    assert attn(ks=float("nan")) == 1 and attn(vs=0.0) == 1
+    assert attn(d=64) == 2 and attn(bs=4) == 2
+    assert attn(hq=6, hkv=4) == 1
+    assert attn(max_ctx=65) == 1
+    assert attn(B=0, out=None, query=None) == 0
+    # copies of E4M3 pools are accepted; an unknown element type is not
+    assert L.pa_copy_blocks(A, A, A, 1, 16, 16, 2, 128, 2, None, None) != 2
+    assert L.pa_copy_blocks(A, A, A, 1, 16, 16, 2, 128, 3, None, None) == 2

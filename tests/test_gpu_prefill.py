@@ -37,6 +37,15 @@ def _case(seed, ctxs, chunks, hq, hkv, d, bs, spare=5):
     g.manual_seed(seed)
     k_pool = torch.randn(nb, bs, hkv, d, generator=g, device=DEV).to(torch.bfloat16)
     v_pool = torch.randn(nb, bs, hkv, d, generator=g, device=DEV).to(torch.bfloat16)
+    # NaN in every slot past each context and in every block no sequence owns,
+    # so that a masking slip shows as a non-finite output
+    valid = np.zeros((nb, bs), bool)
+    for b, c in enumerate(ctxs):
+        t = np.arange(c)
+        valid[tables[b, t // bs], t % bs] = True
+    invalid = torch.from_numpy(~valid).to(DEV)
+    k_pool[invalid] = float("nan")
+    v_pool[invalid] = float("nan")
     cu = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
     q = torch.randn(int(cu[-1]), hq, d, generator=g, device=DEV).to(torch.bfloat16)
     return q, k_pool, v_pool, tables, np.array(ctxs, np.int32), cu
@@ -71,6 +80,23 @@ def test_random_chunks_match_oracle(pa, d, hq, hkv, bs):
     assert status == 0
     ref = _oracle(q, kp, vp, tab, lens, cu, scale)
     assert np.abs(out.double().cpu().numpy() - ref).max() <= TOL
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_every_tail_length_up_to_80(pa, bs):
+    """Contexts of 1 .. 80 tokens (every position of the last block, and
+    chunks that are whole prompts or end part-way into a 64-token tile) on
+    the tensor-core path (blocks of 16 and 32)."""
+    ctxs = list(range(1, 81))
+    chunks = [c if c % 3 else max(1, c // 2) for c in ctxs]
+    q, kp, vp, tab, lens, cu = _case(100 + bs, ctxs, chunks, 8, 2, 128, bs)
+    scale = 128 ** -0.5
+    out, status = _run(pa, q, kp, vp, tab, lens, cu, scale)
+    assert status == 0
+    ref = _oracle(q, kp, vp, tab, lens, cu, scale)
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= TOL
 
 
 def test_512_token_chunk_after_a_long_prefix(pa):

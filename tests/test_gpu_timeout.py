@@ -1,0 +1,80 @@
+"""The decode kernel's bounded waits, made to run out on purpose.
+
+Every wait inside the decode kernel is bounded; one that runs out sets
+PA_DEV_WAIT_TIMEOUT and the kernel returns normally, so the CUDA context stays
+usable.  The test hooks of include/pa_testing.h shorten the limit to 2 ms and
+make one CTA withhold its pieces of a sequence split over many CTAs: the
+merge of that sequence then waits for a count that never completes.  No
+fault, trap or hang is involved.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from paged_kv_cache_455_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+TOL = 2e-2
+
+
+def _case(seed, lens, hq=16, hkv=4, d=256, bs=16):
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens, np.int32)
+    need = -(-lens // bs)
+    nb = int(need.sum()) + 8
+    perm = rng.permutation(nb)
+    tables = np.full((len(lens), int(need.max())), -1, np.int32)
+    pos = 0
+    for b in range(len(lens)):
+        tables[b, :need[b]] = perm[pos:pos + need[b]]
+        pos += need[b]
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    q = torch.randn(len(lens), hq, d, generator=g, device=DEV).to(torch.bfloat16)
+    kp = torch.randn(nb, bs, hkv, d, generator=g, device=DEV).to(torch.bfloat16)
+    vp = torch.randn(nb, bs, hkv, d, generator=g, device=DEV).to(torch.bfloat16)
+    return q, kp, vp, tables, lens
+
+
+def test_a_wait_that_runs_out_sets_the_status_zeroes_its_outputs_and_leaves_the_context_usable():
+    from paged_kv_cache_455_b200 import pa
+    # sequence 0 is split over (nearly) every CTA, so its pieces are merged
+    # cooperatively and every holder waits for the count; sequence 1 is short
+    # and far from CTA 1, whose pieces are withheld
+    q, kp, vp, tables, lens = _case(21, [8192, 100])
+    tab, cl = torch.from_numpy(tables).to(DEV), torch.from_numpy(lens).to(DEV)
+    ws = torch.empty(pa.pa_decode_workspace_bytes(2, 16, 4, 256, 8192), dtype=torch.uint8,
+                     device=DEV)
+    ref = O.paged_attention(W.to_numpy_elems(q), W.to_numpy_elems(kp), W.to_numpy_elems(vp),
+                            tables, lens, 1.0 / 16.0, "bf16")
+
+    def run():
+        out = torch.full_like(q, float("nan"))
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        pa.pa_decode_attention(out, q, kp, vp, tab, cl, 8192, 1.0 / 16.0, ws, status)
+        torch.cuda.synchronize()
+        return out, int(status.item())
+
+    pa.testing_set_wait_limit_ns(2_000_000)
+    pa.testing_withhold_pieces(1)
+    try:
+        out, status = run()
+    finally:
+        pa.testing_withhold_pieces(-1)
+        pa.testing_set_wait_limit_ns(0)
+    assert status & pa.PA_DEV_WAIT_TIMEOUT
+    assert status & ~pa.PA_DEV_WAIT_TIMEOUT == 0
+    assert (out[0].float() == 0).all(), "the merge that ran out must leave zeros"
+    got1 = out[1].double().cpu().numpy()
+    assert np.isfinite(got1).all()
+    assert np.abs(got1 - ref[1]).max() <= TOL
+
+    # the context is still usable, and the next call is exact again
+    out, status = run()
+    assert status == 0
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= TOL
