@@ -1,7 +1,7 @@
 #!/usr/bin/env python3
 """Paged decode attention benchmark (one JSON line on stdout, rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config qwen]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
                     [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
 
 A step is one decode step of the whole workload: for each of the 16 layers,
@@ -10,6 +10,13 @@ paged attention (pa_decode_attention), each layer with its own K/V pool, on
 seeded synthetic data already resident in device memory.  Metric: attention
 bytes (query read + KV read + output write) per step over the step time, in
 GB/s, summed over ranks; also decode tokens/s per layer.
+
+Without --config the line's headline is the memory-pressure workload (B=512,
+~120 GB of pools, the largest that fits one GPU), with its end-to-end
+number and the CPU oracle beside it; `per_config` holds the same
+measurement for the Qwen-shaped, long-context and continuous-batch
+workloads (and their FP8-cache variants), and `prefill` the chunked-prefill
+path.  --config NAME measures that one workload as the headline.
 
 With N > 1 (one process per GPU under torch.distributed.run) each rank runs
 its own batch of the same shape (a data-parallel shard drawn with its own
@@ -46,18 +53,24 @@ FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_qwen.md")
 PREFILL_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "prefill_tc_kernel_chunk512.md")
 CSRC = os.path.join(ROOT, "paged_kv_cache_455_b200", "csrc")
+# the default run: the largest single-GPU workload as the headline, the others
+# (the long-context and mixed-batch ones among them) as per-config records
+HEADLINE = "pressure"
+PER_CONFIG = ("qwen", "long", "mix")
 
 
 # ---------------------------------------------------------------------------
 # helpers
 # ---------------------------------------------------------------------------
 
-def attention_bytes(layout: W.BatchLayout) -> int:
-    """Bytes the method must move per layer: Q read + KV read + output write."""
+def attention_bytes(layout: W.BatchLayout, kv_elem: int = 0) -> int:
+    """Bytes the method must move per layer: Q read + KV read + output write
+    (KV elements of kv_elem bytes; 0: the config's element size)."""
     cfg = layout.config
     s = cfg.elem_size
+    kv_elem = kv_elem or s
     qo = 2 * cfg.num_seqs * cfg.num_q_heads * cfg.head_dim * s
-    kv = int(layout.context_lens.astype(np.int64).sum()) * 2 * cfg.num_kv_heads * cfg.head_dim * s
+    kv = int(layout.context_lens.astype(np.int64).sum()) * 2 * cfg.num_kv_heads * cfg.head_dim * kv_elem
     return qo + kv
 
 
@@ -157,13 +170,15 @@ class ClockSampler:
 
 class Workload:
     def __init__(self, cfg: W.DecodeConfig, device, shard: int, length_scale: float = 1.0,
-                 layers=None):
+                 layers=None, fp8: bool = False):
         from paged_kv_cache_455_b200 import pa
         self.pa = pa
         self.cfg = cfg
         self.device = device
+        self.fp8 = fp8
         self.layout = W.make_layout(cfg, length_scale=length_scale, shard=shard)
-        self.layers = W.make_layers(self.layout, device, layers=layers)
+        self.layers = (W.make_layers_fp8 if fp8 else W.make_layers)(self.layout, device,
+                                                                    layers=layers)
         self.tables, self.lens, self.slots = W.device_metadata(self.layout, device)
         L = self.layout
         nbytes = pa.pa_decode_workspace_bytes(cfg.num_seqs, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
@@ -174,15 +189,27 @@ class Workload:
 
     def attention(self, i, tables=None, lens=None):
         pa, l, L = self.pa, self.layers[i], self.layout
-        pa.pa_decode_attention(self.outs[i], l.query, l.k_pool, l.v_pool,
-                               self.tables if tables is None else tables,
-                               self.lens if lens is None else lens, L.max_context_len,
-                               self.cfg.scale, self.workspace, self.status)
+        tables = self.tables if tables is None else tables
+        lens = self.lens if lens is None else lens
+        if self.fp8:
+            pa.pa_decode_attention_fp8(self.outs[i], l.query, l.k_pool, l.v_pool, tables, lens,
+                                       L.max_context_len, self.cfg.scale, W.FP8_SCALE,
+                                       W.FP8_SCALE, self.workspace, self.status)
+        else:
+            pa.pa_decode_attention(self.outs[i], l.query, l.k_pool, l.v_pool, tables, lens,
+                                   L.max_context_len, self.cfg.scale, self.workspace, self.status)
+
+    def cache_write(self, i, key, value, slots):
+        l = self.layers[i]
+        if self.fp8:
+            self.pa.pa_reshape_and_cache_fp8(key, value, l.k_pool, l.v_pool, slots, W.FP8_SCALE,
+                                             W.FP8_SCALE, self.status)
+        else:
+            self.pa.pa_reshape_and_cache(key, value, l.k_pool, l.v_pool, slots, self.status)
 
     def layer_step(self, i, tables=None, lens=None, slots=None):
         l = self.layers[i]
-        self.pa.pa_reshape_and_cache(l.key, l.value, l.k_pool, l.v_pool,
-                                     self.slots if slots is None else slots, self.status)
+        self.cache_write(i, l.key, l.value, self.slots if slots is None else slots)
         self.attention(i, tables, lens)
 
     def step(self):
@@ -190,24 +217,33 @@ class Workload:
             self.layer_step(i)
 
 
-def run_ours(args, rank, world, device, dist):
+def profile_summary(name: str) -> str:
+    return os.path.join(ROOT, "profiles", f"decode_kernel_{name}.md")
+
+
+def measure_decode(cfg: W.DecodeConfig, args, rank, world, device, dist, headline: bool,
+                   fp8: bool = False):
+    """Times one workload: K replays of a CUDA graph of the 16-layer step
+    (cache write + attention per layer) and K replays of a graph of the
+    attention calls alone, on device events, with clocks sampled meanwhile.
+    Returns the headline record (with end-to-end and CPU-baseline legs) or a
+    per-config record."""
     from paged_kv_cache_455_b200 import pa
-    cfg = W.CONFIGS[args.config]
-    length_scale = 1.0
-    if cfg.name == "pressure":
+    length_scale = args.length_scale
+    if cfg.name == "pressure" and length_scale == 1.0:
         free, _ = torch.cuda.mem_get_info(device)
         length_scale = W.fit_length_scale(cfg, free)
-    wl = Workload(cfg, device, shard=rank, length_scale=length_scale, layers=args.layers)
+    wl = Workload(cfg, device, shard=rank, length_scale=length_scale, layers=args.layers, fp8=fp8)
     L = wl.layout
     nl = len(wl.layers)
-    bytes_layer = attention_bytes(L)
+    bytes_layer = attention_bytes(L, 1 if fp8 else 0)
     torch.cuda.synchronize(device)
 
     for _ in range(args.warmup):
         wl.step()
     torch.cuda.synchronize(device)
     if int(wl.status.item()) != 0:
-        raise RuntimeError(f"device status {int(wl.status.item())} during warm-up")
+        raise RuntimeError(f"device status {int(wl.status.item())} during warm-up ({cfg.name})")
 
     # ---- one decode step (every layer: cache write then attention) and the
     # attention calls alone, each captured once as a CUDA graph and replayed;
@@ -261,15 +297,17 @@ def run_ours(args, rank, world, device, dist):
     torch.cuda.synchronize(device)
     attn_ms_mean = a0.elapsed_time(a1) / (args.steps * nl)
 
-    # ---- the same step launched eagerly (host overhead included), for context
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(max(3, args.steps // 4)):
-        wl.step()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    eager_ms = e0.elapsed_time(e1) / max(3, args.steps // 4)
+    eager_ms = None
+    if headline:
+        # ---- the same step launched eagerly (host overhead included)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(max(3, args.steps // 4)):
+            wl.step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        eager_ms = e0.elapsed_time(e1) / max(3, args.steps // 4)
     del step_graph, attn_graph
 
     # max over ranks of the step time, sum over ranks of the work
@@ -281,15 +319,43 @@ def run_ours(args, rank, world, device, dist):
     value = step_bytes_all / (ms_per_step * 1e-3) / 1e9
     t_layer_s = ms_per_step * 1e-3 / nl
     tokens_per_s_layer = seqs_all / t_layer_s
+    peak, peak_kind = measured_peak()
+    achieved = bytes_layer / (attn_ms_mean * 1e-3) / 1e9
+    traffic = profiled_traffic(profile_summary(cfg.name + ("_fp8" if fp8 else "")))
+    if traffic is not None and length_scale != 1.0:
+        traffic = None   # the committed capture is of the unscaled workload
+
+    if not headline:
+        rec = {
+            "workload": f"{cfg.name}: {cfg.description}" + (
+                f"; FP8 (E4M3) cache, per-tensor scales {W.FP8_SCALE:.6g}, bf16 query and "
+                "output" if fp8 else ""),
+            "layers": nl, "num_seqs_per_gpu": cfg.num_seqs,
+            "sum_context_lens_per_gpu": int(L.context_lens.sum()),
+            "max_context_len": L.max_context_len,
+            "step_ms": round(ms_per_step, 4),
+            "step_gbs": round(value, 1),
+            "step_pct_of_8tbs_per_gpu": round(100 * value / (NOMINAL_HBM_GBS * world), 2),
+            "attention_us_per_launch": round(attn_ms_mean * 1e3, 2),
+            "attention_us_worst_rank": round(attn_ms_worst * 1e3, 2),
+            "attention_gbs_per_gpu": round(achieved, 1),
+            "attention_pct_of_8tbs": round(100 * achieved / NOMINAL_HBM_GBS, 2),
+            "frac": round(achieved / peak, 4),
+            "peak": peak, "peak_source": f"{peak_kind} HBM copy bandwidth",
+            "algorithmic_bytes_per_launch": bytes_layer,
+            "traffic": traffic,
+            "tokens_per_s_per_layer": round(tokens_per_s_layer, 1),
+            "gpu_launches": int(launches),
+            "clocks": clocks.summary(),
+        }
+        del wl
+        torch.cuda.empty_cache()
+        return rec
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(wl, args, device, dist, world, bytes_layer)
-
-    peak, peak_kind = measured_peak()
-    achieved = bytes_layer / (attn_ms_mean * 1e-3) / 1e9
-    traffic = profiled_traffic()
 
     out = {
         "metric": METRIC,
@@ -302,7 +368,7 @@ def run_ours(args, rank, world, device, dist):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": cfg.dtype,
+        "dtype": "e4m3 KV, bf16 query/output" if fp8 else cfg.dtype,
         "data": "synthetic (seeded N(0,1) Q/K/V, seeded lengths and block tables)",
         "config": {
             "workload": f"{cfg.name}: {cfg.description}",
@@ -330,8 +396,10 @@ def run_ours(args, rank, world, device, dist):
         "clocks": clocks.summary(),
         "e2e": e2e,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         out["cpu_baseline"] = cpu_baseline(cfg, L, wl.layers[0], budget_s=args.cpu_seconds)
+    del wl
+    torch.cuda.empty_cache()
     return out
 
 
@@ -348,33 +416,88 @@ def combine_ranks(dist, device, ms_per_step, attn_ms, step_bytes, seqs):
 
 
 def run_e2e(wl: Workload, args, device, dist, world, bytes_layer):
-    """Same metric through the public API with host (pinned) buffers: each
-    step copies every layer's query / new key / new value and the batch
-    metadata host->device, runs the 16 layers, and copies every output back."""
+    """Same metric through the public API with host (pinned) buffers.  Every
+    step copies each layer's query, new key and new value (one pinned block
+    per layer) and the batch metadata host->device, runs the layers, and
+    copies every layer's output back.  The host->device copies run on one
+    side stream and the device->host copies on another, ordered by events,
+    so that they overlap the layers' kernels; the timed region starts before
+    the first step's first copy and ends after its last one."""
     L, cfg = wl.layout, wl.cfg
-    host_q = [l.query.cpu().pin_memory() for l in wl.layers]
-    host_k = [l.key.cpu().pin_memory() for l in wl.layers]
-    host_v = [l.value.cpu().pin_memory() for l in wl.layers]
-    host_tab = torch.from_numpy(L.block_tables).pin_memory()
-    host_len = torch.from_numpy(L.context_lens).pin_memory()
-    host_slot = torch.from_numpy(L.slot_mapping).pin_memory()
-    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in wl.outs]
-    dev_tab, dev_len, dev_slot = (torch.empty_like(wl.tables), torch.empty_like(wl.lens),
-                                  torch.empty_like(wl.slots))
-    h2d = sum(t.numel() * t.element_size() for t in host_q + host_k + host_v) + \
-        sum(t.numel() * t.element_size() for t in (host_tab, host_len, host_slot))
-    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    nl = len(wl.layers)
+    l0 = wl.layers[0]
+    parts = (l0.query, l0.key, l0.value)
+    sizes = [t.numel() * t.element_size() for t in parts]
+    per_layer = sum(sizes)
+    host_in = torch.empty((nl, per_layer), dtype=torch.uint8).pin_memory()
+    dev_in = torch.empty((nl, per_layer), dtype=torch.uint8, device=device)
+    for i, l in enumerate(wl.layers):
+        off = 0
+        for t, n in zip((l.query, l.key, l.value), sizes):
+            host_in[i, off:off + n].copy_(t.contiguous().view(-1).view(torch.uint8).cpu())
+            off += n
+    views = []
+    for i in range(nl):
+        off, vs = 0, []
+        for t, n in zip(parts, sizes):
+            vs.append(dev_in[i, off:off + n].view(t.dtype).view(t.shape))
+            off += n
+        views.append(vs)
+    # metadata: slots (int64) first, then tables and lengths (int32)
+    tab, lens, slots = L.block_tables, L.context_lens, L.slot_mapping
+    mbytes = [slots.nbytes, tab.nbytes, lens.nbytes]
+    host_meta = torch.empty(sum(mbytes), dtype=torch.uint8).pin_memory()
+    off = 0
+    for a, n in zip((slots, tab, lens), mbytes):
+        host_meta[off:off + n].copy_(torch.from_numpy(np.ascontiguousarray(a)).view(-1).view(torch.uint8))
+        off += n
+    dev_meta = torch.empty_like(host_meta, device=device)
+    d_slots = dev_meta[:mbytes[0]].view(torch.int64)
+    d_tab = dev_meta[mbytes[0]:mbytes[0] + mbytes[1]].view(torch.int32).view(tab.shape)
+    d_lens = dev_meta[mbytes[0] + mbytes[1]:].view(torch.int32)
+    host_out = torch.empty((nl,) + tuple(l0.query.shape), dtype=l0.query.dtype).pin_memory()
+    h2d_bytes = host_in.numel() + host_meta.numel()
+    d2h_bytes = host_out.numel() * host_out.element_size()
+
+    compute = torch.cuda.current_stream(device)
+    up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()
+    ev_in, ev_used, ev_done, ev_back = ([ev() for _ in range(nl)] for _ in range(4))
+    ev_meta, ev_meta_used = ev(), ev()
+
+    def layer(i):
+        q, k, v = views[i]
+        l = wl.layers[i]
+        wl.cache_write(i, k, v, d_slots)
+        if wl.fp8:
+            wl.pa.pa_decode_attention_fp8(wl.outs[i], q, l.k_pool, l.v_pool, d_tab, d_lens,
+                                          L.max_context_len, cfg.scale, W.FP8_SCALE, W.FP8_SCALE,
+                                          wl.workspace, wl.status)
+        else:
+            wl.pa.pa_decode_attention(wl.outs[i], q, l.k_pool, l.v_pool, d_tab, d_lens,
+                                      L.max_context_len, cfg.scale, wl.workspace, wl.status)
 
     def step():
-        dev_tab.copy_(host_tab, non_blocking=True)
-        dev_len.copy_(host_len, non_blocking=True)
-        dev_slot.copy_(host_slot, non_blocking=True)
-        for i, l in enumerate(wl.layers):
-            l.query.copy_(host_q[i], non_blocking=True)
-            l.key.copy_(host_k[i], non_blocking=True)
-            l.value.copy_(host_v[i], non_blocking=True)
-            wl.layer_step(i, dev_tab, dev_len, dev_slot)
-            host_out[i].copy_(wl.outs[i], non_blocking=True)
+        with torch.cuda.stream(up):
+            up.wait_event(ev_meta_used)
+            dev_meta.copy_(host_meta, non_blocking=True)
+            ev_meta.record(up)
+            for i in range(nl):
+                up.wait_event(ev_used[i])        # the previous step has read layer i's inputs
+                dev_in[i].copy_(host_in[i], non_blocking=True)
+                ev_in[i].record(up)
+        compute.wait_event(ev_meta)
+        for i in range(nl):
+            compute.wait_event(ev_in[i])
+            compute.wait_event(ev_back[i])       # the previous step's output i is on the host
+            layer(i)
+            ev_used[i].record(compute)
+            ev_done[i].record(compute)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_done[i])
+                host_out[i].copy_(wl.outs[i], non_blocking=True)
+                ev_back[i].record(down)
+        ev_meta_used.record(compute)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -383,19 +506,27 @@ def run_e2e(wl: Workload, args, device, dist, world, bytes_layer):
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
-    s.record()
+    s.record(compute)
+    up.wait_event(s)
     for _ in range(steps):
         step()
-    e.record()
+    for i in range(nl):
+        compute.wait_event(ev_back[i])
+    e.record(compute)
     torch.cuda.synchronize(device)
+    if int(wl.status.item()) != 0:
+        raise RuntimeError(f"device status {int(wl.status.item())} in the end-to-end leg")
     ms = s.elapsed_time(e) / steps
     if dist is not None:
         t = torch.tensor([ms], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t[0])
-    value = world * bytes_layer * len(wl.layers) / (ms * 1e-3) / 1e9
+    value = world * bytes_layer * nl / (ms * 1e-3) / 1e9
     return {"value": round(value, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+            "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(d2h_bytes),
+            "copies": "one pinned block per layer (query, new key, new value) and one of "
+                      "metadata host->device on a side stream, every layer's output "
+                      "device->host on another, overlapping the kernels"}
 
 
 # ---------------------------------------------------------------------------
@@ -453,7 +584,7 @@ def cpu_baseline(cfg, layout, layer, budget_s=10.0, threads=0):
 
 
 def run_reference(args, rank, world, device):
-    cfg = W.CONFIGS[args.config]
+    cfg = W.CONFIGS[args.config or HEADLINE]
     layout = W.make_layout(cfg)
     (layer,) = W.make_layers(layout, device, layers=1)
     from oracle import oracle as O
@@ -540,9 +671,11 @@ def prefill_workload(device, layers: int, seed: int = 455 + 6):
     return L, dev, meta
 
 
-def run_prefill(args, device):
+def run_prefill(args, device, record: bool = False):
+    """Times the chunked-prefill step (--path prefill), or, with record=True,
+    the same measurement as a sub-record of the default decode line."""
     from paged_kv_cache_455_b200 import pa
-    layers = args.layers or 4
+    layers = 4 if record else (args.layers or 4)
     L, dev, meta = prefill_workload(device, layers)
     status = torch.zeros(1, dtype=torch.int32, device=device)
     maxctx = int(meta["lens"].max())
@@ -634,9 +767,11 @@ def run_prefill(args, device):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="qwen", choices=sorted(W.CONFIGS))
+    ap.add_argument("--config", default=None, choices=sorted(W.CONFIGS),
+                    help="measure only this workload (default: the memory-pressure headline "
+                         "plus the per-config records)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -645,6 +780,13 @@ def main(argv=None):
                     help="layers per step (default: the workload's 16); fewer only for profiling")
     ap.add_argument("--path", default="decode", choices=["decode", "prefill"],
                     help="decode (the default measurement) or the chunked-prefill path")
+    ap.add_argument("--length-scale", type=float, default=1.0,
+                    help="shrink every context length (profiling captures of the large "
+                         "workloads only)")
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="with --config: measure the workload over an FP8 (E4M3) cache")
+    ap.add_argument("--no-prefill", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -680,7 +822,26 @@ def main(argv=None):
         print(json.dumps(run_prefill(args, device)), flush=True)
         return 0
     try:
-        line = run_ours(args, rank, world, device, dist)
+        if args.config is not None:
+            line = measure_decode(W.CONFIGS[args.config], args, rank, world, device, dist,
+                                  headline=True, fp8=args.fp8)
+        else:
+            per = {}
+            if not args.no_per_config:
+                for name in PER_CONFIG:
+                    per[name] = measure_decode(W.CONFIGS[name], args, rank, world, device, dist,
+                                               headline=False)
+                for name in PER_CONFIG:
+                    per[name + "_fp8"] = measure_decode(W.CONFIGS[name], args, rank, world, device,
+                                                        dist, headline=False, fp8=True)
+            prefill = None
+            if world == 1 and not args.no_prefill:
+                prefill = run_prefill(args, device, record=True)
+                torch.cuda.empty_cache()
+            line = measure_decode(W.CONFIGS[HEADLINE], args, rank, world, device, dist,
+                                  headline=True)
+            line["per_config"] = per
+            line["prefill"] = prefill
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
