@@ -43,11 +43,15 @@
  *     launch), and each lets the kernel after it start early, so that a
  *     kernel's set-up overlaps the tail of the one ahead.  The cache write
  *     touches no memory before the kernel ahead has completed.  The decode
- *     kernels read context_lens and block_tables before it has completed
- *     (everything else after): a kernel ahead of them that allows an early
- *     start (griddepcontrol.launch_dependents) must not write those two
- *     arrays.  Kernels that do not allow an early start, host copies and
- *     this library's own kernels need no care.
+ *     kernels read context_lens, block_tables and the K/V pool rows of
+ *     cached tokens other than each sequence's last one before it has
+ *     completed (the query, the last rows, the outputs and the workspace
+ *     after): a kernel ahead of them that allows an early start
+ *     (griddepcontrol.launch_dependents) must not write those arrays or
+ *     rows.  pa_reshape_and_cache, which stores exactly each sequence's
+ *     last row, is such a kernel and is safe; kernels that do not allow an
+ *     early start, host copies and this library's other kernels need no
+ *     care.
  */
 #ifndef PA_H_
 #define PA_H_
@@ -141,7 +145,7 @@ pa_status pa_decode_attention(void *out, const void *query, const void *k_pool,
                               int32_t *dev_status, void *stream);
 
 /* Workspace bytes pa_decode_attention wants for these sizes (enough for GPUs
- * of up to 256 SMs; about 8.5 MB for Hkv = 4, Hq/Hkv = 4, d = 256).  Host
+ * of up to 256 SMs; about 8.7 MB for Hkv = 4, Hq/Hkv = 4, d = 256).  Host
  * only; touches no device.  num_seqs and max_context_len are accepted for
  * symmetry and unused. */
 size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,

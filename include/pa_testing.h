@@ -1,15 +1,17 @@
 /*
  * pa_testing.h -- test hooks of libpa.so.  Not for use in production code.
  *
- * The decode kernels bound every wait: on a stage barrier of their
- * shared-memory ring, and, in a merge of a sequence split over many CTAs,
- * on the count of the pieces the other CTAs have published.  A wait that
- * runs out sets PA_DEV_WAIT_TIMEOUT in *dev_status and the kernel returns
- * normally, leaving the CUDA context usable.  These hooks let a test make
- * such a wait run out, on purpose and quickly, without any fault or hang:
- * one CTA simply does not count its pieces in, so the waits of the CTAs
- * merging with it expire after the limit.  The pages have no counterpart;
- * the hooks exist to test this library's failure handling.
+ * Every wait inside the decode kernels is bounded: a warp waiting for a
+ * stage of its shared-memory ring to be filled (or emptied) gives up after
+ * a time limit, sets PA_DEV_WAIT_TIMEOUT in *dev_status, and the kernel
+ * returns normally, leaving the CUDA context usable.  The outputs of every
+ * sequence whose remaining work that CTA held are then zeros.  No warp of
+ * the decode kernels ever waits for another CTA.  These hooks let a test
+ * make such a wait run out, on purpose and quickly, without any fault or
+ * hang: one CTA's producer leaves the copies of one tile unissued, so the
+ * stage they would fill never completes and the waits on it expire after
+ * the limit.  The pages have no counterpart; the hooks exist to test this
+ * library's failure handling.
  *
  * Both settings are process-wide, apply to decode launches made after the
  * call, and are not thread-safe with respect to concurrent launches.
@@ -25,12 +27,12 @@ extern "C" {
  * restores the default (2 s). */
 void pa_testing_set_wait_limit_ns(unsigned long long ns);
 
-/* CTA `cta` of every following stream-K decode launch publishes no piece
- * of a sequence split across CTAs and does not count it in; it still takes
- * its share of the merges of sequences split into more than 8 pieces.
- * Those merges then run out of time: their outputs are zeros and
- * PA_DEV_WAIT_TIMEOUT is set.  A negative value turns the hook off. */
-void pa_testing_withhold_pieces(int cta);
+/* CTA `cta` of every following decode launch (when its range holds at
+ * least two tiles) issues no copy for its second tile.  Its waits then run
+ * out: PA_DEV_WAIT_TIMEOUT is set, and the outputs of the sequences whose
+ * work from that tile on the CTA held are zeros.  A negative value turns
+ * the hook off. */
+void pa_testing_withhold_copy(int cta);
 
 #ifdef __cplusplus
 }

@@ -36,7 +36,7 @@ using pa::TileGeo;
 std::atomic<unsigned long long> g_launches{0};
 
 // Test hooks (include/pa_testing.h): the bounded-wait limit of the decode
-// kernels and a CTA that withholds its cut pieces.
+// kernels and a CTA whose producer withholds one tile's copies.
 std::atomic<unsigned long long> g_test_wait_ns{0};
 std::atomic<int> g_test_withhold{-1};
 
@@ -516,14 +516,20 @@ int64_t slot_floats(int64_t group, int64_t head_dim)
 
 // Stream-K workspace: two partial slots per CTA and head of the group (a CTA
 // holds at most two pieces of cut segments: one met at the start of its
-// range, one running past its end), then one 64-bit arrival counter per CTA
-// and head (for the cut segment that starts in the CTA's range).
+// range, one running past its end); from the next 128-byte boundary, one
+// arrival counter per CTA and head (for the cut segment that starts in the
+// CTA's range), each on a 128-byte line of its own.
+int64_t partials_bytes(int64_t heads, int64_t group, int64_t head_dim)
+{
+    return round_up(2 * heads * slot_floats(group, head_dim) * 4, 128);
+}
+
 size_t stream_k_bytes(int64_t num_seqs, int64_t num_kv_heads, int64_t group, int64_t head_dim,
                       int64_t ctas)
 {
     (void)num_seqs;
     const int64_t heads = ctas * heads_per_cta((int)num_kv_heads);
-    return (size_t)(2 * heads * slot_floats(group, head_dim) * 4 + round_up(heads * 8, 16));
+    return (size_t)(partials_bytes(heads, group, head_dim) + heads * 128);
 }
 
 // Epoch of a stream-K call: the tag its arrival counters carry.  Distinct
@@ -665,7 +671,7 @@ unsigned long long pa_launch_count(void) { return g_launches.load(); }
 
 void pa_testing_set_wait_limit_ns(unsigned long long ns) { g_test_wait_ns.store(ns); }
 
-void pa_testing_withhold_pieces(int cta) { g_test_withhold.store(cta < 0 ? -1 : cta); }
+void pa_testing_withhold_copy(int cta) { g_test_withhold.store(cta < 0 ? -1 : cta); }
 
 int pa_num_partitions(int max_context_len, int partition_size)
 {
@@ -1040,17 +1046,19 @@ static pa_status decode_entry(void *out, const void *query, const void *k_pool,
         (int64_t)num_seqs * p.head_groups * (round_up(std::max(max_context_len, 1), 16) / 16);
     grid = (int)std::min<int64_t>(grid, tiles_up);
     const size_t need = stream_k_bytes(num_seqs, num_kv_heads, group, head_dim, grid);
-    // the merges use a warp's share of the stage ring as scratch
+    // a merge keeps its pieces' stats and weights in a warp's share of the
+    // stage ring
     const int64_t ring_share = (int64_t)p.geo.spw * p.geo.stage_bytes / p.geo.hpc & ~(int64_t)15;
     const bool stream_k = workspace != nullptr && workspace_bytes >= need &&
                           aligned16(workspace) &&
-                          pa::merge_scratch_bytes(group, head_dim, grid) <= ring_share;
+                          pa::merge_scratch_bytes(group, grid) <= ring_share;
     if (stream_k) {
         p.mode = 0;
         p.slot_floats = (int)slot_floats(group, head_dim);
         p.wpart = static_cast<float *>(workspace);
         p.counters = reinterpret_cast<unsigned long long *>(
-            p.wpart + 2 * (int64_t)grid * p.geo.hpc * p.slot_floats);
+            static_cast<uint8_t *>(workspace) +
+            partials_bytes((int64_t)grid * p.geo.hpc, group, head_dim));
         p.epoch = next_epoch();
     } else {
         p.mode = 1;

@@ -92,7 +92,7 @@ struct DecodeParams {
     float *max_logits;       // [B, Hq, max_parts]
     float *exp_sums;         // [B, Hq, max_parts]
     float *wpart;            // mode 0: two partial slots per CTA and head
-    unsigned long long *counters;  // mode 0: arrivals per cut segment (owner CTA, head)
+    unsigned long long *counters;  // mode 0: arrivals per cut segment (owner CTA, head), a line each
     int32_t *dev_status;
     int64_t num_blocks;
     int num_seqs;
@@ -112,7 +112,7 @@ struct DecodeParams {
     float scale_log2;
     float out_scale;         // multiplies every output (the V scale of an FP8 cache; else 1)
     uint64_t wait_ns;        // limit of every bounded wait (kWaitLimitNs unless a test sets it)
-    int withhold_cta;        // test hook: this CTA does not count its cut pieces in (-1: none)
+    int withhold_cta;        // test hook: this CTA's producer withholds its second tile's copy (-1: none)
     TileGeo geo;
 };
 
@@ -1144,6 +1144,15 @@ __device__ __forceinline__ int piece_slot(int x, bool first, int hpc, int hl)
     return (2 * x + (first ? 1 : 0)) * hpc + hl;
 }
 
+// 64-bit words per 128-byte line: every arrival counter sits on a line of
+// its own, so that the atomics of one segment do not queue behind another's.
+constexpr int kLineWords = 16;
+
+__device__ __forceinline__ unsigned long long *counter_of(const DecodeParams &p, int x, int hl)
+{
+    return p.counters + ((int64_t)x * p.geo.hpc + hl) * kLineWords;
+}
+
 // Offset (floats) of a published piece's max / sum / bad mark: after the
 // accumulator units of either tile math (the tensor-core layout pads an odd
 // group to an even one).
@@ -1153,11 +1162,10 @@ __host__ __device__ constexpr int piece_stats_off(int D, int G) { return 2 * D *
 __host__ __device__ constexpr int stats_units(int G) { return (2 * G + 1 + 3) / 4; }
 
 // Bytes of per-warp shared scratch a merge of a cut segment of up to np
-// pieces needs: np stats blocks, np x G weights, 2 G totals, and the units of
-// at least one piece (more pieces per copy round when the scratch allows).
-__host__ __device__ constexpr int64_t merge_scratch_bytes(int G, int D, int64_t np)
+// pieces needs: np stats blocks and np x G weights.
+__host__ __device__ constexpr int64_t merge_scratch_bytes(int G, int64_t np)
 {
-    return 4 * ((int64_t)piece_stats_off(D, G) + 4 * np * stats_units(G) + np * G + 2 * G + 4);
+    return 4 * (4 * np * stats_units(G) + np * G);
 }
 
 // Counts one more arrival at a cut segment's counter for this call and
@@ -1202,187 +1210,193 @@ __device__ __forceinline__ int segment_arrive(unsigned long long *c, uint32_t ep
     return 0;
 }
 
-// Segments cut into more pieces than this are merged by all of their
-// CTAs together (each a slice of the outputs) rather than by the last one.
-constexpr int kLastMergesPieces = 8;
+// Weight of head g among a lane's G per-head values (G is small: the
+// selection unrolls into compares, keeping the values in registers).
+template <int G>
+__device__ __forceinline__ float pick(const float (&v)[G], int g)
+{
+    float r = 0.f;
+#pragma unroll
+    for (int k = 0; k < G; ++k)
+        r = (k == g) ? v[k] : r;
+    return r;
+}
 
-// Merge of a segment cut across the CTAs x0..xl (mode 0, np pieces), for
-// this warp's head of the group, after the warp's range, over the published
-// units [lo, lo + S) of every piece:
-//   - np <= kLastMergesPieces: the warp whose arrival completed the count
-//     merges every unit (lo = 0, S = U), all pieces being published;
-//   - otherwise every participant q = blockIdx.x - x0 takes the units
-//     [q U / np, (q + 1) U / np), after waiting (bounded) for the count.
-// The result is the log-sum-exp combination of the pieces' partial softmax
-// states (max m_i, sum l_i, accumulator a_i, log2 domain):
+// Per-head maxima, sums and weights of a cut segment's pieces from the
+// stats block `st` ([np][4 SU] floats in shared memory, or NULL to read
+// piece `lane` of `np <= 32` from `gst`), by a whole warp: lane i handles
+// pieces i, i + 32, ...; the butterflies run in a fixed order, so the result
+// does not depend on timing.  Leaves w_i = 2^(m_i - M) / L * out_scale for
+// the pieces a lane handles in wl[G] (first piece only) and, with `w`, for
+// every piece in w[np][G].
+template <int G>
+__device__ __forceinline__ void piece_weights(const float *st, int np, float out_scale, float *w,
+                                              float (&wl)[G], int lane)
+{
+    constexpr int SU = stats_units(G);
+    float M[G], L[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        M[g] = -INFINITY;
+        L[g] = 0.f;
+    }
+    for (int i = lane; i < np; i += 32)
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            M[g] = fmaxf(M[g], st[i * 4 * SU + g]);
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            M[g] = fmaxf(M[g], __shfl_xor_sync(kFull, M[g], o));
+    for (int i = lane; i < np; i += 32)
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float mi = st[i * 4 * SU + g];
+            if (M[g] != -INFINITY && mi != -INFINITY)
+                L[g] = fmaf(st[i * 4 * SU + G + g], ptx::ex2(mi - M[g]), L[g]);
+        }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            L[g] += __shfl_xor_sync(kFull, L[g], o);
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+        wl[g] = 0.f;
+    for (int i = lane; i < np; i += 32)
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float mi = st[i * 4 * SU + g];
+            // out_scale (1 unless the cache is FP8) multiplies the weights exactly
+            const float wi = (mi == -INFINITY || !(L[g] > 0.f))
+                                 ? 0.f
+                                 : ptx::ex2(mi - M[g]) / L[g] * out_scale;
+            if (w)
+                w[i * G + g] = wi;
+            if (i == lane)
+                wl[g] = wi;
+        }
+}
+
+// Merge of a segment cut into np pieces (CTAs x0 .. x0 + np - 1), for head
+// hl of the group, by the warp whose arrival completed the segment's count,
+// after its range.  The result is the log-sum-exp combination of the pieces'
+// partial softmax states (max m_i, sum l_i, accumulator a_i, log2 domain):
 //     M = max_i m_i,   L = sum_i l_i 2^(m_i - M),   o = sum_i a_i 2^(m_i - M) / L,
-// the identity the split-K reduction uses, with every sum taken in piece
-// order so that the result does not depend on timing.  The stats and units
-// come into shared memory by 16-byte asynchronous copies, as many pieces per
-// round as `buf` holds.
+// the identity the split-K reduction uses.  The pieces' stats go through
+// shared memory (`scratch`, 16 np (SU + G) bytes at least); the units come
+// straight into registers through L2 (lane e holds units e, e + 32, ...),
+// four pieces in flight at a time, and the weighted sums run in piece order,
+// so that the result does not depend on timing.
 template <typename T, int D, int G, typename Math>
-__device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, int total, int segS,
-                                                  int ns, int64_t bh0, int hl, float *buf,
-                                                  int buf_floats, int lane)
+__device__ __forceinline__ void merge_last(const DecodeParams &p, int x0, int np, int64_t bh0,
+                                           int hl, float *scratch, int lane)
 {
     constexpr int U = Math::kUnits;
-    constexpr int UL = (U + 31) / 32;     // units per lane, at most
+    constexpr int UL = (U + 31) / 32;
     constexpr int SO = piece_stats_off(D, G);
     constexpr int SU = stats_units(G);
     const int hpc = p.geo.hpc;
-    const int x0 = cta_of(segS, C, total);
-    const int np = cta_of(segS + ns - 1, C, total) - x0 + 1;
-    int lo = 0, S = U;
     T *out = static_cast<T *>(p.out) + bh0 * D;
-    if (np > kLastMergesPieces) {
-        const int q = (int)blockIdx.x - x0;
-        lo = (int)((int64_t)q * U / np);
-        S = (int)((int64_t)(q + 1) * U / np) - lo;
-        bool done = false;
-        if (lane == 0) {
-            const unsigned long long want = ((unsigned long long)p.epoch << 32) | (unsigned)np;
-            unsigned long long *c = p.counters + (int64_t)x0 * hpc + hl;
-            const uint64_t t0 = ptx::globaltimer_ns();
-            for (uint32_t i = 0; i < (1u << 26); ++i) {
-                if (ptx::ld_acquire_gpu_u64(c) == want) {
-                    done = true;
-                    break;
-                }
-                __nanosleep(64);
-                if ((i & 15u) == 0 && ptx::globaltimer_ns() - t0 > p.wait_ns)
-                    break;
-            }
-            if (!done)
-                report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
-        }
-        done = __shfl_sync(kFull, done, 0);
-        // the warp barrier orders the lanes' copies below after lane 0's
-        // acquiring load (the copies bypass L1)
-        __syncwarp();
-        if (!done) {
-            for (int f = lane; f < 4 * S; f += 32) {
-                int g, d;
-                Math::unit_coords(lo + (f >> 2), f & 3, g, d);
-                if (g < G)
-                    store_out<T>(out + g * D + d, 0.f);
-            }
-            return;
-        }
-    }
-    float *st = buf;                      // [np][SU] float4
-    float *w = st + 4 * np * SU;          // [np][G]
-    float *tot = w + np * G;              // [G] M, [G] L
-    float *raw = buf + ((4 * np * SU + np * G + 2 * G + 3) & ~3);   // [CP][S] float4
-    const int CP = max(1, (buf_floats - (int)(raw - buf)) / (4 * max(S, 1)));
+    float *stats = scratch;                 // [np][SU] float4
+    float *w = scratch + 4 * np * SU;       // [np][G]
     auto src = [&](int i) {
         return p.wpart + (int64_t)piece_slot(x0 + i, i == 0, hpc, hl) * p.slot_floats;
     };
-    auto copy_units = [&](int i0, int i1) {
-        for (int f = lane; f < (i1 - i0) * S; f += 32) {
-            const int i = f / S;
-            ptx::cp_async16(ptx::smem_u32(raw + 4 * f), src(i0 + i) + 4 * (lo + f - i * S));
-        }
-    };
-
-    // 1. every piece's stats and the first round of units
-    for (int f = lane; f < np * SU; f += 32) {
-        const int i = f / SU;
-        ptx::cp_async16(ptx::smem_u32(st + 4 * f), src(i) + SO + 4 * (f - i * SU));
-    }
-    int i1 = min(np, CP);
-    copy_units(0, i1);
-    ptx::cp_async_wait_all();
-    __syncwarp();
-
     bool bad = false;
-    for (int i = lane; i < np; i += 32)
-        bad |= st[i * 4 * SU + 2 * G] != 0.f;
+    for (int i = lane; i < np; i += 32) {
+        const float4 *s4 = reinterpret_cast<const float4 *>(src(i) + SO);
+#pragma unroll
+        for (int u = 0; u < SU; ++u)
+            reinterpret_cast<float4 *>(stats)[i * SU + u] = __ldcg(s4 + u);
+        bad |= stats[i * 4 * SU + 2 * G] != 0.f;
+    }
     if (__any_sync(kFull, bad)) {
         if (lane == 0)
             report(p.dev_status, PA_DEV_BAD_BLOCK);
-        for (int f = lane; f < 4 * S; f += 32) {
-            int g, d;
-            Math::unit_coords(lo + (f >> 2), f & 3, g, d);
-            if (g < G)
-                store_out<T>(out + g * D + d, 0.f);
+#pragma unroll
+        for (int t = 0; t < UL; ++t) {
+            const int e = lane + 32 * t;
+            if (e < U)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    int g, d;
+                    Math::unit_coords(e, j, g, d);
+                    if (g < G)
+                        store_out<T>(out + g * D + d, 0.f);
+                }
         }
+        __syncwarp();
         return;
     }
-
-    // 2. per-head totals (lane g, pieces in order), then the weights
-    if (lane < G) {
-        float M = -INFINITY, L = 0.f;
-        for (int i = 0; i < np; ++i)
-            M = fmaxf(M, st[i * 4 * SU + lane]);
-        if (M != -INFINITY)
-            for (int i = 0; i < np; ++i) {
-                const float mi = st[i * 4 * SU + lane];
-                if (mi != -INFINITY)
-                    L = fmaf(st[i * 4 * SU + G + lane], ptx::ex2(mi - M), L);
-            }
-        tot[lane] = M;
-        tot[G + lane] = L;
-    }
     __syncwarp();
-    for (int f = lane; f < np * G; f += 32) {
-        const int i = f / G, g = f - i * G;
-        const float mi = st[i * 4 * SU + g], M = tot[g], L = tot[G + g];
-        // out_scale (1 unless the cache is FP8) multiplies the weights exactly
-        w[f] = (mi == -INFINITY || !(L > 0.f)) ? 0.f : ptx::ex2(mi - M) / L * p.out_scale;
-    }
+    float wl[G];
+    piece_weights<G>(stats, np, p.out_scale, w, wl, lane);
     __syncwarp();
-
-    // 3. weighted sums in piece order: the lane holds units lo + lane + 32 t
     float o[UL][4];
 #pragma unroll
     for (int t = 0; t < UL; ++t)
         o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
-    const float4 *raw4 = reinterpret_cast<const float4 *>(raw);
-    for (int i0 = 0; i0 < np;) {
+#pragma unroll 4
+    for (int i = 0; i < np; ++i) {
+        float wp[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            wp[g] = w[i * G + g];
+        const float4 *src4 = reinterpret_cast<const float4 *>(src(i));
 #pragma unroll
         for (int t = 0; t < UL; ++t) {
             const int e = lane + 32 * t;
-            if (e < S) {
-                int gw[4];
+            if (e < U) {
+                const float4 v = __ldcg(src4 + e);
+                const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    int d;
-                    Math::unit_coords(lo + e, j, gw[j], d);
-                    gw[j] = min(gw[j], G - 1);   // padding heads read a real weight
-                }
-                for (int i = i0; i < i1; ++i) {
-                    const float4 v = raw4[(i - i0) * S + e];
-                    const float *wi = w + i * G;
-                    o[t][0] = fmaf(wi[gw[0]], v.x, o[t][0]);
-                    o[t][1] = fmaf(wi[gw[1]], v.y, o[t][1]);
-                    o[t][2] = fmaf(wi[gw[2]], v.z, o[t][2]);
-                    o[t][3] = fmaf(wi[gw[3]], v.w, o[t][3]);
+                    int g, d;
+                    Math::unit_coords(e, j, g, d);
+                    o[t][j] = fmaf(pick<G>(wp, g), vv[j], o[t][j]);
                 }
             }
-        }
-        i0 = i1;
-        if (i0 < np) {
-            i1 = min(np, i0 + CP);
-            __syncwarp();
-            copy_units(i0, i1);
-            ptx::cp_async_wait_all();
-            __syncwarp();
         }
     }
 #pragma unroll
     for (int t = 0; t < UL; ++t) {
         const int e = lane + 32 * t;
-        if (e < S) {
+        if (e < U)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 int g, d;
-                Math::unit_coords(lo + e, j, g, d);
+                Math::unit_coords(e, j, g, d);
                 if (g < G)
                     store_out<T>(out + g * D + d, o[t][j]);
             }
-        }
     }
     __syncwarp();
+}
+
+// Sequence, head group, index in the segment and the segment's tiles of
+// global tile g (no block-table loads).  Warp-uniform; g below the total.
+__device__ __forceinline__ void tile_segment(int g, const DecodeParams &p, const int *cbase,
+                                             int lane, int &b, int &hg, int &j, int &ns)
+{
+    SeqWindow w;
+    const int c = chunk_of(cbase, (p.num_seqs + 31) >> 5, g);
+    window_load(w, c * 32, cbase[c], p, lane);
+    int seqbase, ctx;
+    window_find(w, g, true, b, seqbase, ctx, p, cbase, lane);
+    const int HG = p.head_groups;
+    const int nt = ntiles(ctx);
+    const int PT = p.partition_size >> 4;
+    const int x = g - seqbase;
+    const int nparts = num_parts(ctx, p.partition_size);
+    int part = (int)((int64_t)x / ((int64_t)HG * PT));
+    if (part > nparts - 1)
+        part = nparts - 1;
+    const int rem = x - (int)((int64_t)part * HG * PT);
+    ns = max(1, min(PT, nt - part * PT));
+    hg = rem / ns;
+    j = rem - hg * ns;
 }
 
 // =====================================================================
@@ -1397,19 +1411,21 @@ __device__ __forceinline__ void merge_cut_segment(const DecodeParams &p, int C, 
 // Mode 0 cuts segments at range borders and merges them inside the kernel.
 // Each CTA holding a piece of a cut segment publishes the piece's partial
 // state (acc, max, sum, bad) in its slot, then counts itself in at the
-// segment's counter with an acquire-release atomic add.  A segment of a few
-// pieces is merged, after its range, by the warp whose arrival completed the
-// count; everyone else moves on.  A segment of many pieces is merged by all
-// of its CTAs, each a slice, after waiting for the count (merge_cut_segment).
-// A CTA waits only after its range, when all of its own pieces are counted
-// in, and every CTA of the persistent grid is resident, so every wait ends;
-// each is bounded all the same.
+// segment's counter with an acquire-release atomic add (segment_arrive).
+// The warp whose arrival completes the count merges the segment's head
+// after its range (merge_last); everyone else moves on.  No CTA ever waits
+// for another: a merge reads only pieces whose arrivals it has counted.
+// A stage wait that runs out (bounded, PA_DEV_WAIT_TIMEOUT) makes the warp
+// zero the outputs of every segment its range touches, and the CTA counts
+// nothing in, so those segments keep zeros.
 //
 // The kernel is launched as a programmatic dependent of the kernel before it
 // on the stream.  Before griddepcontrol.wait it reads only the context
-// lengths and the block tables (the kernel ahead must not write them); the
-// query, the pools, the outputs and the workspace come after the wait.  It
-// lets the kernel after it start early in the same way.
+// lengths, the block tables, and the K/V rows of its first tiles that hold
+// no sequence's last cached token (the kernel ahead must write none of
+// them; the cache write stores only last rows); the query, the last rows,
+// the outputs and the workspace come after the wait.  It lets the kernel
+// after it start early in the same way.
 // =====================================================================
 template <typename T, int D, int G, bool MMA, bool TR16, bool KV8>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -1472,36 +1488,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         TileDesc bat0, bat1;
         fill_batch(bat0, win, R0, R1, p, cbase, lane);
         fill_batch(bat1, win, R0 + 32, R1, p, cbase, lane);
-        // the pools and the query may be written by the kernel ahead
-        ptx::grid_wait_prerequisites();
         int filled = 2;
-        int issued = R0;
-        for (; issued < R1; ++issued) {
-            const int i = issued;
-            const int k = i - R0;
+        // Fills ring position k with tile R0 + k (descriptor d): the
+        // metadata, the expected bytes, and the K/V copies (kv) and/or the
+        // segment's query rows (q).  False if the bounded wait for the stage
+        // ran out.
+        auto issue = [&](int k, const TileDesc &d, bool kv, bool q) -> bool {
             const int s = k % spw;
             const uint32_t bar = full0 + 8u * s;
-            if (k >= spw && !ptx::mbar_wait_bounded(empty0 + 8u * s,
-                                                    (uint32_t)(((k / spw) - 1) & 1), p.wait_ns)) {
+            if (kv && k >= spw &&
+                !ptx::mbar_wait_bounded(empty0 + 8u * s, (uint32_t)(((k / spw) - 1) & 1),
+                                        p.wait_ns)) {
                 if (lane == 0)
                     report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
-                break;
+                return false;
             }
-            const TileDesc d = ((k >> 5) & 1) ? shfl_desc(bat1, k & 31) : shfl_desc(bat0, k & 31);
-            const bool newseg = d.j == 0 || i == R0;
-            int tx = newseg ? geo.q_bytes : 0;
-            bool bad = false;
-#pragma unroll
-            for (int bx = 0; bx < 4; ++bx) {
-                if (bx < geo.bpt && bx * geo.tr < d.n) {
-                    if (d.phys[bx] < 0 || (int64_t)d.phys[bx] >= p.num_blocks)
-                        bad = true;
-                    else
-                        tx += 2 * geo.box_tx;
-                }
-            }
+            const bool newseg = d.j == 0 || k == 0;
             const uint32_t stage = sbase + (uint32_t)(s * geo.stage_bytes);
-            if (lane == 0) {
+            // test hook: the copies of this CTA's second tile are not issued,
+            // so the stage never completes and the bounded waits run out
+            const bool withhold = (int)blockIdx.x == p.withhold_cta && k == 1;
+            const int h0 = d.h * hpc;
+            if (kv && lane == 0) {
+                int tx = newseg ? geo.q_bytes : 0;
+                bool bad = false;
+#pragma unroll
+                for (int bx = 0; bx < 4; ++bx) {
+                    if (bx < geo.bpt && bx * geo.tr < d.n) {
+                        if (d.phys[bx] < 0 || (int64_t)d.phys[bx] >= p.num_blocks)
+                            bad = true;
+                        else
+                            tx += 2 * geo.box_tx;
+                    }
+                }
                 StageMeta m;
                 m.b = d.b;
                 m.hg = d.h;
@@ -1514,11 +1533,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 meta[s] = m;
                 // release: consumers see the metadata once the phase completes
                 ptx::mbar_arrive_expect_tx(bar, (uint32_t)tx);
-                const int h0 = d.h * hpc;
 #pragma unroll
                 for (int bx = 0; bx < 4; ++bx) {
                     if (bx >= geo.bpt || bx * geo.tr >= d.n || d.phys[bx] < 0 ||
-                        (int64_t)d.phys[bx] >= p.num_blocks)
+                        (int64_t)d.phys[bx] >= p.num_blocks || withhold)
                         continue;
                     const int row =
                         d.phys[bx] * p.block_size + ((d.t0 + bx * geo.tr) & (p.block_size - 1));
@@ -1527,13 +1545,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tma_load_4d(stage + (uint32_t)geo.kv_bytes + off, &tmap_v, 0, row, 0, h0,
                                      bar, policy);
                 }
-                if (newseg) {
-                    const T *qsrc =
-                        static_cast<const T *>(p.q) + ((int64_t)d.b * Hq + (int64_t)h0 * G) * D;
-                    ptx::bulk_g2s(stage + (uint32_t)geo.q_off, qsrc, (uint32_t)geo.q_bytes, bar);
-                }
+            }
+            if (q && newseg && !withhold && lane == 0) {
+                const T *qsrc = static_cast<const T *>(p.q) + ((int64_t)d.b * Hq + (int64_t)h0 * G) * D;
+                ptx::bulk_g2s(stage + (uint32_t)geo.q_off, qsrc, (uint32_t)geo.q_bytes, bar);
             }
             __syncwarp();
+            return true;
+        };
+        // Before the kernel ahead has completed, the K/V rows of the range's
+        // first tiles are already fetched, as long as none of them holds its
+        // sequence's last cached token: that row is the only one the cache
+        // write ahead of this kernel stores.  Their query rows come after the
+        // wait, as everything else.
+        int early = 0;
+        for (; early < min(spw, R1 - R0); ++early) {
+            const TileDesc d = shfl_desc(bat0, early);
+            if (d.t0 + d.n >= d.ctx)
+                break;
+            issue(early, d, true, false);
+        }
+        // the query, the last rows and the outputs may be written or read by
+        // the kernel ahead
+        ptx::grid_wait_prerequisites();
+        for (int k = 0; k < early; ++k)
+            issue(k, shfl_desc(bat0, k), false, true);
+        int issued = R0 + early;
+        for (; issued < R1; ++issued) {
+            const int i = issued;
+            const int k = i - R0;
+            const TileDesc d = ((k >> 5) & 1) ? shfl_desc(bat1, k & 31) : shfl_desc(bat0, k & 31);
+            if (!issue(k, d, true, true))
+                break;
             // descriptors of batch k/32 are used up: prepare the batch after next
             if ((k & 31) == 31) {
                 if (filled & 1)
@@ -1595,6 +1638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int segS = 0;          // global index of the current segment's first tile
     bool seg_bad = false;
     bool timed_out = false;
+    int lost = R1;         // first tile of the range lost to a wait that ran out
     // cut segments this warp merges (mode 0): one met at the start of the
     // range, one that runs past its end
     int laterS = -1, laterN = 0, laterB = 0, laterHG = 0;
@@ -1603,7 +1647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // this CTA's arrival counters start the call at (epoch, 0) unless an
     // arrival has already counted in them (see segment_arrive)
     if (p.mode == 0 && lane == 0)
-        ptx::red_max_relaxed_gpu_u64(p.counters + (int64_t)blockIdx.x * hpc + hl,
+        ptx::red_max_relaxed_gpu_u64(counter_of(p, blockIdx.x, hl),
                                      (unsigned long long)p.epoch << 32);
 
     for (int i = R0; i < R1; ++i) {
@@ -1613,6 +1657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0)
                 report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
             timed_out = true;
+            lost = i;
             break;
         }
         const StageMeta d = meta[s];
@@ -1677,23 +1722,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // release (the counter update)
                 __syncwarp();
                 const int x0 = cta_of(segS, C, total);
+                const int np = cta_of(segS + d.ns - 1, C, total) - x0 + 1;
                 int arrived = 0;
-                if ((int)blockIdx.x == p.withhold_cta) {
-                    // test hook: the piece is never counted in, so the waits
-                    // of a cooperative merge run out; this CTA still takes
-                    // its share of such a merge
-                    const int npw = cta_of(segS + d.ns - 1, C, total) - x0 + 1;
-                    if (npw > kLastMergesPieces) {
-                        if (first) {
-                            firstS = segS; firstN = d.ns; firstB = d.b; firstHG = d.hg;
-                        } else {
-                            laterS = segS; laterN = d.ns; laterB = d.b; laterHG = d.hg;
-                        }
-                    }
-                    continue;
-                }
                 if (lane == 0)
-                    arrived = segment_arrive(p.counters + (int64_t)x0 * hpc + hl, p.epoch);
+                    arrived = segment_arrive(counter_of(p, x0, hl), p.epoch);
                 arrived = __shfl_sync(kFull, arrived, 0);
                 __syncwarp();
                 if (arrived == 0) {
@@ -1701,8 +1733,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
                     continue;
                 }
-                const int np = cta_of(segS + d.ns - 1, C, total) - x0 + 1;
-                if (np <= kLastMergesPieces && arrived != np)
+                if (arrived != np)
                     continue;   // a later arrival merges the segment
                 if (first) {
                     firstS = segS;
@@ -1748,6 +1779,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    if (timed_out) {
+        // the rest of the range is lost: zero this warp's head of every
+        // segment from the lost tile on (their pieces here are never counted
+        // in, so no merge overwrites the zeros), and of the segments this
+        // warp was to merge; the CTA's other warps do the same for their heads
+        auto zero_segment = [&](int b, int hg) {
+            T *o = static_cast<T *>(p.out) + ((int64_t)b * Hq + (int64_t)(hg * hpc + hl) * G) * D;
+            for (int e = lane; e < G * D; e += 32)
+                store_out<T>(o + e, 0.f);
+        };
+        for (int g = lost; g < R1;) {
+            int b, hg, j, ns;
+            tile_segment(g, p, cbase, lane, b, hg, j, ns);
+            zero_segment(b, hg);
+            g += ns - j;
+        }
+        if (laterS >= 0)
+            zero_segment(laterB, laterHG);
+        if (firstS >= 0)
+            zero_segment(firstB, firstHG);
+    }
     if (p.mode == 0) {
         // every consumer warp is past its last stage (and with it every copy
         // into the ring has landed): the ring is free scratch for the merges
@@ -1756,15 +1808,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             return;
         float *buf = reinterpret_cast<float *>(
             sgen + (int64_t)hl * ((int64_t)stages_bytes / hpc & ~(int64_t)15));
-        const int buf_floats = (int)((int64_t)stages_bytes / hpc / 4) & ~3;
+        auto merge = [&](int S0, int N0, int B0, int HG0) {
+            const int x0 = cta_of(S0, C, total);
+            const int np = cta_of(S0 + N0 - 1, C, total) - x0 + 1;
+            merge_last<T, D, G, Math>(p, x0, np,
+                                      (int64_t)B0 * Hq + (int64_t)(HG0 * hpc + hl) * G, hl, buf,
+                                      lane);
+        };
         if (laterS >= 0)
-            merge_cut_segment<T, D, G, Math>(
-                p, C, total, laterS, laterN,
-                (int64_t)laterB * Hq + (int64_t)(laterHG * hpc + hl) * G, hl, buf, buf_floats, lane);
+            merge(laterS, laterN, laterB, laterHG);
         if (firstS >= 0)
-            merge_cut_segment<T, D, G, Math>(
-                p, C, total, firstS, firstN,
-                (int64_t)firstB * Hq + (int64_t)(firstHG * hpc + hl) * G, hl, buf, buf_floats, lane);
+            merge(firstS, firstN, firstB, firstHG);
     }
 }
 

@@ -89,6 +89,11 @@ __device__ __forceinline__ void st_relaxed_gpu_u64(unsigned long long *p, unsign
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
 // Atomic add with acquire-release semantics at gpu scope; returns the old value.
 __device__ __forceinline__ unsigned long long atom_add_acq_rel_gpu(unsigned long long *p,
                                                                    unsigned long long v)

@@ -57,7 +57,7 @@ SIGNATURES = {
     "pa_launch_count": (ctypes.c_ulonglong, []),
     # include/pa_testing.h
     "pa_testing_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
-    "pa_testing_withhold_pieces": (None, [_I]),
+    "pa_testing_withhold_copy": (None, [_I]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _fn = getattr(lib, _name)
@@ -114,9 +114,10 @@ def testing_set_wait_limit_ns(ns: int) -> None:
     lib.pa_testing_set_wait_limit_ns(int(ns))
 
 
-def testing_withhold_pieces(cta: int) -> None:
-    """Test hook: CTA `cta` of later decode launches withholds its pieces (-1: off)."""
-    lib.pa_testing_withhold_pieces(int(cta))
+def testing_withhold_copy(cta: int) -> None:
+    """Test hook: CTA `cta` of later decode launches withholds the copies of its
+    second tile, so its bounded waits run out (-1: off)."""
+    lib.pa_testing_withhold_copy(int(cta))
 
 
 def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int,
@@ -363,7 +364,7 @@ def pa_splitk_reduce(out: torch.Tensor, tmp_out: torch.Tensor, max_logits: torch
 __all__ = [
     "lib", "LIB_PATH", "SIGNATURES", "PaError", "launch_count",
     "pa_reshape_and_cache", "pa_reshape_and_cache_fp8", "pa_decode_attention_fp8",
-    "testing_set_wait_limit_ns", "testing_withhold_pieces", "pa_copy_blocks", "pa_swap_blocks", "pa_prefill_attention", "pa_decode_attention", "pa_decode_workspace_bytes",
+    "testing_set_wait_limit_ns", "testing_withhold_copy", "pa_copy_blocks", "pa_swap_blocks", "pa_prefill_attention", "pa_decode_attention", "pa_decode_workspace_bytes",
     "pa_decode_attention_static", "PA_STATIC_SCRATCH_BYTES",
     "pa_num_partitions", "pa_splitk_workspace_bytes", "pa_decode_splitk", "pa_splitk_reduce",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA", "PA_ERR_WORKSPACE",

@@ -48,15 +48,16 @@ def test_size_helpers(pa):
     assert pa.pa_num_partitions(8193, 256) == 33
     assert pa.pa_num_partitions(0, 256) == 1
     assert pa.pa_splitk_workspace_bytes(8, 16, 256, 32) == 8 * 16 * 32 * (256 + 2) * 4
-    # two partial slots (G*d + 2G + 1 floats, rounded up to 4) and two flags
-    # per CTA and KV head of the group, for up to 256 CTAs
+    # two partial slots (G*d + 2G + 1 floats, rounded up to 4) per CTA and KV
+    # head of the group, rounded up to 128 bytes; a 128-byte line per arrival
+    # counter (CTA, head); for up to 256 CTAs
+    def ws(heads, slot):
+        return -(-(2 * heads * slot * 4) // 128) * 128 + heads * 128
     slot = -(-(4 * 256 + 2 * 4 + 1) // 4) * 4
-    assert pa.pa_decode_workspace_bytes(8, 16, 4, 256, 8192) == \
-        2 * 256 * 4 * slot * 4 + 2 * 256 * 4 * 4
+    assert pa.pa_decode_workspace_bytes(8, 16, 4, 256, 8192) == ws(256 * 4, slot)
     # two KV heads form one group of two
     slot8 = -(-(8 * 128 + 2 * 8 + 1) // 4) * 4
-    assert pa.pa_decode_workspace_bytes(3, 16, 2, 128, 64) == \
-        2 * 256 * 2 * slot8 * 4 + 2 * 256 * 2 * 4
+    assert pa.pa_decode_workspace_bytes(3, 16, 2, 128, 64) == ws(256 * 2, slot8)
     assert pa.pa_decode_workspace_bytes(8, 16, 4, 256, 1) == \
         pa.pa_decode_workspace_bytes(8, 16, 4, 256, 8192)
     assert pa.pa_decode_workspace_bytes(8, 16, 5, 256, 64) == 0        # Hq % Hkv != 0

@@ -3,8 +3,9 @@
 Every wait inside the decode kernel is bounded; one that runs out sets
 PA_DEV_WAIT_TIMEOUT and the kernel returns normally, so the CUDA context stays
 usable.  The test hooks of include/pa_testing.h shorten the limit to 2 ms and
-make one CTA withhold its pieces of a sequence split over many CTAs: the
-merge of that sequence then waits for a count that never completes.  No
+make one CTA's producer leave one tile's copies unissued: the stage they would
+fill never completes, the CTA's consumer warps give up waiting for it, zero
+the outputs of the sequence whose work they held, and count nothing in.  No
 fault, trap or hang is involved.
 """
 import numpy as np
@@ -41,9 +42,8 @@ def _case(seed, lens, hq=16, hkv=4, d=256, bs=16):
 
 def test_a_wait_that_runs_out_sets_the_status_zeroes_its_outputs_and_leaves_the_context_usable():
     from paged_kv_cache_455_b200 import pa
-    # sequence 0 is split over (nearly) every CTA, so its pieces are merged
-    # cooperatively and every holder waits for the count; sequence 1 is short
-    # and far from CTA 1, whose pieces are withheld
+    # sequence 0 is split over (nearly) every CTA, CTA 1 among them; sequence
+    # 1 is short and held by the last CTAs only
     q, kp, vp, tables, lens = _case(21, [8192, 100])
     tab, cl = torch.from_numpy(tables).to(DEV), torch.from_numpy(lens).to(DEV)
     ws = torch.empty(pa.pa_decode_workspace_bytes(2, 16, 4, 256, 8192), dtype=torch.uint8,
@@ -59,15 +59,15 @@ def test_a_wait_that_runs_out_sets_the_status_zeroes_its_outputs_and_leaves_the_
         return out, int(status.item())
 
     pa.testing_set_wait_limit_ns(2_000_000)
-    pa.testing_withhold_pieces(1)
+    pa.testing_withhold_copy(1)
     try:
         out, status = run()
     finally:
-        pa.testing_withhold_pieces(-1)
+        pa.testing_withhold_copy(-1)
         pa.testing_set_wait_limit_ns(0)
     assert status & pa.PA_DEV_WAIT_TIMEOUT
     assert status & ~pa.PA_DEV_WAIT_TIMEOUT == 0
-    assert (out[0].float() == 0).all(), "the merge that ran out must leave zeros"
+    assert (out[0].float() == 0).all(), "a sequence whose work was lost must be zeros"
     got1 = out[1].double().cpu().numpy()
     assert np.isfinite(got1).all()
     assert np.abs(got1 - ref[1]).max() <= TOL
