@@ -263,11 +263,16 @@ pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_p
  * their dequantised values code * k_scale and code * v_scale.  query and out
  * are bf16 [B, Hq, d]; other arguments, the workspace and the errors as in
  * pa_decode_attention (pa_decode_workspace_bytes sizes the workspace).
- * Arithmetic: codes convert exactly to f16; the query is rounded to f16
- * (components must stay below 65504 in magnitude; those below 2^-14 keep
- * f16's subnormal precision); logits, the softmax and the accumulators are
- * fp32; the softmax weights are rounded to f16 for the P.V product (the same
- * rounded weights make the row sum); the output is rounded to bf16.
+ * Arithmetic: both tile products run on E4M3 tensor cores with the codes as
+ * stored and fp32 accumulation.  Each query row is scaled by a power of two
+ * and split into two E4M3 parts, hi = e4m3(q) and lo = e4m3(q - hi): hi + lo
+ * equals every query component of at least 2^-9 of its row's largest (a
+ * bf16 value has 8 significant bits, hi and lo 4 each); smaller components
+ * carry an absolute error of at most 2^-17 of the row's largest.  A
+ * row with a non-finite component gives NaN logits.  Logits, the softmax and
+ * the accumulators are fp32; the softmax weights (scaled by 2^8) are split
+ * the same way for the P.V product, about 8 significant bits, and the same
+ * split weights make the row sum; the output is rounded to bf16.
  */
 pa_status pa_decode_attention_fp8(void *out, const void *query, const void *k_pool,
                                   const void *v_pool, const int32_t *block_tables,

@@ -383,12 +383,15 @@ bool make_geo(TileGeo &g, int D, int es, int es_q, int bs, int group, int hpc, i
     g.box_stride = (int)round_up((int64_t)hpc * g.head_lines * 128, 1024);
     g.kv_bytes = g.bpt * g.box_stride;
     g.q_head_bytes = group * D * es_q;
-    g.q_bytes = hpc * g.q_head_bytes;
+    // an E4M3 cache's stages carry no query rows (its consumer warps read
+    // them from global memory)
+    g.q_bytes = es == 1 ? 0 : hpc * g.q_head_bytes;
     g.q_off = 2 * g.kv_bytes;
     g.stage_bytes = (int)round_up((int64_t)g.q_off + g.q_bytes, 1024);
     g.box_tx = hpc * g.tr * rowb;
-    const int fixed = pa::decode_smem_fixed(group);
-    const int spw = std::min(pa::kMaxSpw, (pa::kSmemBudget - fixed) / g.stage_bytes);
+    const int fixed = pa::decode_smem_fixed(group, D, es == 1);   // es 1: an E4M3 cache
+    const int spw =
+        std::min(es == 1 ? pa::kMaxSpw : pa::kMaxSpw16, (pa::kSmemBudget - fixed) / g.stage_bytes);
     if (spw < 1)
         return false;
     g.spw = spw;
@@ -1048,7 +1051,8 @@ static pa_status decode_entry(void *out, const void *query, const void *k_pool,
     const size_t need = stream_k_bytes(num_seqs, num_kv_heads, group, head_dim, grid);
     // a merge keeps its pieces' stats and weights in a warp's share of the
     // stage ring
-    const int64_t ring_share = (int64_t)p.geo.spw * p.geo.stage_bytes / p.geo.hpc & ~(int64_t)15;
+    const int64_t ring_share =
+        (int64_t)p.geo.spw * p.geo.stage_bytes / (p.geo.hpc * (kv8 ? pa::kSubs8 : 1)) & ~(int64_t)15;
     const bool stream_k = workspace != nullptr && workspace_bytes >= need &&
                           aligned16(workspace) &&
                           pa::merge_scratch_bytes(group, grid) <= ring_share;

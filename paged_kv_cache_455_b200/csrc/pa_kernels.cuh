@@ -49,12 +49,25 @@
 namespace pa {
 
 #ifndef PA_MAX_SPW
-#define PA_MAX_SPW 4
+#define PA_MAX_SPW 6
 #endif
 
 constexpr int kMaxHpc = 4;                  // KV heads per CTA tile, at most
 constexpr int kThreads = 32 * (kMaxHpc + 1);// launch bound: consumers + producer
-constexpr int kMaxSpw = PA_MAX_SPW;         // stages in the ring, at most
+// Over an FP8 cache each KV head has two consumer warps, taking alternate
+// tiles (the E4M3 tile math is bound by instruction latency, not by issue)
+// (two warpgroups of consumers, then a producer warpgroup of which one warp
+// works; the producer warpgroup hands its registers to the consumers)
+constexpr int kSubs8 = 2;
+constexpr int kThreads8 = 32 * (kMaxHpc * kSubs8 + 4);
+constexpr int kRegsLaunch8 = 65536 / kThreads8 / 8 * 8;   // 168 per thread at launch
+constexpr int kRegsProducer8 = 72;
+constexpr int kRegsConsumer8 = 216;
+static_assert(kMaxHpc * kSubs8 * kRegsConsumer8 + 4 * kRegsProducer8 <=
+                  (kThreads8 / 32) * kRegsLaunch8,
+              "the register split must fit the launch's registers");
+constexpr int kMaxSpw = PA_MAX_SPW;         // stages in the ring, at most (FP8 cache)
+constexpr int kMaxSpw16 = 4;                // stages in the ring, at most (bf16, f32 caches)
 constexpr int kTile = 16;                   // tokens per tile (= MMA M and K)
 constexpr int kSmemBudget = 227 * 1024;     // opt-in dynamic shared memory per CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded copy waits: 2 s
@@ -648,22 +661,34 @@ struct MmaMath {
 
 // =====================================================================
 // Tile math over an E4M3 (FP8) cache: bf16 query and output, one byte per
-// K / V element with a per-tensor scale.  Codes convert exactly to f16
-// (cvt.f16x2.e4m3x2), and the tile products run on f16 tensor cores with
-// fp32 accumulation; the query is rounded to f16 and the softmax weights
-// are f16.  The K scale is folded into the logit scale, the V scale into
-// the output scale.
+// K / V element with a per-tensor scale.  The K scale is folded into the
+// logit scale, the V scale into the output scale.
+//
+// Both tile products run on E4M3 tensor cores (mma m16n8k32, fp32
+// accumulation) with the K and V codes as they are, so the query and the
+// softmax weights must be E4M3 too.  Each query row, scaled by a power of
+// two, is split into hi = e4m3(q) and lo = e4m3(q - hi); S = K hi + K lo is
+// exact for every element of at least 2^-9 of the row's largest (a bf16
+// element has 8 significant bits, hi and lo 4 each).  Each weight, scaled
+// by 2^8 (the row's largest is exactly 256), is split into hi = e4m3(x) and
+// lo = e4m3(x - hi): hi + lo carries about 8 significant bits, as a bf16
+// weight does.  The MMA's reduction index runs over the tile's 16 tokens
+// twice, paired once with hi and once with lo, so one MMA adds V (hi + lo).
+// The running sums take the same hi + lo values, also scaled by 2^8, so the
+// scale cancels in acc / sum (and in the merge of split pieces).
 //
 // One 16-byte unit of a row holds 16 elements.  ldmatrix reads 8 x 8
 // matrices of 16-bit elements, i.e. 8 rows x 16 bytes:
-//   S = K Q^T: lane (r, c) receives bytes 4c .. 4c+3 of row r of a unit.
-//     Bytes 4c, 4c+1 serve as the MMA's columns 2c, 2c+1 and bytes 4c+2,
-//     4c+3 as columns 2c+8, 2c+9 (a fixed permutation of the reduction
-//     index); the query fragment is built with the same permutation.
-//   O^T += V^T P^T (ldmatrix.trans): lane (r, c) receives tokens 2c, 2c+1
-//     of bytes 2r, 2r+1 of a unit; a byte permute pairs the two tokens of
-//     each byte, so MMA row r is element 2r of the unit and row r + 8 is
-//     element 2r + 1.  Accumulator acc[k][0..3] thus holds
+//   S = K Q^T: lane (r, c) receives bytes 4c .. 4c+3 of row (token) r of a
+//     unit; four matrices (tokens 0-7 and 8-15 of two consecutive units)
+//     are exactly the MMA's A fragment over 32 elements, and the query
+//     fragments hold elements 4c .. 4c+3 and 16 + 4c .. 16 + 4c+3 of head r.
+//   O^T += V^T P^T (ldmatrix.trans): lane (r, c) receives, from the matrix of
+//     tokens 0-7 (m0) and of tokens 8-15 (m1), bytes 2r, 2r+1 of tokens 2c,
+//     2c+1.  Byte permutes gather element 2r of tokens 2c, 2c+1, 2c+8, 2c+9
+//     (MMA row r, reduction index 4c .. 4c+3) and element 2r+1 (row r + 8);
+//     the weight fragment lists the same four tokens, gathered by shuffles
+//     from the lanes that computed them.  Accumulator acc[k][0..3] thus holds
 //     O[head 2c][16k + 2r], O[head 2c+1][16k + 2r], O[head 2c][16k + 2r + 1],
 //     O[head 2c+1][16k + 2r + 1].
 // =====================================================================
@@ -674,34 +699,83 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes)
     return (uint32_t)h.x | ((uint32_t)h.y << 16);
 }
 
+// Two fp32 values to E4M3 codes (round to nearest even, saturating to
+// +-448): `lo` in byte 0, `hi` in byte 1.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi)
+{
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3) &
+           0xffffu;
+}
+
 template <int D, int G>
 struct MmaMath8 {
     static_assert(G <= 8, "group must fit the N = 8 MMA");
     static constexpr int KS = D / 16;   // 16-byte units per row
+    static constexpr int K32 = D / 32;  // 32-element reduction steps
 
-    uint32_t qf[KS][2];
+    uint32_t qh[K32][2];   // E4M3 hi parts of sigma * q, this lane's fragment
+    uint32_t ql[K32][2];   // E4M3 lo parts
+    float sf[2];           // logit factor (scale_log2 / sigma) of heads 2c, 2c+1
     float acc[KS][4];
     float m[2];
     float l[2];
 
-    // Query fragments from the stage's query slot ([G][D] bf16).
-    __device__ __forceinline__ void begin(const uint8_t *qslot, int lane)
+    // Query fragments from the segment's query rows ([G][D] bf16, global
+    // memory, read through the read-only path).  Head h's row is scaled by a power of two sigma_h (max |sigma_h q| in [128, 256)),
+    // then split into hi = e4m3(sigma_h q) and lo = e4m3(sigma_h q - hi):
+    // every element of at least 2^-9 max |q| is exactly hi + lo (its 8
+    // significant bits land in two 4-bit codes), smaller ones to within
+    // 2^-10 / sigma_h.  A non-finite row makes its logits NaN.
+    __device__ __forceinline__ void begin(const uint8_t *qrows, int lane, float scale_log2)
     {
         const int r = lane >> 2, c = lane & 3;
+        float x[K32][2][4];
+        float amax = 0.f;
 #pragma unroll
-        for (int k = 0; k < KS; ++k) {
-            if (r < G) {
-                const uint2 w = *reinterpret_cast<const uint2 *>(qslot + (r * D + 16 * k + 4 * c) * 2);
-                qf[k][0] = ptx::pack_f16x2(ptx::bf16lo_to_f32(w.x), ptx::bf16hi_to_f32(w.x));
-                qf[k][1] = ptx::pack_f16x2(ptx::bf16lo_to_f32(w.y), ptx::bf16hi_to_f32(w.y));
-            } else {
-                qf[k][0] = 0u;
-                qf[k][1] = 0u;
+        for (int k = 0; k < K32; ++k)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint2 w = make_uint2(0u, 0u);
+                if (r < G)
+                    w = __ldg(reinterpret_cast<const uint2 *>(qrows + (r * D + 32 * k + 16 * h + 4 * c) * 2));
+                x[k][h][0] = ptx::bf16lo_to_f32(w.x);
+                x[k][h][1] = ptx::bf16hi_to_f32(w.x);
+                x[k][h][2] = ptx::bf16lo_to_f32(w.y);
+                x[k][h][3] = ptx::bf16hi_to_f32(w.y);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    amax = fmaxf(amax, fabsf(x[k][h][i]));
             }
+        amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+        // sigma = 2^(7 - floor(log2 amax)), from the exponent field
+        const int ef = (int)((__float_as_uint(amax) >> 23) & 0xffu);
+        const float sigma = __uint_as_float((uint32_t)min(254, 261 - ef) << 23);
+        const float fac = amax <= 3.4028235e38f ? scale_log2 / sigma : __int_as_float(0x7fc00000);
+#pragma unroll
+        for (int k = 0; k < K32; ++k)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float y0 = x[k][h][0] * sigma, y1 = x[k][h][1] * sigma;
+                const float y2 = x[k][h][2] * sigma, y3 = x[k][h][3] * sigma;
+                const uint32_t h01 = f32x2_to_e4m3x2(y0, y1), h23 = f32x2_to_e4m3x2(y2, y3);
+                const uint32_t f01 = e4m3x2_to_f16x2(h01), f23 = e4m3x2_to_f16x2(h23);
+                const uint32_t l01 = f32x2_to_e4m3x2(y0 - ptx::f16lo_to_f32(f01),
+                                                     y1 - ptx::f16hi_to_f32(f01));
+                const uint32_t l23 = f32x2_to_e4m3x2(y2 - ptx::f16lo_to_f32(f23),
+                                                     y3 - ptx::f16hi_to_f32(f23));
+                qh[k][h] = h01 | (h23 << 16);
+                ql[k][h] = l01 | (l23 << 16);
+            }
+        // lane (r, c) scales the logits of heads 2c, 2c+1, whose factors the
+        // lanes of rows 2c, 2c+1 computed
+        sf[0] = __shfl_sync(kFull, fac, 8 * c);
+        sf[1] = __shfl_sync(kFull, fac, 8 * c + 4);
+#pragma unroll
+        for (int k = 0; k < KS; ++k)
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 acc[k][i] = 0.f;
-        }
         m[0] = m[1] = -INFINITY;
         l[0] = l[1] = 0.f;
     }
@@ -711,23 +785,22 @@ struct MmaMath8 {
     {
         const int r = lane >> 2;
         const int row = (lane & 7) + (((lane >> 3) & 1) << 3), half = lane >> 4;
-        // ---- S = K Q^T (two accumulation chains), two units per ldmatrix
-        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- S = K (hi + lo)^T on E4M3 tensor cores, four accumulation chains
+        float c4[4][4];
 #pragma unroll
-        for (int k2 = 0; k2 < KS / 2; ++k2) {
+        for (int j = 0; j < 4; ++j)
+            c4[j][0] = c4[j][1] = c4[j][2] = c4[j][3] = 0.f;
+#pragma unroll
+        for (int k = 0; k < K32; ++k) {
             uint32_t a[4];
-            ptx::ldsm_x4(kv_addr16(ks, hline, row, 2 * k2 + half), a);
-            const uint32_t f0[4] = {e4m3x2_to_f16x2(a[0]), e4m3x2_to_f16x2(a[1]),
-                                    e4m3x2_to_f16x2(a[0] >> 16), e4m3x2_to_f16x2(a[1] >> 16)};
-            const uint32_t f1[4] = {e4m3x2_to_f16x2(a[2]), e4m3x2_to_f16x2(a[3]),
-                                    e4m3x2_to_f16x2(a[2] >> 16), e4m3x2_to_f16x2(a[3] >> 16)};
-            ptx::mma_f16_16816(sa, f0, qf[2 * k2][0], qf[2 * k2][1]);
-            ptx::mma_f16_16816(sb, f1, qf[2 * k2 + 1][0], qf[2 * k2 + 1][1]);
+            ptx::ldsm_x4(kv_addr16(ks, hline, row, 2 * k + half), a);
+            ptx::mma_e4m3_16832(c4[2 * (k & 1)], a, qh[k][0], qh[k][1]);
+            ptx::mma_e4m3_16832(c4[2 * (k & 1) + 1], a, ql[k][0], ql[k][1]);
         }
         float s[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            s[i] = (sa[i] + sb[i]) * scale_log2;
+            s[i] = ((c4[0][i] + c4[1][i]) + (c4[2][i] + c4[3][i])) * sf[i & 1];
         if (r >= n) {
             s[0] = -INFINITY;
             s[1] = -INFINITY;
@@ -746,15 +819,24 @@ struct MmaMath8 {
         const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
         const float al0 = mn0 == -INFINITY ? 1.f : ptx::ex2(m[0] - mn0);
         const float al1 = mn1 == -INFINITY ? 1.f : ptx::ex2(m[1] - mn1);
-        const float rf0 = mn0 == -INFINITY ? 0.f : mn0;
-        const float rf1 = mn1 == -INFINITY ? 0.f : mn1;
+        // weights x = 2^8 p: exponents against the new max less 8
+        const float rf0 = (mn0 == -INFINITY ? 0.f : mn0) - 8.f;
+        const float rf1 = (mn1 == -INFINITY ? 0.f : mn1) - 8.f;
         m[0] = mn0;
         m[1] = mn1;
-        const uint32_t p01 = ptx::pack_f16x2(ptx::ex2(s[0] - rf0), ptx::ex2(s[1] - rf1));
-        const uint32_t p23 = ptx::pack_f16x2(ptx::ex2(s[2] - rf0), ptx::ex2(s[3] - rf1));
-        // the sum uses the same rounded weights as the MMA
-        l[0] = l[0] * al0 + ptx::f16lo_to_f32(p01) + ptx::f16lo_to_f32(p23);
-        l[1] = l[1] * al1 + ptx::f16hi_to_f32(p01) + ptx::f16hi_to_f32(p23);
+        const float x0 = ptx::ex2(s[0] - rf0), x1 = ptx::ex2(s[1] - rf1);
+        const float x2 = ptx::ex2(s[2] - rf0), x3 = ptx::ex2(s[3] - rf1);
+        // hi = e4m3(x), lo = e4m3(x - hi); x - hi is exact in fp32
+        const uint32_t h01 = f32x2_to_e4m3x2(x0, x1), h23 = f32x2_to_e4m3x2(x2, x3);
+        const uint32_t hf01 = e4m3x2_to_f16x2(h01), hf23 = e4m3x2_to_f16x2(h23);
+        const float y0 = ptx::f16lo_to_f32(hf01), y1 = ptx::f16hi_to_f32(hf01);
+        const float y2 = ptx::f16lo_to_f32(hf23), y3 = ptx::f16hi_to_f32(hf23);
+        const uint32_t l01 = f32x2_to_e4m3x2(x0 - y0, x1 - y1);
+        const uint32_t l23 = f32x2_to_e4m3x2(x2 - y2, x3 - y3);
+        const uint32_t lf01 = e4m3x2_to_f16x2(l01), lf23 = e4m3x2_to_f16x2(l23);
+        // the sums use the same hi + lo as the MMA
+        l[0] = l[0] * al0 + ((y0 + ptx::f16lo_to_f32(lf01)) + (y2 + ptx::f16lo_to_f32(lf23)));
+        l[1] = l[1] * al1 + ((y1 + ptx::f16hi_to_f32(lf01)) + (y3 + ptx::f16hi_to_f32(lf23)));
         if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
             for (int k = 0; k < KS; ++k) {
@@ -764,20 +846,28 @@ struct MmaMath8 {
                 acc[k][3] *= al1;
             }
         }
-        const uint32_t b0 = ptx::movmatrix_trans(p01);
-        const uint32_t b1 = ptx::movmatrix_trans(p23);
-        // ---- O^T += V^T P^T, two units per ldmatrix
+        // lane (r, c) holds the weights of tokens r, r + 8 for heads 2c, 2c+1:
+        // bytes [x(r, 2c), x(r, 2c+1), x(r+8, 2c), x(r+8, 2c+1)].  The weight
+        // fragment of lane (r, c) wants head r at tokens 2c, 2c+1, 2c+8, 2c+9,
+        // held by lanes (2c, r/2) and (2c+1, r/2), byte r%2 and 2 + r%2.
+        const uint32_t whi = h01 | (h23 << 16), wlo = l01 | (l23 << 16);
+        const int srcA = 8 * (lane & 3) + (r >> 1);
+        const uint32_t sel = (r & 1) ? 0x7351u : 0x6240u;
+        const uint32_t b0 =
+            ptx::prmt(__shfl_sync(kFull, whi, srcA), __shfl_sync(kFull, whi, srcA + 4), sel);
+        const uint32_t b1 =
+            ptx::prmt(__shfl_sync(kFull, wlo, srcA), __shfl_sync(kFull, wlo, srcA + 4), sel);
+        // ---- O^T += V^T (hi + lo)^T, two 16-element units per ldmatrix
 #pragma unroll
         for (int k2 = 0; k2 < KS / 2; ++k2) {
             uint32_t a[4];
             ptx::ldsm_x4_trans(kv_addr16(vs, hline, row, 2 * k2 + half), a);
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-                const uint32_t lo = ptx::prmt(a[2 * u], 0u, 0x3120u);       // tokens 0-7
-                const uint32_t hi = ptx::prmt(a[2 * u + 1], 0u, 0x3120u);   // tokens 8-15
-                const uint32_t f[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(lo >> 16),
-                                       e4m3x2_to_f16x2(hi), e4m3x2_to_f16x2(hi >> 16)};
-                ptx::mma_f16_16816(acc[2 * k2 + u], f, b0, b1);
+                const uint32_t e0 = ptx::prmt(a[2 * u], a[2 * u + 1], 0x6420u);   // element 2r
+                const uint32_t e1 = ptx::prmt(a[2 * u], a[2 * u + 1], 0x7531u);   // element 2r+1
+                const uint32_t f[4] = {e0, e1, e0, e1};
+                ptx::mma_e4m3_16832(acc[2 * k2 + u], f, b0, b1);
             }
         }
     }
@@ -789,6 +879,58 @@ struct MmaMath8 {
             l[0] += __shfl_xor_sync(kFull, l[0], o);
             l[1] += __shfl_xor_sync(kFull, l[1], o);
         }
+    }
+
+    // Hands this warp's partial state (before finish) to the head's other
+    // warp: accumulator element e (= 4 k + j) of lane x at kx[32 e + x] for
+    // e < 2 KS (the head's K lines of the stage just used) and at
+    // vx[32 (e - 2 KS) + x] for the rest (its V lines); max, sum and bad mark
+    // at st[32 i + x].
+    __device__ __forceinline__ void save(float *kx, float *vx, float *st, bool bad,
+                                         int lane) const
+    {
+#pragma unroll
+        for (int k = 0; k < KS; ++k)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int e = 4 * k + j;
+                if (e < 2 * KS)
+                    kx[32 * e + lane] = acc[k][j];
+                else
+                    vx[32 * (e - 2 * KS) + lane] = acc[k][j];
+            }
+        st[lane] = m[0];
+        st[32 + lane] = m[1];
+        st[64 + lane] = l[0];
+        st[96 + lane] = l[1];
+        st[128 + lane] = bad ? 1.f : 0.f;
+    }
+
+    // Adds the other warp's partial state (same lane layout, disjoint tiles
+    // of the segment; placed as `save` does): the log-sum-exp combination of
+    // two online-softmax states.  Returns its bad mark.
+    __device__ __forceinline__ bool absorb(const float *kx, const float *vx, const float *st,
+                                           int lane)
+    {
+        const float mp0 = st[lane], mp1 = st[32 + lane];
+        const float mn0 = fmaxf(m[0], mp0), mn1 = fmaxf(m[1], mp1);
+        const float a0 = mn0 == -INFINITY ? 1.f : ptx::ex2(m[0] - mn0);
+        const float a1 = mn1 == -INFINITY ? 1.f : ptx::ex2(m[1] - mn1);
+        const float b0 = mn0 == -INFINITY ? 1.f : ptx::ex2(mp0 - mn0);
+        const float b1 = mn1 == -INFINITY ? 1.f : ptx::ex2(mp1 - mn1);
+#pragma unroll
+        for (int k = 0; k < KS; ++k)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int e = 4 * k + j;
+                const float o = e < 2 * KS ? kx[32 * e + lane] : vx[32 * (e - 2 * KS) + lane];
+                acc[k][j] = acc[k][j] * ((j & 1) ? a1 : a0) + o * ((j & 1) ? b1 : b0);
+            }
+        l[0] = l[0] * a0 + st[64 + lane] * b0;
+        l[1] = l[1] * a1 + st[96 + lane] * b1;
+        m[0] = mn0;
+        m[1] = mn1;
+        return st[128 + lane] != 0.f;
     }
 
     // Published piece layout: as MmaMath (one float4 acc[k][0..3] per unit
@@ -1117,12 +1259,29 @@ struct SimtMath {
     }
 };
 
+// Bytes of one head's exchange area (FP8 cache, two warps per head): the
+// max, sum and bad mark of the partial softmax state one warp hands the
+// other at a segment end, one float per lane and item, then a "full" and a
+// "free" mbarrier.  (The accumulator goes through the stage the handing
+// warp used last, which it keeps until the state has been read.)
+__host__ __device__ constexpr int exchange_bytes(int D)
+{
+    return (32 * 5 * 4 + 16 + 127) / 128 * 128 + 0 * D;
+}
+
+// Offset of the exchange areas from the end of the stages.
+__host__ __device__ constexpr int exchange_off(int G)
+{
+    return (48 * kMaxSpw + kMaxHpc * kTile * G * 4 + 4 * (kMaxChunks + 1) + 127) / 128 * 128;
+}
+
 // Bytes of the decode kernel's dynamic shared memory besides the stages:
 // alignment slack, full and empty barriers, per-stage tile metadata, the
-// CUDA-core math's score rows, and the chunk prefix of the tile counts.
-__host__ __device__ constexpr int decode_smem_fixed(int G)
+// CUDA-core math's score rows, the chunk prefix of the tile counts, and
+// (FP8 cache) the heads' exchange areas.
+__host__ __device__ constexpr int decode_smem_fixed(int G, int D = 0, bool kv8 = false)
 {
-    return 1024 + 16 * kMaxSpw + 32 * kMaxSpw + kMaxHpc * kTile * G * 4 + 4 * (kMaxChunks + 1);
+    return 1024 + exchange_off(G) + (kv8 ? kMaxHpc * exchange_bytes(D) : 0);
 }
 
 // Tile metadata the producer warp hands to the consumer warps with a stage.
@@ -1428,7 +1587,7 @@ __device__ __forceinline__ void tile_segment(int g, const DecodeParams &p, const
 // after it start early in the same way.
 // =====================================================================
 template <typename T, int D, int G, bool MMA, bool TR16, bool KV8>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p)
 {
@@ -1441,8 +1600,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int total_ctas = gridDim.x;
     const int HG = p.head_groups;
     const int Hq = p.num_q_heads;
+    constexpr int SUBS = KV8 ? kSubs8 : 1;   // consumer warps per KV head
 
     // 1024-byte aligned layout: [stages][full bars][empty bars][meta][score rows][chunk prefix]
+    // [exchange areas (FP8)]
     const uint32_t raw = ptx::smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     uint8_t *sgen = smem_raw + (sbase - raw);
@@ -1452,11 +1613,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     StageMeta *meta = reinterpret_cast<StageMeta *>(sgen + stages_bytes + 16 * kMaxSpw);
     float *scores_all = reinterpret_cast<float *>(sgen + stages_bytes + 48 * kMaxSpw);
     int *cbase = reinterpret_cast<int *>(scores_all + kMaxHpc * kTile * G);
+    uint8_t *xarea = sgen + stages_bytes + exchange_off(G);
+    constexpr uint32_t kXBars = 32u * 5u * 4u;   // barriers' offset in an exchange area
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < spw; ++s) {
             ptx::mbar_init(full0 + 8u * s, 1);
             ptx::mbar_init(empty0 + 8u * s, hpc);
+        }
+        if constexpr (SUBS > 1) {
+            for (int h = 0; h < hpc; ++h) {
+                const uint32_t xb = ptx::smem_u32(xarea + h * exchange_bytes(D)) + kXBars;
+                ptx::mbar_init(xb, 1);        // full: the state is in the area
+                ptx::mbar_init(xb + 8u, 1);   // free: the state has been read
+            }
         }
     }
     ptx::fence_mbar_init();
@@ -1472,9 +1642,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // grid leaves; it waits for this grid to complete before using its results
     if (threadIdx.x == 0)
         ptx::grid_launch_dependents();
+    // the producer warp: the last warp of the consumers (bf16, f32), the
+    // first of the producer warpgroup (FP8)
+    const int pw = KV8 ? kMaxHpc * SUBS : hpc;
 
-    if (warp == hpc) {
-        // =================================================== producer warp
+    // =================================================== producer warp
+    auto producer = [&]() {
         if (R0 >= R1)
             return;
         ptx::prefetch_tensormap(&tmap_k);
@@ -1503,7 +1676,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
                 return false;
             }
-            const bool newseg = d.j == 0 || k == 0;
+            // the first tile of each consumer warp of a head in the segment
+            // carries the segment's query rows
+            const bool newseg = d.j < SUBS || k < SUBS;
             const uint32_t stage = sbase + (uint32_t)(s * geo.stage_bytes);
             // test hook: the copies of this CTA's second tile are not issued,
             // so the stage never completes and the bounded waits run out
@@ -1546,9 +1721,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      bar, policy);
                 }
             }
-            if (q && newseg && !withhold && lane == 0) {
+            if (q && newseg && !withhold && lane == 0 && geo.q_bytes > 0) {
                 const T *qsrc = static_cast<const T *>(p.q) + ((int64_t)d.b * Hq + (int64_t)h0 * G) * D;
                 ptx::bulk_g2s(stage + (uint32_t)geo.q_off, qsrc, (uint32_t)geo.q_bytes, bar);
+            }
+            if constexpr (KV8) {
+                // FP8 stages carry no query rows: the consumers read them
+                // from global memory when they start the segment; bring
+                // them into L2 now
+                if (q && (d.j == 0 || k == 0)) {
+                    const uint8_t *qsrc = static_cast<const uint8_t *>(p.q) +
+                                          ((int64_t)d.b * Hq + (int64_t)h0 * G) * D * 2;
+                    for (int off = lane * 128; off < hpc * geo.q_head_bytes; off += 32 * 128)
+                        ptx::prefetch_l2(qsrc + off);
+                }
             }
             __syncwarp();
             return true;
@@ -1594,18 +1780,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        p.wait_ns);
             }
         }
+    };
+    if constexpr (KV8) {
+        // each role's code runs under its own register count
+        if (warp >= kMaxHpc * SUBS) {
+            ptx::setmaxnreg_dec<kRegsProducer8>();
+            if (warp == pw)
+                producer();
+            return;
+        }
+        ptx::setmaxnreg_inc<kRegsConsumer8>();
+        if (warp >= hpc * SUBS)
+            return;   // no work for this warp
+    } else if (warp == pw) {
+        producer();
         return;
     }
 
     // ====================================================== consumer warps
-    const int hl = warp;                        // head within the group
+    const int hl = warp % hpc;                  // head within the group
+    const int sub = warp / hpc;                 // which of the head's SUBS warps
     const int hline = hl * geo.head_lines;      // its first 128-byte line in a box
     float *scores = scores_all + hl * kTile * G;
     // outputs and the workspace may still be in use by the kernel ahead
     ptx::grid_wait_prerequisites();
 
     // Sequences without tiles (length 0 or invalid) get a zero output.
-    for (int b = blockIdx.x; b < p.num_seqs; b += total_ctas) {
+    for (int b = blockIdx.x; sub == 0 && b < p.num_seqs; b += total_ctas) {
         const int rawc = p.context_lens[b];
         if (eff_ctx(rawc, p.ctx_cap) > 0)
             continue;
@@ -1639,6 +1840,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool seg_bad = false;
     bool timed_out = false;
     int lost = R1;         // first tile of the range lost to a wait that ran out
+    int xc = 0;            // state exchanges so far between the head's two warps (FP8)
     // cut segments this warp merges (mode 0): one met at the start of the
     // range, one that runs past its end
     int laterS = -1, laterN = 0, laterB = 0, laterHG = 0;
@@ -1646,11 +1848,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // this CTA's arrival counters start the call at (epoch, 0) unless an
     // arrival has already counted in them (see segment_arrive)
-    if (p.mode == 0 && lane == 0)
+    if (p.mode == 0 && lane == 0 && sub == 0)
         ptx::red_max_relaxed_gpu_u64(counter_of(p, blockIdx.x, hl),
                                      (unsigned long long)p.epoch << 32);
 
-    for (int i = R0; i < R1; ++i) {
+    // with SUBS warps per head, warp `sub` takes tiles R0 + sub, R0 + sub + SUBS, ...
+    for (int i = R0 + sub; i < R1; i += SUBS) {
         const int k = i - R0;
         const int s = k % spw;
         if (!ptx::mbar_wait_bounded(full0 + 8u * s, (uint32_t)((k / spw) & 1), p.wait_ns)) {
@@ -1661,14 +1864,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
         }
         const StageMeta d = meta[s];
-        const bool newseg = d.j == 0 || i == R0;
+        const bool newseg = d.j < SUBS || k < SUBS;   // this warp's first tile of the segment
         const uint32_t kreg = sbase + (uint32_t)(s * geo.stage_bytes);
         const uint32_t vreg = kreg + (uint32_t)geo.kv_bytes;
         const uint8_t *qslot = sgen + s * geo.stage_bytes + geo.q_off + hl * geo.q_head_bytes;
         if (newseg) {
             segS = i - d.j;
             seg_bad = false;
-            if constexpr (MMA)
+            if constexpr (KV8)
+                math.begin(static_cast<const uint8_t *>(p.q) +
+                               ((int64_t)d.b * Hq + (int64_t)(d.hg * hpc + hl) * G) * D * 2,
+                           lane, p.scale_log2);
+            else if constexpr (MMA)
                 math.begin(qslot, lane);
             else
                 math.begin(qslot, lane, p.scale_log2);
@@ -1696,15 +1903,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             else
                 math.tile(kreg, vreg, hline, d.n, scores, geo, lane);
         }
-        // the stage may be refilled: order this warp's shared-memory accesses
-        // before the producer's next TMA into it, then release it
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0)
-            ptx::mbar_arrive(empty0 + 8u * s);
+        const int last = min(segS + d.ns, R1) - 1;   // the segment's last tile in the range
+        // (FP8) the warp handing its partial state over at a segment end keeps
+        // its stage: the state goes through the stage's lines of its head
+        const bool hand_over = SUBS > 1 && i + SUBS > last && i != last;
+        if (!hand_over) {
+            // the stage may be refilled: order this warp's shared-memory
+            // accesses before the producer's next TMA into it, then release it
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                ptx::mbar_arrive(empty0 + 8u * s);
+        }
 
-        // ---- end of a segment (or of this CTA's range)
-        if (d.j == d.ns - 1 || i == R1 - 1) {
+        // ---- end of this warp's share of a segment (or of this CTA's range)
+        if (i + SUBS > last) {
+            if constexpr (SUBS > 1) {
+                // Two warps per head: the one holding the segment's last tile
+                // in the range completes it; the other hands it its partial
+                // state (bounded waits).
+                float *st = reinterpret_cast<float *>(xarea + hl * exchange_bytes(D));
+                const uint32_t xfull = ptx::smem_u32(st) + kXBars, xfree = xfull + 8u;
+                auto head_lines = [&](int stage, int v) {
+                    return reinterpret_cast<float *>(sgen + stage * geo.stage_bytes +
+                                                     v * geo.kv_bytes + hline * 128);
+                };
+                if (hand_over) {
+                    if (xc > 0 &&
+                        !ptx::mbar_wait_bounded(xfree, (uint32_t)((xc - 1) & 1), p.wait_ns)) {
+                        if (lane == 0)
+                            report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+                        timed_out = true;
+                        lost = i;
+                        break;
+                    }
+                    __syncwarp();
+                    math.save(head_lines(s, 0), head_lines(s, 1), st, seg_bad, lane);
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0)
+                        ptx::mbar_arrive(xfull);
+                    ++xc;
+                    continue;
+                }
+                if (last - 1 >= max(segS, R0)) {
+                    if (!ptx::mbar_wait_bounded(xfull, (uint32_t)(xc & 1), p.wait_ns)) {
+                        if (lane == 0)
+                            report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+                        timed_out = true;
+                        lost = i;
+                        break;
+                    }
+                    // the other warp's last tile of the segment is last - 1
+                    const int sh = (last - 1 - R0) % spw;
+                    seg_bad |= math.absorb(head_lines(sh, 0), head_lines(sh, 1), st, lane);
+                    // its stage may be refilled now (released on its behalf)
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::mbar_arrive(empty0 + 8u * sh);
+                        ptx::mbar_arrive(xfree);
+                    }
+                    ++xc;
+                }
+            }
             math.finish();
             const int segE = segS + d.ns;
             const bool complete = segS >= R0 && segE <= R1;
@@ -1803,11 +2065,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.mode == 0) {
         // every consumer warp is past its last stage (and with it every copy
         // into the ring has landed): the ring is free scratch for the merges
-        asm volatile("bar.sync 1, %0;" ::"r"(32 * hpc) : "memory");
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * hpc * SUBS) : "memory");
         if (timed_out)
             return;
         float *buf = reinterpret_cast<float *>(
-            sgen + (int64_t)hl * ((int64_t)stages_bytes / hpc & ~(int64_t)15));
+            sgen + (int64_t)warp * ((int64_t)stages_bytes / (hpc * SUBS) & ~(int64_t)15));
         auto merge = [&](int S0, int N0, int B0, int HG0) {
             const int x0 = cta_of(S0, C, total);
             const int np = cta_of(S0 + N0 - 1, C, total) - x0 + 1;

@@ -67,11 +67,24 @@ template <typename T, int D, int G, bool MMA, bool TR16, bool KV8 = false>
 pa_status decode_one(DecodeLaunch &L, int *grid, bool launch)
 {
     auto fn = &decode_kernel<T, D, G, MMA, TR16, KV8>;
-    const int threads = 32 * (L.p.geo.hpc + 1);
+    const int threads = KV8 ? kThreads8 : 32 * (L.p.geo.hpc + 1);
     int cap = 0;
     pa_status st = grid_capacity(reinterpret_cast<const void *>(fn), threads, L.smem_bytes, &cap);
     if (st != PA_OK)
         return st;
+    if constexpr (KV8) {
+        // the kernel moves registers from its producer warpgroup to its
+        // consumers; that needs the launch to hold the registers it assumes
+        static int regs = -1;
+        if (regs < 0) {
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess)
+                return PA_ERR_CUDA;
+            regs = fa.numRegs;
+        }
+        if (regs != kRegsLaunch8)
+            return PA_ERR_UNSUPPORTED;
+    }
     if (!launch) {
         *grid = cap;
         return PA_OK;
