@@ -46,7 +46,8 @@
  *     kernels read context_lens, block_tables and the K/V pool rows of
  *     cached tokens other than each sequence's last one before it has
  *     completed (the query, the last rows, the outputs and the workspace
- *     after): a kernel ahead of them that allows an early start
+ *     after; the query rows are only prefetched into L2 before, which reads
+ *     no value): a kernel ahead of them that allows an early start
  *     (griddepcontrol.launch_dependents) must not write those arrays or
  *     rows.  pa_reshape_and_cache, which stores exactly each sequence's
  *     last row, is such a kernel and is safe; kernels that do not allow an

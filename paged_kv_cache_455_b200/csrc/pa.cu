@@ -1049,13 +1049,13 @@ static pa_status decode_entry(void *out, const void *query, const void *k_pool,
         (int64_t)num_seqs * p.head_groups * (round_up(std::max(max_context_len, 1), 16) / 16);
     grid = (int)std::min<int64_t>(grid, tiles_up);
     const size_t need = stream_k_bytes(num_seqs, num_kv_heads, group, head_dim, grid);
-    // a merge keeps its pieces' stats and weights in a warp's share of the
-    // stage ring
+    // a merge keeps its pieces' stats and weights, and two copy buffers of
+    // piece accumulators, in a warp's share of the stage ring
     const int64_t ring_share =
-        (int64_t)p.geo.spw * p.geo.stage_bytes / (p.geo.hpc * (kv8 ? pa::kSubs8 : 1)) & ~(int64_t)15;
+        (int64_t)p.geo.spw * p.geo.stage_bytes / (p.geo.hpc * (kv8 ? pa::kSubs8 : 1)) & ~(int64_t)127;
     const bool stream_k = workspace != nullptr && workspace_bytes >= need &&
                           aligned16(workspace) &&
-                          pa::merge_scratch_bytes(group, grid) <= ring_share;
+                          pa::merge_scratch_bytes(group, head_dim, grid) <= ring_share;
     if (stream_k) {
         p.mode = 0;
         p.slot_floats = (int)slot_floats(group, head_dim);

@@ -445,6 +445,17 @@ __device__ __forceinline__ uint32_t tile_addr(uint32_t reg, int hline, int t, in
         return kv_addr(reg, hline, t, u, g);
 }
 
+// Stores unit u (four accumulator elements) of a published piece whose
+// elements have type P: fp32 as they are, bf16 rounded to nearest even.
+template <typename P>
+__device__ __forceinline__ void put_unit(void *ps, int u, float x, float y, float z, float w)
+{
+    if constexpr (sizeof(P) == 2)
+        reinterpret_cast<uint2 *>(ps)[u] = make_uint2(ptx::pack_bf16x2(x, y), ptx::pack_bf16x2(z, w));
+    else
+        reinterpret_cast<float4 *>(ps)[u] = make_float4(x, y, z, w);
+}
+
 // =====================================================================
 // Tile math, bf16 tensor cores (warp-level MMA)
 //
@@ -574,14 +585,15 @@ struct MmaMath {
     static constexpr int CU = (G + 1) / 2;
     static constexpr int kUnits = KS * 8 * CU;
 
-    __device__ __forceinline__ void publish(float *ps, int lane) const
+    template <typename P>
+    __device__ __forceinline__ void publish(void *ps, int lane) const
     {
         const int r = lane >> 2, c = lane & 3;
         if (c < CU) {
-            float4 *p4 = reinterpret_cast<float4 *>(ps) + r * CU + c;
 #pragma unroll
             for (int k = 0; k < KS; ++k)
-                p4[k * 8 * CU] = make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
+                put_unit<P>(ps, k * 8 * CU + r * CU + c, acc[k][0], acc[k][1], acc[k][2],
+                            acc[k][3]);
         }
     }
 
@@ -938,14 +950,15 @@ struct MmaMath8 {
     static constexpr int CU = (G + 1) / 2;
     static constexpr int kUnits = KS * 8 * CU;
 
-    __device__ __forceinline__ void publish(float *ps, int lane) const
+    template <typename P>
+    __device__ __forceinline__ void publish(void *ps, int lane) const
     {
         const int r = lane >> 2, c = lane & 3;
         if (c < CU) {
-            float4 *p4 = reinterpret_cast<float4 *>(ps) + r * CU + c;
 #pragma unroll
             for (int k = 0; k < KS; ++k)
-                p4[k * 8 * CU] = make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
+                put_unit<P>(ps, k * 8 * CU + r * CU + c, acc[k][0], acc[k][1], acc[k][2],
+                            acc[k][3]);
         }
     }
 
@@ -1183,7 +1196,8 @@ struct SimtMath {
     // sum per head (publish_stats).
     static constexpr int kUnits = G * D / 4;
 
-    __device__ __forceinline__ void publish(float *ps, int lane) const
+    template <typename P>
+    __device__ __forceinline__ void publish(void *ps, int lane) const
     {
         const int li = lane % LPR;
         if (lane / LPR != 0)
@@ -1194,9 +1208,9 @@ struct SimtMath {
             for (int c = 0; c < UPL; ++c)
 #pragma unroll
                 for (int q = 0; q < VEC / 4; ++q)
-                    *reinterpret_cast<float4 *>(ps + g * D + (c * LPR + li) * VEC + 4 * q) =
-                        make_float4(acc[g][c * VEC + 4 * q], acc[g][c * VEC + 4 * q + 1],
-                                    acc[g][c * VEC + 4 * q + 2], acc[g][c * VEC + 4 * q + 3]);
+                    put_unit<P>(ps, (g * D + (c * LPR + li) * VEC + 4 * q) / 4,
+                                acc[g][c * VEC + 4 * q], acc[g][c * VEC + 4 * q + 1],
+                                acc[g][c * VEC + 4 * q + 2], acc[g][c * VEC + 4 * q + 3]);
     }
 
     __device__ __forceinline__ void publish_stats(float *st, int lane) const
@@ -1269,7 +1283,11 @@ __host__ __device__ constexpr int exchange_bytes(int D)
     return (32 * 5 * 4 + 16 + 127) / 128 * 128 + 0 * D;
 }
 
-// Offset of the exchange areas from the end of the stages.
+// Two mbarriers per consumer warp for the bulk copies of its merges.
+constexpr int kMergeBarBytes = 16 * kMaxHpc * kSubs8;
+
+// Offset of the merge barriers (then the exchange areas) from the end of
+// the stages.
 __host__ __device__ constexpr int exchange_off(int G)
 {
     return (48 * kMaxSpw + kMaxHpc * kTile * G * 4 + 4 * (kMaxChunks + 1) + 127) / 128 * 128;
@@ -1281,7 +1299,7 @@ __host__ __device__ constexpr int exchange_off(int G)
 // (FP8 cache) the heads' exchange areas.
 __host__ __device__ constexpr int decode_smem_fixed(int G, int D = 0, bool kv8 = false)
 {
-    return 1024 + exchange_off(G) + (kv8 ? kMaxHpc * exchange_bytes(D) : 0);
+    return 1024 + exchange_off(G) + kMergeBarBytes + (kv8 ? kMaxHpc * exchange_bytes(D) : 0);
 }
 
 // Tile metadata the producer warp hands to the consumer warps with a stage.
@@ -1317,14 +1335,26 @@ __device__ __forceinline__ unsigned long long *counter_of(const DecodeParams &p,
 // group to an even one).
 __host__ __device__ constexpr int piece_stats_off(int D, int G) { return 2 * D * ((G + 1) / 2); }
 
+// The same, in floats, for a piece whose accumulator elements have `bytes`
+// bytes (4: fp32, 2: bf16); the stats follow the accumulator directly.
+__host__ __device__ constexpr int piece_stats_off(int D, int G, int bytes)
+{
+    return piece_stats_off(D, G) * bytes / 4;
+}
+
 // A published piece's stats (max [G], sum [G], bad mark) in float4 units.
 __host__ __device__ constexpr int stats_units(int G) { return (2 * G + 1 + 3) / 4; }
 
 // Bytes of per-warp shared scratch a merge of a cut segment of up to np
-// pieces needs: np stats blocks and np x G weights.
-__host__ __device__ constexpr int64_t merge_scratch_bytes(int G, int64_t np)
+// pieces needs: np stats blocks and np x G weights (rounded to 128 bytes),
+// then two copy buffers of at least one piece's accumulator each.
+__host__ __device__ constexpr int64_t merge_header_bytes(int G, int64_t np)
 {
-    return 4 * (4 * np * stats_units(G) + np * G);
+    return (4 * (4 * np * stats_units(G) + np * G) + 127) / 128 * 128;
+}
+__host__ __device__ constexpr int64_t merge_scratch_bytes(int G, int D, int64_t np)
+{
+    return merge_header_bytes(G, np) + 2 * 4 * (int64_t)piece_stats_off(D, G);
 }
 
 // Counts one more arrival at a cut segment's counter for this call and
@@ -1381,18 +1411,17 @@ __device__ __forceinline__ float pick(const float (&v)[G], int g)
     return r;
 }
 
-// Per-head maxima, sums and weights of a cut segment's pieces from the
-// stats block `st` ([np][4 SU] floats in shared memory, or NULL to read
-// piece `lane` of `np <= 32` from `gst`), by a whole warp: lane i handles
+// Per-head maxima, sums and weights of a cut segment's pieces from their
+// stats in shared memory (piece i's max [G] and sum [G] at st[i * stride]),
+// by a whole warp: lane i handles
 // pieces i, i + 32, ...; the butterflies run in a fixed order, so the result
 // does not depend on timing.  Leaves w_i = 2^(m_i - M) / L * out_scale for
 // the pieces a lane handles in wl[G] (first piece only) and, with `w`, for
 // every piece in w[np][G].
 template <int G>
-__device__ __forceinline__ void piece_weights(const float *st, int np, float out_scale, float *w,
-                                              float (&wl)[G], int lane)
+__device__ __forceinline__ void piece_weights(const float *st, int stride, int np, float out_scale,
+                                              float *w, float (&wl)[G], int lane)
 {
-    constexpr int SU = stats_units(G);
     float M[G], L[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -1402,7 +1431,7 @@ __device__ __forceinline__ void piece_weights(const float *st, int np, float out
     for (int i = lane; i < np; i += 32)
 #pragma unroll
         for (int g = 0; g < G; ++g)
-            M[g] = fmaxf(M[g], st[i * 4 * SU + g]);
+            M[g] = fmaxf(M[g], st[i * stride + g]);
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
@@ -1411,9 +1440,9 @@ __device__ __forceinline__ void piece_weights(const float *st, int np, float out
     for (int i = lane; i < np; i += 32)
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const float mi = st[i * 4 * SU + g];
+            const float mi = st[i * stride + g];
             if (M[g] != -INFINITY && mi != -INFINITY)
-                L[g] = fmaf(st[i * 4 * SU + G + g], ptx::ex2(mi - M[g]), L[g]);
+                L[g] = fmaf(st[i * stride + G + g], ptx::ex2(mi - M[g]), L[g]);
         }
 #pragma unroll
     for (int g = 0; g < G; ++g)
@@ -1426,7 +1455,7 @@ __device__ __forceinline__ void piece_weights(const float *st, int np, float out
     for (int i = lane; i < np; i += 32)
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const float mi = st[i * 4 * SU + g];
+            const float mi = st[i * stride + g];
             // out_scale (1 unless the cache is FP8) multiplies the weights exactly
             const float wi = (mi == -INFINITY || !(L[g] > 0.f))
                                  ? 0.f
@@ -1444,36 +1473,39 @@ __device__ __forceinline__ void piece_weights(const float *st, int np, float out
 // partial softmax states (max m_i, sum l_i, accumulator a_i, log2 domain):
 //     M = max_i m_i,   L = sum_i l_i 2^(m_i - M),   o = sum_i a_i 2^(m_i - M) / L,
 // the identity the split-K reduction uses.  The pieces' stats go through
-// shared memory (`scratch`, 16 np (SU + G) bytes at least); the units come
-// straight into registers through L2 (lane e holds units e, e + 32, ...),
-// four pieces in flight at a time, and the weighted sums run in piece order,
-// so that the result does not depend on timing.
+// shared memory (`scratch`, `cap` bytes, at least merge_scratch_bytes); the
+// accumulators come into two shared buffers by bulk copies (H pieces per
+// copy, the next copy in flight while a buffer is summed; two mbarriers at
+// `bars`, their phase parities in `phase`), and the weighted sums run in
+// piece order, so that the result does not depend on timing.
 template <typename T, int D, int G, typename Math>
 __device__ __forceinline__ void merge_last(const DecodeParams &p, int x0, int np, int64_t bh0,
-                                           int hl, float *scratch, int lane)
+                                           int hl, uint8_t *scratch, int cap, uint32_t bars,
+                                           uint32_t &phase, int lane)
 {
     constexpr int U = Math::kUnits;
     constexpr int UL = (U + 31) / 32;
-    constexpr int SO = piece_stats_off(D, G);
+    constexpr int SO = piece_stats_off(D, G, (int)sizeof(T));
+    constexpr int UB = SO * 4;   // bytes of a piece's accumulator region (U units, padded)
     constexpr int SU = stats_units(G);
     const int hpc = p.geo.hpc;
     T *out = static_cast<T *>(p.out) + bh0 * D;
-    float *stats = scratch;                 // [np][SU] float4
-    float *w = scratch + 4 * np * SU;       // [np][G]
+    float *stats = reinterpret_cast<float *>(scratch);   // [np][SU] float4
+    float *w = stats + 4 * np * SU;                      // [np][G]
+    constexpr int PB = UB + 16 * SU;   // a piece: accumulator, then its stats
+    // one copy of every whole piece when they all fit; otherwise the stats
+    // first, then the accumulators in batches of H, double buffered
+    const int whdr = (np * G * 4 + 127) & ~127;
+    const bool one_shot = whdr + np * PB <= cap;
+    uint8_t *bufs = one_shot ? scratch + whdr : scratch + merge_header_bytes(G, np);
+    if (one_shot)
+        w = reinterpret_cast<float *>(scratch);
+    const int H = one_shot ? np : max(1, min(np, (cap - (int)merge_header_bytes(G, np)) / (2 * UB)));
+    const int CB = one_shot ? PB : UB;   // bytes copied per piece
     auto src = [&](int i) {
         return p.wpart + (int64_t)piece_slot(x0 + i, i == 0, hpc, hl) * p.slot_floats;
     };
-    bool bad = false;
-    for (int i = lane; i < np; i += 32) {
-        const float4 *s4 = reinterpret_cast<const float4 *>(src(i) + SO);
-#pragma unroll
-        for (int u = 0; u < SU; ++u)
-            reinterpret_cast<float4 *>(stats)[i * SU + u] = __ldcg(s4 + u);
-        bad |= stats[i * 4 * SU + 2 * G] != 0.f;
-    }
-    if (__any_sync(kFull, bad)) {
-        if (lane == 0)
-            report(p.dev_status, PA_DEV_BAD_BLOCK);
+    auto zero_out = [&]() {
 #pragma unroll
         for (int t = 0; t < UL; ++t) {
             const int e = lane + 32 * t;
@@ -1487,36 +1519,123 @@ __device__ __forceinline__ void merge_last(const DecodeParams &p, int x0, int np
                 }
         }
         __syncwarp();
-        return;
-    }
+    };
+    // the copies read the pieces (published by generic stores, acquired by
+    // the arrival count) and overwrite shared memory this warp's generic
+    // accesses used before: order both before them
+    ptx::fence_proxy_async_all();
     __syncwarp();
+    const int nb = (np + H - 1) / H;
+    auto issue = [&](int bt) {
+        if (lane == 0) {
+            const int i0 = bt * H, n = min(H, np - i0);
+            const uint32_t bar = bars + 8u * (uint32_t)(bt & 1);
+            ptx::mbar_arrive_expect_tx(bar, (uint32_t)(n * CB));
+            for (int i = 0; i < n; ++i)
+                ptx::bulk_g2s(ptx::smem_u32(bufs + ((bt & 1) * H + i) * CB), src(i0 + i),
+                              (uint32_t)CB, bar);
+        }
+        __syncwarp();
+    };
+    bool bad = false;
     float wl[G];
-    piece_weights<G>(stats, np, p.out_scale, w, wl, lane);
-    __syncwarp();
+    if (one_shot) {
+        issue(0);
+        if (!ptx::mbar_wait_bounded(bars, phase & 1u, p.wait_ns)) {
+            phase ^= 1u;
+            if (lane == 0)
+                report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+            zero_out();
+            return;
+        }
+        phase ^= 1u;
+        const float *st0 = reinterpret_cast<const float *>(bufs + UB);
+        for (int i = lane; i < np; i += 32)
+            bad |= st0[i * (PB / 4) + 2 * G] != 0.f;
+        bad = __any_sync(kFull, bad);
+        if (!bad)
+            piece_weights<G>(st0, PB / 4, np, p.out_scale, w, wl, lane);
+        __syncwarp();
+    } else {
+        // the stats go first: they decide the weights, the copies only the sums
+        for (int i = lane; i < np; i += 32) {
+            const float4 *s4 = reinterpret_cast<const float4 *>(src(i) + SO);
+#pragma unroll
+            for (int u = 0; u < SU; ++u)
+                reinterpret_cast<float4 *>(stats)[i * SU + u] = __ldcg(s4 + u);
+            bad |= stats[i * 4 * SU + 2 * G] != 0.f;
+        }
+        bad = __any_sync(kFull, bad);
+        __syncwarp();
+        issue(0);
+        if (nb > 1)
+            issue(1);
+        if (!bad)
+            piece_weights<G>(stats, 4 * SU, np, p.out_scale, w, wl, lane);
+        __syncwarp();
+    }
     float o[UL][4];
 #pragma unroll
     for (int t = 0; t < UL; ++t)
         o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
-#pragma unroll 4
-    for (int i = 0; i < np; ++i) {
-        float wp[G];
+    for (int bt = 0; bt < nb; ++bt) {
+        const uint32_t bar = bars + 8u * (uint32_t)(bt & 1);
+        bool ok = true;
+        if (!one_shot) {
+            ok = ptx::mbar_wait_bounded(bar, (phase >> (bt & 1)) & 1u, p.wait_ns);
+            phase ^= 1u << (bt & 1);
+        }
+        if (!ok || bad) {
+            // let the other buffer's copy land (bounded) before leaving
+            if (!one_shot && bt + 1 < nb) {
+                ptx::mbar_wait_bounded(bars + 8u * (uint32_t)((bt + 1) & 1),
+                                       (phase >> ((bt + 1) & 1)) & 1u, p.wait_ns);
+                phase ^= 1u << ((bt + 1) & 1);
+            }
+            if (lane == 0)
+                report(p.dev_status, ok ? PA_DEV_BAD_BLOCK : PA_DEV_WAIT_TIMEOUT);
+            zero_out();
+            return;
+        }
+        const int i0 = bt * H, n = min(H, np - i0);
+        for (int i = 0; i < n; ++i) {
+            float wp[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-            wp[g] = w[i * G + g];
-        const float4 *src4 = reinterpret_cast<const float4 *>(src(i));
+            for (int g = 0; g < G; ++g)
+                wp[g] = w[(i0 + i) * G + g];
+            const uint8_t *bp = bufs + ((bt & 1) * H + i) * CB;
 #pragma unroll
-        for (int t = 0; t < UL; ++t) {
-            const int e = lane + 32 * t;
-            if (e < U) {
-                const float4 v = __ldcg(src4 + e);
-                const float vv[4] = {v.x, v.y, v.z, v.w};
+            for (int t = 0; t < UL; ++t) {
+                const int e = lane + 32 * t;
+                if (e < U) {
+                    float vv[4];
+                    if constexpr (sizeof(T) == 2) {
+                        const uint2 v = reinterpret_cast<const uint2 *>(bp)[e];
+                        vv[0] = ptx::bf16lo_to_f32(v.x);
+                        vv[1] = ptx::bf16hi_to_f32(v.x);
+                        vv[2] = ptx::bf16lo_to_f32(v.y);
+                        vv[3] = ptx::bf16hi_to_f32(v.y);
+                    } else {
+                        const float4 v = reinterpret_cast<const float4 *>(bp)[e];
+                        vv[0] = v.x;
+                        vv[1] = v.y;
+                        vv[2] = v.z;
+                        vv[3] = v.w;
+                    }
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    int g, d;
-                    Math::unit_coords(e, j, g, d);
-                    o[t][j] = fmaf(pick<G>(wp, g), vv[j], o[t][j]);
+                    for (int j = 0; j < 4; ++j) {
+                        int g, d;
+                        Math::unit_coords(e, j, g, d);
+                        o[t][j] = fmaf(pick<G>(wp, g), vv[j], o[t][j]);
+                    }
                 }
             }
+        }
+        if (bt + 2 < nb) {
+            // this buffer's generic reads come before the next copy into it
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            issue(bt + 2);
         }
     }
 #pragma unroll
@@ -1603,7 +1722,7 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
     constexpr int SUBS = KV8 ? kSubs8 : 1;   // consumer warps per KV head
 
     // 1024-byte aligned layout: [stages][full bars][empty bars][meta][score rows][chunk prefix]
-    // [exchange areas (FP8)]
+    // [merge barriers][exchange areas (FP8)]
     const uint32_t raw = ptx::smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     uint8_t *sgen = smem_raw + (sbase - raw);
@@ -1613,13 +1732,18 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
     StageMeta *meta = reinterpret_cast<StageMeta *>(sgen + stages_bytes + 16 * kMaxSpw);
     float *scores_all = reinterpret_cast<float *>(sgen + stages_bytes + 48 * kMaxSpw);
     int *cbase = reinterpret_cast<int *>(scores_all + kMaxHpc * kTile * G);
-    uint8_t *xarea = sgen + stages_bytes + exchange_off(G);
+    const uint32_t mbars0 = ptx::smem_u32(sgen + stages_bytes + exchange_off(G));
+    uint8_t *xarea = sgen + stages_bytes + exchange_off(G) + kMergeBarBytes;
     constexpr uint32_t kXBars = 32u * 5u * 4u;   // barriers' offset in an exchange area
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < spw; ++s) {
             ptx::mbar_init(full0 + 8u * s, 1);
             ptx::mbar_init(empty0 + 8u * s, hpc);
+        }
+        for (int w = 0; w < kMaxHpc * kSubs8; ++w) {
+            ptx::mbar_init(mbars0 + 16u * w, 1);
+            ptx::mbar_init(mbars0 + 16u * w + 8u, 1);
         }
         if constexpr (SUBS > 1) {
             for (int h = 0; h < hpc; ++h) {
@@ -1662,6 +1786,14 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
         fill_batch(bat0, win, R0, R1, p, cbase, lane);
         fill_batch(bat1, win, R0 + 32, R1, p, cbase, lane);
         int filled = 2;
+        // Brings the query rows of tile d's segment (this CTA's heads) into
+        // L2; no value is read.
+        auto prefetch_query = [&](const TileDesc &d) {
+            const uint8_t *qsrc = static_cast<const uint8_t *>(p.q) +
+                                  ((int64_t)d.b * Hq + (int64_t)d.h * hpc * G) * D * sizeof(T);
+            for (int off = lane * 128; off < hpc * geo.q_head_bytes; off += 32 * 128)
+                ptx::prefetch_l2(qsrc + off);
+        };
         // Fills ring position k with tile R0 + k (descriptor d): the
         // metadata, the expected bytes, and the K/V copies (kv) and/or the
         // segment's query rows (q).  False if the bounded wait for the stage
@@ -1729,12 +1861,8 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
                 // FP8 stages carry no query rows: the consumers read them
                 // from global memory when they start the segment; bring
                 // them into L2 now
-                if (q && (d.j == 0 || k == 0)) {
-                    const uint8_t *qsrc = static_cast<const uint8_t *>(p.q) +
-                                          ((int64_t)d.b * Hq + (int64_t)h0 * G) * D * 2;
-                    for (int off = lane * 128; off < hpc * geo.q_head_bytes; off += 32 * 128)
-                        ptx::prefetch_l2(qsrc + off);
-                }
+                if (q && (d.j == 0 || k == 0))
+                    prefetch_query(d);
             }
             __syncwarp();
             return true;
@@ -1744,12 +1872,16 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
         // sequence's last cached token: that row is the only one the cache
         // write ahead of this kernel stores.  Their query rows come after the
         // wait, as everything else.
+        // Their segments' query rows are prefetched into L2 meanwhile (no
+        // value is read before the wait; L2 keeps the latest writes).
         int early = 0;
         for (; early < min(spw, R1 - R0); ++early) {
             const TileDesc d = shfl_desc(bat0, early);
             if (d.t0 + d.n >= d.ctx)
                 break;
             issue(early, d, true, false);
+            if (d.j == 0 || early == 0)
+                prefetch_query(d);
         }
         // the query, the last rows and the outputs may be written or read by
         // the kernel ahead
@@ -1843,8 +1975,9 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
     int xc = 0;            // state exchanges so far between the head's two warps (FP8)
     // cut segments this warp merges (mode 0): one met at the start of the
     // range, one that runs past its end
-    int laterS = -1, laterN = 0, laterB = 0, laterHG = 0;
-    int firstS = -1, firstN = 0, firstB = 0, firstHG = 0;
+    // (its first CTA and piece count, sequence and head group)
+    int laterS = -1, laterX = 0, laterN = 0, laterB = 0, laterHG = 0;
+    int firstS = -1, firstX = 0, firstN = 0, firstB = 0, firstHG = 0;
 
     // this CTA's arrival counters start the call at (epoch, 0) unless an
     // arrival has already counted in them (see segment_arrive)
@@ -1976,10 +2109,12 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
                 const bool first = segS >= R0;
                 const int slot = piece_slot(blockIdx.x, first, hpc, hl);
                 float *ps = p.wpart + (int64_t)slot * p.slot_floats;
-                math.publish(ps, lane);
-                math.publish_stats(ps + piece_stats_off(D, G), lane);
+                // the accumulator in the output's type (bf16 rounds it once)
+                constexpr int SOT = piece_stats_off(D, G, (int)sizeof(T));
+                math.template publish<T>(ps, lane);
+                math.publish_stats(ps + SOT, lane);
                 if (lane == 0)
-                    ps[piece_stats_off(D, G) + 2 * G] = seg_bad ? 1.f : 0.f;
+                    ps[SOT + 2 * G] = seg_bad ? 1.f : 0.f;
                 // the warp barrier orders every lane's stores before lane 0's
                 // release (the counter update)
                 __syncwarp();
@@ -1999,12 +2134,14 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
                     continue;   // a later arrival merges the segment
                 if (first) {
                     firstS = segS;
-                    firstN = d.ns;
+                    firstX = x0;
+                    firstN = np;
                     firstB = d.b;
                     firstHG = d.hg;
                 } else {
                     laterS = segS;
-                    laterN = d.ns;
+                    laterX = x0;
+                    laterN = np;
                     laterB = d.b;
                     laterHG = d.hg;
                 }
@@ -2068,19 +2205,18 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
         asm volatile("bar.sync 1, %0;" ::"r"(32 * hpc * SUBS) : "memory");
         if (timed_out)
             return;
-        float *buf = reinterpret_cast<float *>(
-            sgen + (int64_t)warp * ((int64_t)stages_bytes / (hpc * SUBS) & ~(int64_t)15));
-        auto merge = [&](int S0, int N0, int B0, int HG0) {
-            const int x0 = cta_of(S0, C, total);
-            const int np = cta_of(S0 + N0 - 1, C, total) - x0 + 1;
+        const int cap = (int)((int64_t)stages_bytes / (hpc * SUBS) & ~(int64_t)127);
+        uint8_t *buf = sgen + (int64_t)warp * cap;
+        uint32_t mphase = 0;
+        auto merge = [&](int x0, int np, int B0, int HG0) {
             merge_last<T, D, G, Math>(p, x0, np,
                                       (int64_t)B0 * Hq + (int64_t)(HG0 * hpc + hl) * G, hl, buf,
-                                      lane);
+                                      cap, mbars0 + 16u * (uint32_t)warp, mphase, lane);
         };
         if (laterS >= 0)
-            merge(laterS, laterN, laterB, laterHG);
+            merge(laterX, laterN, laterB, laterHG);
         if (firstS >= 0)
-            merge(firstS, firstN, firstB, firstHG);
+            merge(firstX, firstN, firstB, firstHG);
     }
 }
 
