@@ -76,6 +76,7 @@ def attention_bytes(layout: W.BatchLayout, kv_elem: int = 0) -> int:
 
 # the sources each profiled kernel is built and launched from
 DECODE_SOURCES = ("pa.cu", "pa_inst_bf16.cu", "pa_kernels.cuh", "pa_launch.cuh", "pa_ptx.cuh")
+DECODE8_SOURCES = DECODE_SOURCES + ("pa_inst_fp8.cu",)
 PREFILL_SOURCES = ("pa.cu", "pa_inst_prefill.cu", "pa_launch.cuh", "pa_prefill.cuh",
                    "pa_prefill_tc.cuh", "pa_ptx.cuh")
 
@@ -321,7 +322,8 @@ def measure_decode(cfg: W.DecodeConfig, args, rank, world, device, dist, headlin
     tokens_per_s_layer = seqs_all / t_layer_s
     peak, peak_kind = measured_peak()
     achieved = bytes_layer / (attn_ms_mean * 1e-3) / 1e9
-    traffic = profiled_traffic(profile_summary(cfg.name + ("_fp8" if fp8 else "")))
+    traffic = profiled_traffic(profile_summary(cfg.name + ("_fp8" if fp8 else "")),
+                               DECODE8_SOURCES if fp8 else DECODE_SOURCES)
     if traffic is not None and length_scale != 1.0:
         traffic = None   # the committed capture is of the unscaled workload
 
