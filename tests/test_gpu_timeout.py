@@ -78,3 +78,51 @@ def test_a_wait_that_runs_out_sets_the_status_zeroes_its_outputs_and_leaves_the_
     got = out.double().cpu().numpy()
     assert np.isfinite(got).all()
     assert np.abs(got - ref).max() <= TOL
+
+
+def test_a_wait_that_runs_out_with_merges_inside_the_decode_kernel():
+    """Many sequences per CTA: cut segments are merged by their last arriving
+    piece inside the decode kernel (no merge pass).  CTA 1's range is lost
+    from its second tile on; every output is then exactly zero or matches
+    the oracle, some are zero, and the next call is exact."""
+    from paged_kv_cache_455_b200 import pa
+    lens = [3000 + 37 * i for i in range(48)]
+    q, kp, vp, tables, lens = _case(22, lens)
+    tab, cl = torch.from_numpy(tables).to(DEV), torch.from_numpy(lens).to(DEV)
+    ws = torch.empty(pa.pa_decode_workspace_bytes(len(lens), 16, 4, 256, int(lens.max())),
+                     dtype=torch.uint8, device=DEV)
+    ref = O.paged_attention(W.to_numpy_elems(q), W.to_numpy_elems(kp), W.to_numpy_elems(vp),
+                            tables, lens, 1.0 / 16.0, "bf16")
+
+    def run():
+        out = torch.full_like(q, float("nan"))
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        launches = pa.launch_count()
+        pa.pa_decode_attention(out, q, kp, vp, tab, cl, int(lens.max()), 1.0 / 16.0, ws, status)
+        torch.cuda.synchronize()
+        assert pa.launch_count() - launches == 1, "expected no merge pass"
+        return out, int(status.item())
+
+    pa.testing_set_wait_limit_ns(2_000_000)
+    pa.testing_withhold_copy(1)
+    try:
+        out, status = run()
+    finally:
+        pa.testing_withhold_copy(-1)
+        pa.testing_set_wait_limit_ns(0)
+    assert status & pa.PA_DEV_WAIT_TIMEOUT
+    assert status & ~pa.PA_DEV_WAIT_TIMEOUT == 0
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    heads = got.reshape(len(lens), 4, -1)          # per (sequence, KV head group of 4 heads)
+    want = ref.reshape(len(lens), 4, -1)
+    zero = (heads == 0).all(axis=2)
+    exact = np.abs(heads - want).max(axis=2) <= TOL
+    assert (zero | exact).all(), "an output is neither zeros nor the oracle's"
+    assert zero.any(), "the lost range zeroed nothing"
+
+    out, status = run()
+    assert status == 0
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= TOL
