@@ -1290,7 +1290,7 @@ constexpr int kMergeBarBytes = 16 * kMaxHpc * kSubs8;
 // the stages.
 __host__ __device__ constexpr int exchange_off(int G)
 {
-    return (48 * kMaxSpw + kMaxHpc * kTile * G * 4 + 4 * (kMaxChunks + 1) + 127) / 128 * 128;
+    return (48 * kMaxSpw + kMaxHpc * kTile * G * 4 + 4 * (kMaxChunks + 1) + 16 + 127) / 128 * 128;
 }
 
 // Bytes of the decode kernel's dynamic shared memory besides the stages:
@@ -1732,11 +1732,14 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
     StageMeta *meta = reinterpret_cast<StageMeta *>(sgen + stages_bytes + 16 * kMaxSpw);
     float *scores_all = reinterpret_cast<float *>(sgen + stages_bytes + 48 * kMaxSpw);
     int *cbase = reinterpret_cast<int *>(scores_all + kMaxHpc * kTile * G);
+    // set when a consumer warp of this CTA gave up waiting
+    volatile int *cta_lost = cbase + kMaxChunks + 1;
     const uint32_t mbars0 = ptx::smem_u32(sgen + stages_bytes + exchange_off(G));
     uint8_t *xarea = sgen + stages_bytes + exchange_off(G) + kMergeBarBytes;
     constexpr uint32_t kXBars = 32u * 5u * 4u;   // barriers' offset in an exchange area
 
     if (threadIdx.x == 0) {
+        *cta_lost = 0;
         for (int s = 0; s < spw; ++s) {
             ptx::mbar_init(full0 + 8u * s, 1);
             ptx::mbar_init(empty0 + 8u * s, hpc);
@@ -2178,16 +2181,16 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
         }
     }
 
+    auto zero_segment = [&](int b, int hg) {
+        T *o = static_cast<T *>(p.out) + ((int64_t)b * Hq + (int64_t)(hg * hpc + hl) * G) * D;
+        for (int e = lane; e < G * D; e += 32)
+            store_out<T>(o + e, 0.f);
+    };
     if (timed_out) {
         // the rest of the range is lost: zero this warp's head of every
         // segment from the lost tile on (their pieces here are never counted
         // in, so no merge overwrites the zeros), and of the segments this
         // warp was to merge; the CTA's other warps do the same for their heads
-        auto zero_segment = [&](int b, int hg) {
-            T *o = static_cast<T *>(p.out) + ((int64_t)b * Hq + (int64_t)(hg * hpc + hl) * G) * D;
-            for (int e = lane; e < G * D; e += 32)
-                store_out<T>(o + e, 0.f);
-        };
         for (int g = lost; g < R1;) {
             int b, hg, j, ns;
             tile_segment(g, p, cbase, lane, b, hg, j, ns);
@@ -2198,6 +2201,8 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
             zero_segment(laterB, laterHG);
         if (firstS >= 0)
             zero_segment(firstB, firstHG);
+        if (lane == 0)
+            *cta_lost = 1;
     }
     if (p.mode == 0) {
         // every consumer warp is past its last stage (and with it every copy
@@ -2205,6 +2210,20 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
         asm volatile("bar.sync 1, %0;" ::"r"(32 * hpc * SUBS) : "memory");
         if (timed_out)
             return;
+        if (*cta_lost != 0) {
+            // another warp of this CTA gave up: copies into the ring may still
+            // be landing, so it is no scratch; the segments this warp was to
+            // merge get zeros, as lost ones
+            if (laterS >= 0 || firstS >= 0) {
+                if (lane == 0)
+                    report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+                if (laterS >= 0)
+                    zero_segment(laterB, laterHG);
+                if (firstS >= 0)
+                    zero_segment(firstB, firstHG);
+            }
+            return;
+        }
         const int cap = (int)((int64_t)stages_bytes / (hpc * SUBS) & ~(int64_t)127);
         uint8_t *buf = sgen + (int64_t)warp * cap;
         uint32_t mphase = 0;

@@ -126,3 +126,69 @@ def test_a_wait_that_runs_out_with_merges_inside_the_decode_kernel():
     got = out.double().cpu().numpy()
     assert np.isfinite(got).all()
     assert np.abs(got - ref).max() <= TOL
+
+
+def test_a_wait_that_runs_out_over_an_fp8_cache():
+    """Two consumer warps per KV head (E4M3 cache): the withheld tile is the
+    second warp's first; its partner's hand-off waits run out as well.  The
+    long sequence is zeros, the short one exact, the next call exact."""
+    import dataclasses
+    from paged_kv_cache_455_b200 import pa
+    base = W.CONFIGS["qwen"]
+    lens = np.array([8192, 100], np.int32)
+    bs = 16
+    cfg = dataclasses.replace(base, num_seqs=2)
+    rng = np.random.default_rng(23)
+    need = -(-lens // bs)
+    nb = int(need.sum()) + 8
+    perm = rng.permutation(nb)
+    tables = np.full((2, int(need.max())), -1, np.int32)
+    pos = 0
+    for b in range(2):
+        tables[b, :need[b]] = perm[pos:pos + need[b]]
+        pos += need[b]
+    slots = np.array([tables[b, (n - 1) // bs] * bs + (n - 1) % bs for b, n in enumerate(lens)],
+                     np.int64)
+    layout = W.BatchLayout(cfg, lens, tables, slots, nb)
+    (layer,) = W.make_layers_fp8(layout, DEV, layers=1)
+    s = W.compact_sample(layout, layer, np.arange(2))
+    tab, cl, sl = W.device_metadata(layout, DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pa.pa_reshape_and_cache_fp8(layer.key, layer.value, layer.k_pool, layer.v_pool, sl,
+                                W.FP8_SCALE, W.FP8_SCALE, status)
+    k_ref, v_ref = O.reshape_and_cache_fp8_np(s["key"], s["value"], s["k_pool"], s["v_pool"],
+                                              s["slot_mapping"], W.FP8_SCALE, W.FP8_SCALE)
+    ref = O.paged_attention_fp8_np(s["query"], k_ref, v_ref, s["block_tables"],
+                                   s["context_lens"], cfg.scale, W.FP8_SCALE, W.FP8_SCALE)
+    ws = torch.empty(pa.pa_decode_workspace_bytes(2, 16, 4, 256, 8192), dtype=torch.uint8,
+                     device=DEV)
+
+    def run():
+        out = torch.full_like(layer.query, float("nan"))
+        st = torch.zeros(1, dtype=torch.int32, device=DEV)
+        pa.pa_decode_attention_fp8(out, layer.query, layer.k_pool, layer.v_pool, tab, cl, 8192,
+                                   cfg.scale, W.FP8_SCALE, W.FP8_SCALE, ws, st)
+        torch.cuda.synchronize()
+        return out, int(st.item())
+
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    pa.testing_set_wait_limit_ns(2_000_000)
+    pa.testing_withhold_copy(1)
+    try:
+        out, st = run()
+    finally:
+        pa.testing_withhold_copy(-1)
+        pa.testing_set_wait_limit_ns(0)
+    assert st & pa.PA_DEV_WAIT_TIMEOUT
+    assert st & ~pa.PA_DEV_WAIT_TIMEOUT == 0
+    assert (out[0].float() == 0).all(), "a sequence whose work was lost must be zeros"
+    got1 = out[1].double().cpu().numpy()
+    assert np.isfinite(got1).all()
+    assert np.abs(got1 - ref[1]).max() <= TOL
+
+    out, st = run()
+    assert st == 0
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= TOL
