@@ -382,11 +382,14 @@ bool make_geo(TileGeo &g, int D, int es, int es_q, int bs, int group, int hpc, i
     g.head_lines = nch * g.tr;
     g.box_stride = (int)round_up((int64_t)hpc * g.head_lines * 128, 1024);
     g.kv_bytes = g.bpt * g.box_stride;
+    // over an E4M3 cache a stage holds two consecutive tiles of a segment
+    // (64 KB at d = 256, as one bf16 tile)
+    g.tps = es == 1 ? 2 : 1;
     g.q_head_bytes = group * D * es_q;
     // an E4M3 cache's stages carry no query rows (its consumer warps read
     // them from global memory)
     g.q_bytes = es == 1 ? 0 : hpc * g.q_head_bytes;
-    g.q_off = 2 * g.kv_bytes;
+    g.q_off = 2 * g.tps * g.kv_bytes;
     g.stage_bytes = (int)round_up((int64_t)g.q_off + g.q_bytes, 1024);
     g.box_tx = hpc * g.tr * rowb;
     const int fixed = pa::decode_smem_fixed(group, D, es == 1);   // es 1: an E4M3 cache

@@ -87,7 +87,8 @@ struct TileGeo {
     int hpc;           // KV heads per CTA tile (= consumer warps)
     int head_lines;    // 128-byte lines per head in a box = nch * tr
     int box_stride;    // bytes between boxes
-    int kv_bytes;      // bytes of a K (or V) region
+    int kv_bytes;      // bytes of one tile's K (or V) region
+    int tps;           // tiles per stage: 1, or 2 over an FP8 cache (K of both, then V of both)
     int q_off;         // offset of the query slot in a stage
     int stage_bytes;   // K + V + query, multiple of 1024
     int spw;           // stages in the ring
@@ -105,7 +106,7 @@ struct DecodeParams {
     float *max_logits;       // [B, Hq, max_parts]
     float *exp_sums;         // [B, Hq, max_parts]
     float *wpart;            // mode 0: two partial slots per CTA and head
-    unsigned long long *counters;  // mode 0: arrivals per cut segment (owner CTA, head), a line each
+    unsigned long long *counters;  // mode 0: arrivals per cut segment (its first CTA, head), a line each
     int32_t *dev_status;
     int64_t num_blocks;
     int num_seqs;
@@ -1290,7 +1291,7 @@ constexpr int kMergeBarBytes = 16 * kMaxHpc * kSubs8;
 // the stages.
 __host__ __device__ constexpr int exchange_off(int G)
 {
-    return (48 * kMaxSpw + kMaxHpc * kTile * G * 4 + 4 * (kMaxChunks + 1) + 16 + 127) / 128 * 128;
+    return (64 * kMaxSpw + kMaxHpc * kTile * G * 4 + 4 * (kMaxChunks + 1) + 16 + 127) / 128 * 128;
 }
 
 // Bytes of the decode kernel's dynamic shared memory besides the stages:
@@ -1304,7 +1305,11 @@ __host__ __device__ constexpr int decode_smem_fixed(int G, int D = 0, bool kv8 =
 
 // Tile metadata the producer warp hands to the consumer warps with a stage.
 struct StageMeta {
-    int b, hg, part, j, ns, n, ctx, bad;
+    int b, hg, part, j, ns, n, ctx, bad;   // of the stage's first tile (bad: either tile)
+    int k;                                 // the first tile's offset in the CTA's range
+    int nt;                                // tiles in the stage (1 or 2, same segment)
+    int n1;                                // tokens of the second tile
+    int end;                               // no tiles: the range is done (FP8 ring)
 };
 
 // Index of the CTA whose range [R(x), R(x + 1)), R(x) = x T / C, holds tile t.
@@ -1730,7 +1735,7 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
     const uint32_t full0 = sbase + (uint32_t)stages_bytes;
     const uint32_t empty0 = full0 + 8u * kMaxSpw;
     StageMeta *meta = reinterpret_cast<StageMeta *>(sgen + stages_bytes + 16 * kMaxSpw);
-    float *scores_all = reinterpret_cast<float *>(sgen + stages_bytes + 48 * kMaxSpw);
+    float *scores_all = reinterpret_cast<float *>(sgen + stages_bytes + 64 * kMaxSpw);
     int *cbase = reinterpret_cast<int *>(scores_all + kMaxHpc * kTile * G);
     // set when a consumer warp of this CTA gave up waiting
     volatile int *cta_lost = cbase + kMaxChunks + 1;
@@ -1840,6 +1845,10 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
                 m.n = d.n;
                 m.ctx = d.ctx;
                 m.bad = bad ? 1 : 0;
+                m.k = k;
+                m.nt = 1;
+                m.n1 = 0;
+                m.end = 0;
                 meta[s] = m;
                 // release: consumers see the metadata once the phase completes
                 ptx::mbar_arrive_expect_tx(bar, (uint32_t)tx);
@@ -1916,12 +1925,188 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
             }
         }
     };
+    // ============================================ producer warp (FP8 cache)
+    // A stage holds two consecutive tiles of one segment when the range has
+    // them (tile k pairs with k + 1 if both lie in the same segment inside
+    // the range), else one; the consumer warps of a head take alternate
+    // stages.  After the last stage come SUBS end stages (no tiles), one per
+    // consumer warp of a head.
+    auto producer8 = [&]() {
+        if (R0 >= R1)
+            return;
+        ptx::prefetch_tensormap(&tmap_k);
+        ptx::prefetch_tensormap(&tmap_v);
+        const uint64_t policy = ptx::policy_evict_first();
+        SeqWindow win;
+        {
+            const int c = chunk_of(cbase, (p.num_seqs + 31) >> 5, R0);
+            window_load(win, c * 32, cbase[c], p, lane);
+        }
+        TileDesc bat0, bat1;
+        fill_batch(bat0, win, R0, R1, p, cbase, lane);
+        fill_batch(bat1, win, R0 + 32, R1, p, cbase, lane);
+        int loaded = 1;   // batches 0 and 1 are in bat0, bat1
+        // descriptor of tile R0 + k (whole warp; k only grows, by 1 or 2)
+        auto desc = [&](int k) -> TileDesc {
+            const int bt = k >> 5;
+            if (bt > loaded) {
+                // batch bt replaces batch bt - 2, whose tiles are all issued
+                if (bt & 1)
+                    fill_batch(bat1, win, R0 + 32 * bt, R1, p, cbase, lane);
+                else
+                    fill_batch(bat0, win, R0 + 32 * bt, R1, p, cbase, lane);
+                loaded = bt;
+            }
+            return (bt & 1) ? shfl_desc(bat1, k & 31) : shfl_desc(bat0, k & 31);
+        };
+        auto prefetch_query = [&](const TileDesc &d) {
+            const uint8_t *qsrc = static_cast<const uint8_t *>(p.q) +
+                                  ((int64_t)d.b * Hq + (int64_t)d.h * hpc * G) * D * sizeof(T);
+            for (int off = lane * 128; off < hpc * geo.q_head_bytes; off += 32 * 128)
+                ptx::prefetch_l2(qsrc + off);
+        };
+        auto tile_ok = [&](const TileDesc &d, int bx) {
+            return d.phys[bx] >= 0 && (int64_t)d.phys[bx] < p.num_blocks;
+        };
+        // Fills stage q with tiles R0 + k (d0) and, when `pair`, R0 + k + 1
+        // (d1).  False if the bounded wait for the stage ran out.
+        auto issue = [&](int q, int k, const TileDesc &d0, bool pair,
+                         const TileDesc &d1) -> bool {
+            const int s = q % spw;
+            const uint32_t bar = full0 + 8u * s;
+            if (q >= spw &&
+                !ptx::mbar_wait_bounded(empty0 + 8u * s, (uint32_t)(((q / spw) - 1) & 1),
+                                        p.wait_ns)) {
+                if (lane == 0)
+                    report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+                return false;
+            }
+            const uint32_t stage = sbase + (uint32_t)(s * geo.stage_bytes);
+            // test hook: the copies of this CTA's second stage are not issued,
+            // so the stage never completes and the bounded waits run out
+            const bool withhold = (int)blockIdx.x == p.withhold_cta && q == 1;
+            const int h0 = d0.h * hpc;
+            if (lane == 0) {
+                int tx = 0;
+                bool bad = false;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const TileDesc &d = t ? d1 : d0;
+                    if (t == 1 && !pair)
+                        continue;
+#pragma unroll
+                    for (int bx = 0; bx < 4; ++bx) {
+                        if (bx < geo.bpt && bx * geo.tr < d.n) {
+                            if (!tile_ok(d, bx))
+                                bad = true;
+                            else
+                                tx += 2 * geo.box_tx;
+                        }
+                    }
+                }
+                StageMeta m;
+                m.b = d0.b;
+                m.hg = d0.h;
+                m.part = d0.part;
+                m.j = d0.j;
+                m.ns = d0.ns;
+                m.n = d0.n;
+                m.ctx = d0.ctx;
+                m.bad = bad ? 1 : 0;
+                m.k = k;
+                m.nt = pair ? 2 : 1;
+                m.n1 = pair ? d1.n : 0;
+                m.end = 0;
+                meta[s] = m;
+                // release: consumers see the metadata once the phase completes
+                ptx::mbar_arrive_expect_tx(bar, (uint32_t)tx);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const TileDesc &d = t ? d1 : d0;
+                    if ((t == 1 && !pair) || withhold)
+                        continue;
+#pragma unroll
+                    for (int bx = 0; bx < 4; ++bx) {
+                        if (bx >= geo.bpt || bx * geo.tr >= d.n || !tile_ok(d, bx))
+                            continue;
+                        const int row = d.phys[bx] * p.block_size +
+                                        ((d.t0 + bx * geo.tr) & (p.block_size - 1));
+                        const uint32_t off = (uint32_t)(t * geo.kv_bytes + bx * geo.box_stride);
+                        ptx::tma_load_4d(stage + off, &tmap_k, 0, row, 0, h0, bar, policy);
+                        ptx::tma_load_4d(stage + (uint32_t)(2 * geo.kv_bytes) + off, &tmap_v, 0,
+                                         row, 0, h0, bar, policy);
+                    }
+                }
+            }
+            __syncwarp();
+            return true;
+        };
+        const int nk = R1 - R0;
+        int k = 0, q = 0;
+        TileDesc d0, d1;
+        bool pair = false;
+        auto next = [&]() {
+            d0 = desc(k);
+            pair = k + 1 < nk && d0.j + 1 < d0.ns;
+            d1 = pair ? desc(k + 1) : d0;
+        };
+        // Before the kernel ahead has completed, the K/V rows of the first
+        // stages are already fetched, as long as none of their tiles holds its
+        // sequence's last cached token (the only row the cache write ahead of
+        // this kernel stores), and their segments' query rows are prefetched
+        // into L2 (no value is read before the wait).
+        for (; q < spw && k < nk; ++q) {
+            next();
+            if (d0.t0 + d0.n >= d0.ctx || (pair && d1.t0 + d1.n >= d1.ctx))
+                break;
+            issue(q, k, d0, pair, d1);
+            if (d0.j == 0 || k == 0)
+                prefetch_query(d0);
+            k += pair ? 2 : 1;
+        }
+        ptx::grid_wait_prerequisites();
+        bool ok = true;
+        for (; k < nk; ++q) {
+            next();
+            if (!(ok = issue(q, k, d0, pair, d1)))
+                break;
+            if (d0.j == 0 || k == 0)
+                prefetch_query(d0);
+            k += pair ? 2 : 1;
+        }
+        // one end stage per consumer warp of a head (no copies: the arrival
+        // completes the phase)
+        for (int t = 0; ok && t < SUBS; ++t, ++q) {
+            const int s = q % spw;
+            if (q >= spw &&
+                !ptx::mbar_wait_bounded(empty0 + 8u * s, (uint32_t)(((q / spw) - 1) & 1),
+                                        p.wait_ns)) {
+                if (lane == 0)
+                    report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                StageMeta m = {};
+                m.end = 1;
+                meta[s] = m;
+                ptx::mbar_arrive(full0 + 8u * s);
+            }
+            __syncwarp();
+        }
+        if (!ok) {
+            // aborted: let copies still in flight land before exiting (bounded)
+            for (int x = max(0, q - spw); x < q; ++x)
+                ptx::mbar_wait_bounded(full0 + 8u * (x % spw), (uint32_t)((x / spw) & 1),
+                                       p.wait_ns);
+        }
+    };
     if constexpr (KV8) {
         // each role's code runs under its own register count
         if (warp >= kMaxHpc * SUBS) {
             ptx::setmaxnreg_dec<kRegsProducer8>();
             if (warp == pw)
-                producer();
+                producer8();
             return;
         }
         ptx::setmaxnreg_inc<kRegsConsumer8>();
@@ -1988,24 +2173,39 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
         ptx::red_max_relaxed_gpu_u64(counter_of(p, blockIdx.x, hl),
                                      (unsigned long long)p.epoch << 32);
 
-    // with SUBS warps per head, warp `sub` takes tiles R0 + sub, R0 + sub + SUBS, ...
-    for (int i = R0 + sub; i < R1; i += SUBS) {
-        const int k = i - R0;
-        const int s = k % spw;
-        if (!ptx::mbar_wait_bounded(full0 + 8u * s, (uint32_t)((k / spw) & 1), p.wait_ns)) {
+    // Stage q of the ring holds tile R0 + q (bf16, f32) or one or two
+    // consecutive tiles of one segment (FP8 cache, see producer8); with SUBS
+    // warps per head, warp `sub` takes stages sub, sub + SUBS, ...
+    int done = R0;        // tiles of the range up to this warp's last stage
+    int seg_prev = -1;    // segment of this warp's last stage
+    for (int q = sub;; q += SUBS) {
+        // (an FP8 producer marks the end of a non-empty range with end stages)
+        if (KV8 ? R0 >= R1 : R0 + q >= R1)
+            break;
+        const int s = q % spw;
+        if (!ptx::mbar_wait_bounded(full0 + 8u * s, (uint32_t)((q / spw) & 1), p.wait_ns)) {
             if (lane == 0)
                 report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
             timed_out = true;
-            lost = i;
+            lost = done;
             break;
         }
         const StageMeta d = meta[s];
-        const bool newseg = d.j < SUBS || k < SUBS;   // this warp's first tile of the segment
+        if constexpr (KV8) {
+            if (d.end)
+                break;
+        }
+        // the stage's first and last tiles
+        const int nt = KV8 ? d.nt : 1;
+        const int i = KV8 ? R0 + d.k : R0 + q;
+        const int i_end = i + nt - 1;
+        const bool newseg = i - d.j != seg_prev;   // this warp's first stage of the segment
         const uint32_t kreg = sbase + (uint32_t)(s * geo.stage_bytes);
-        const uint32_t vreg = kreg + (uint32_t)geo.kv_bytes;
+        const uint32_t vreg = kreg + (uint32_t)(geo.tps * geo.kv_bytes);
         const uint8_t *qslot = sgen + s * geo.stage_bytes + geo.q_off + hl * geo.q_head_bytes;
         if (newseg) {
             segS = i - d.j;
+            seg_prev = segS;
             seg_bad = false;
             if constexpr (KV8)
                 math.begin(static_cast<const uint8_t *>(p.q) +
@@ -2019,30 +2219,45 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
         if (d.bad)
             seg_bad = true;
         if (!seg_bad) {
-            if (d.n < kTile) {
-                // rows past the sequence end hold whatever the pool has there:
-                // zero them in this head's V (their weight is 0, but 0 * NaN is NaN)
-                constexpr int NCH = D * (KV8 ? 1 : (int)sizeof(T)) / 128;
-                const int lines = (kTile - d.n) * NCH;
-                for (int idx = lane; idx < lines * 8; idx += 32) {
-                    const int line = idx >> 3;
-                    const int t = d.n + line / NCH;
-                    const int ch = line % NCH;
-                    const uint32_t a = tile_addr<TR16>(vreg, hline, t, ch * 8 + (idx & 7), geo);
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0)
-                                 : "memory");
+            // V rows past the sequence end hold whatever the pool has there:
+            // zero them in this head's V (their weight is 0, but 0 * NaN is NaN)
+#pragma unroll 1
+            for (int t = 0; t < nt; ++t) {
+                const int n = t ? d.n1 : d.n;
+                const uint32_t vt = vreg + (uint32_t)(t * geo.kv_bytes);
+                if (n < kTile) {
+                    constexpr int NCH = D * (KV8 ? 1 : (int)sizeof(T)) / 128;
+                    const int lines = (kTile - n) * NCH;
+                    for (int idx = lane; idx < lines * 8; idx += 32) {
+                        const int line = idx >> 3;
+                        const int tk = n + line / NCH;
+                        const int ch = line % NCH;
+                        const uint32_t a = tile_addr<TR16>(vt, hline, tk, ch * 8 + (idx & 7), geo);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0)
+                                     : "memory");
+                    }
+                    __syncwarp();
                 }
-                __syncwarp();
             }
-            if constexpr (MMA)
-                math.tile(kreg, vreg, hline, d.n, p.scale_log2, geo, lane);
-            else
-                math.tile(kreg, vreg, hline, d.n, scores, geo, lane);
+#pragma unroll 1
+            for (int t = 0; t < nt; ++t) {
+                const int n = t ? d.n1 : d.n;
+                const uint32_t kt = kreg + (uint32_t)(t * geo.kv_bytes);
+                const uint32_t vt = vreg + (uint32_t)(t * geo.kv_bytes);
+                if constexpr (MMA)
+                    math.tile(kt, vt, hline, n, p.scale_log2, geo, lane);
+                else
+                    math.tile(kt, vt, hline, n, scores, geo, lane);
+            }
         }
+        done = i_end + 1;
         const int last = min(segS + d.ns, R1) - 1;   // the segment's last tile in the range
-        // (FP8) the warp handing its partial state over at a segment end keeps
-        // its stage: the state goes through the stage's lines of its head
-        const bool hand_over = SUBS > 1 && i + SUBS > last && i != last;
+        const bool is_final = i_end == last;
+        // (FP8) the warp whose stage comes just before the segment's final one
+        // (the other warp's) hands its partial state over and keeps its stage:
+        // the state goes through the stage's lines of its head.  The final
+        // stage holds the segment's last one or two tiles.
+        const bool hand_over = SUBS > 1 && !is_final && last - i_end <= 2;
         if (!hand_over) {
             // the stage may be refilled: order this warp's shared-memory
             // accesses before the producer's next TMA into it, then release it
@@ -2053,7 +2268,7 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
         }
 
         // ---- end of this warp's share of a segment (or of this CTA's range)
-        if (i + SUBS > last) {
+        if (is_final || hand_over) {
             if constexpr (SUBS > 1) {
                 // Two warps per head: the one holding the segment's last tile
                 // in the range completes it; the other hands it its partial
@@ -2062,7 +2277,7 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
                 const uint32_t xfull = ptx::smem_u32(st) + kXBars, xfree = xfull + 8u;
                 auto head_lines = [&](int stage, int v) {
                     return reinterpret_cast<float *>(sgen + stage * geo.stage_bytes +
-                                                     v * geo.kv_bytes + hline * 128);
+                                                     v * geo.tps * geo.kv_bytes + hline * 128);
                 };
                 if (hand_over) {
                     if (xc > 0 &&
@@ -2082,7 +2297,7 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
                     ++xc;
                     continue;
                 }
-                if (last - 1 >= max(segS, R0)) {
+                if (max(segS, R0) < i) {
                     if (!ptx::mbar_wait_bounded(xfull, (uint32_t)(xc & 1), p.wait_ns)) {
                         if (lane == 0)
                             report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
@@ -2090,8 +2305,8 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
                         lost = i;
                         break;
                     }
-                    // the other warp's last tile of the segment is last - 1
-                    const int sh = (last - 1 - R0) % spw;
+                    // the other warp's last stage of the segment is q - 1
+                    const int sh = (q - 1) % spw;
                     seg_bad |= math.absorb(head_lines(sh, 0), head_lines(sh, 1), st, lane);
                     // its stage may be refilled now (released on its behalf)
                     ptx::fence_proxy_async_smem();
