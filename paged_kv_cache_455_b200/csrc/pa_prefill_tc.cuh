@@ -384,14 +384,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         for (int j = 0; ok && j < ntiles; ++j) {
             const int s = j & 1;
-            if (__any_sync(kFull, *abort_flag != 0)) {
-                ok = false;
-                break;
-            }
-            if (!__all_sync(kFull, ptx::mbar_wait_bounded(sfull, (uint32_t)(j & 1),
-                                                          kWaitLimitNs))) {
-                ok = false;
-                break;
+            // S_j, and P buffer s free (P_{j-2} V_{j-2} done, long since in
+            // the usual case): one non-blocking test of both; only when it
+            // fails, the abort check and the bounded waits
+            const uint32_t pph = (uint32_t)(((j - 2) >> 1) & 1);
+            if (!__all_sync(kFull, ptx::mbar_test_wait(sfull, (uint32_t)(j & 1)) &&
+                                       (j < 2 || ptx::mbar_test_wait(pfree + 8u * s, pph)))) {
+                if (__any_sync(kFull, *abort_flag != 0) ||
+                    !__all_sync(kFull, ptx::mbar_wait_bounded(sfull, (uint32_t)(j & 1),
+                                                              kWaitLimitNs)) ||
+                    (j >= 2 && !__all_sync(kFull, ptx::mbar_wait_bounded(pfree + 8u * s, pph,
+                                                                         kWaitLimitNs)))) {
+                    ok = false;
+                    break;
+                }
             }
             ptx::tc_fence_after();
             float sv[kTcTile];
@@ -494,16 +500,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 l4[k & 3] += (e0 + e1) + (e2 + e3);
             }
             l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            if (j >= 2) {
-                // P buffer s is free once P_{j-2} V_{j-2} is done
-                if (!__all_sync(kFull, ptx::mbar_wait_bounded(pfree + 8u * s,
-                                                              (uint32_t)(((j - 2) >> 1) & 1),
-                                                              kWaitLimitNs))) {
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-            }
             ptx::tmem_st16(p_tm + lane_tm + (uint32_t)(s * 32), w0);
             ptx::tmem_st16(p_tm + lane_tm + (uint32_t)(s * 32 + 16), w1);
             if (tstart + kTcTile > ctx && ((ctx - tstart) & 15) != 0) {
