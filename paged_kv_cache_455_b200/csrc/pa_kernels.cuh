@@ -725,9 +725,15 @@ struct MmaMath8 {
     static_assert(G <= 8, "group must fit the N = 8 MMA");
     static constexpr int KS = D / 16;   // 16-byte units per row
     static constexpr int K32 = D / 32;  // 32-element reduction steps
+    // Up to four heads: the S product's N = 8 columns hold the hi parts of
+    // heads 0-3 (columns 0-3) and their lo parts (columns 4-7), so one MMA
+    // per reduction step covers both; lanes (r, c) and (r, c ^ 2) then add
+    // their halves and hold the same logits (heads 2 (c & 1), 2 (c & 1) + 1).
+    static constexpr bool PACK = G <= 4;
 
     uint32_t qh[K32][2];   // E4M3 hi parts of sigma * q, this lane's fragment
-    uint32_t ql[K32][2];   // E4M3 lo parts
+                           // (PACK: hi for columns 0-3, lo for columns 4-7)
+    uint32_t ql[PACK ? 1 : K32][2];   // E4M3 lo parts (not PACK)
     float sf[2];           // logit factor (scale_log2 / sigma) of heads 2c, 2c+1
     float acc[KS][4];
     float m[2];
@@ -742,6 +748,7 @@ struct MmaMath8 {
     __device__ __forceinline__ void begin(const uint8_t *qrows, int lane, float scale_log2)
     {
         const int r = lane >> 2, c = lane & 3;
+        const int hq = PACK ? (r & 3) : r;   // the head of this lane's column
         float x[K32][2][4];
         float amax = 0.f;
 #pragma unroll
@@ -749,8 +756,8 @@ struct MmaMath8 {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint2 w = make_uint2(0u, 0u);
-                if (r < G)
-                    w = __ldg(reinterpret_cast<const uint2 *>(qrows + (r * D + 32 * k + 16 * h + 4 * c) * 2));
+                if (hq < G)
+                    w = __ldg(reinterpret_cast<const uint2 *>(qrows + (hq * D + 32 * k + 16 * h + 4 * c) * 2));
                 x[k][h][0] = ptx::bf16lo_to_f32(w.x);
                 x[k][h][1] = ptx::bf16hi_to_f32(w.x);
                 x[k][h][2] = ptx::bf16lo_to_f32(w.y);
@@ -777,13 +784,18 @@ struct MmaMath8 {
                                                      y1 - ptx::f16hi_to_f32(f01));
                 const uint32_t l23 = f32x2_to_e4m3x2(y2 - ptx::f16lo_to_f32(f23),
                                                      y3 - ptx::f16hi_to_f32(f23));
-                qh[k][h] = h01 | (h23 << 16);
-                ql[k][h] = l01 | (l23 << 16);
+                if constexpr (PACK) {
+                    qh[k][h] = r < 4 ? h01 | (h23 << 16) : l01 | (l23 << 16);
+                } else {
+                    qh[k][h] = h01 | (h23 << 16);
+                    ql[k][h] = l01 | (l23 << 16);
+                }
             }
-        // lane (r, c) scales the logits of heads 2c, 2c+1, whose factors the
-        // lanes of rows 2c, 2c+1 computed
-        sf[0] = __shfl_sync(kFull, fac, 8 * c);
-        sf[1] = __shfl_sync(kFull, fac, 8 * c + 4);
+        // lane (r, c) scales the logits of heads 2c', 2c'+1 (c' = c, or c & 1
+        // with PACK), whose factors the lanes of rows 2c', 2c'+1 computed
+        const int cs = PACK ? (c & 1) : c;
+        sf[0] = __shfl_sync(kFull, fac, 8 * cs);
+        sf[1] = __shfl_sync(kFull, fac, 8 * cs + 4);
 #pragma unroll
         for (int k = 0; k < KS; ++k)
 #pragma unroll
@@ -803,17 +815,32 @@ struct MmaMath8 {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             c4[j][0] = c4[j][1] = c4[j][2] = c4[j][3] = 0.f;
-#pragma unroll
-        for (int k = 0; k < K32; ++k) {
-            uint32_t a[4];
-            ptx::ldsm_x4(kv_addr16(ks, hline, row, 2 * k + half), a);
-            ptx::mma_e4m3_16832(c4[2 * (k & 1)], a, qh[k][0], qh[k][1]);
-            ptx::mma_e4m3_16832(c4[2 * (k & 1) + 1], a, ql[k][0], ql[k][1]);
-        }
         float s[4];
+        if constexpr (PACK) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            s[i] = ((c4[0][i] + c4[1][i]) + (c4[2][i] + c4[3][i])) * sf[i & 1];
+            for (int k = 0; k < K32; ++k) {
+                uint32_t a[4];
+                ptx::ldsm_x4(kv_addr16(ks, hline, row, 2 * k + half), a);
+                ptx::mma_e4m3_16832(c4[k & 3], a, qh[k][0], qh[k][1]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float h = (c4[0][i] + c4[1][i]) + (c4[2][i] + c4[3][i]);
+                // hi (columns 0-3) plus lo (columns 4-7): the same sum in both lanes
+                s[i] = (h + __shfl_xor_sync(kFull, h, 2)) * sf[i & 1];
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < K32; ++k) {
+                uint32_t a[4];
+                ptx::ldsm_x4(kv_addr16(ks, hline, row, 2 * k + half), a);
+                ptx::mma_e4m3_16832(c4[2 * (k & 1)], a, qh[k][0], qh[k][1]);
+                ptx::mma_e4m3_16832(c4[2 * (k & 1) + 1], a, ql[k][0], ql[k][1]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                s[i] = ((c4[0][i] + c4[1][i]) + (c4[2][i] + c4[3][i])) * sf[i & 1];
+        }
         if (r >= n) {
             s[0] = -INFINITY;
             s[1] = -INFINITY;
