@@ -108,7 +108,7 @@ def test_fp8_mix(pa):
 
 
 @pytest.mark.parametrize("d,hq,hkv,bs", [(256, 16, 4, 16), (128, 8, 8, 32), (128, 16, 2, 16),
-                                         (256, 8, 1, 32), (128, 32, 4, 16)])
+                                         (256, 8, 1, 32), (128, 32, 4, 16), (256, 8, 4, 16)])
 def test_fp8_every_tail_length(pa, d, hq, hkv, bs):
     """Lengths 1 .. 40 (every position of the last tile), groups 1 to 8."""
     base = W.CONFIGS["qwen"]
