@@ -6,8 +6,8 @@
 //
 // One CTA per (sequence, KV head, 128 query rows); row r is (token r / G,
 // query head r % G of the group), so one K/V tile serves the whole group.
-// Warps 0-3 own one query row per thread; warp 4 issues the S MMAs, warp 7
-// the P V MMAs, warps 5 and 6 the TMA copies of K and V.
+// Warps 0-3 own one query row per thread; warp 4 issues the MMAs, warps 5
+// and 6 the TMA copies of K and V (warp 7 has no work).
 //
 //   producers (5, 6)    TMA: Q once; K tiles into four stages, V tiles into
 //                       three (one of each in the space Q held before it
@@ -16,13 +16,13 @@
 //                       lands as [8-token group][128-byte column][token]
 //                       [128 bytes] with 128-byte swizzle, so 8-token groups
 //                       are a fixed d * 16 bytes apart across the whole tile
-//   MMA (warps 4, 7)    S_j = Q K_j^T (M=128, N=64, K=16 steps) with Q read
-//                       from tensor memory and K from its stage (warp 4);
-//                       O += P_j V_j (M=128, N=d, K=16 per block) with P_j
-//                       read from tensor memory and V MN-major straight from
-//                       its stage (warp 7).  The two write disjoint tensor
-//                       memory and every reuse is guarded by a barrier, so
-//                       their waits overlap.  A K stage is free when its S is
+//   MMA (warp 4)        S_j = Q K_j^T (M=128, N=64, K=16 steps) with Q read
+//                       from tensor memory and K from its stage; O += P_j V_j
+//                       (M=128, N=d, K=16 per block) with P_j read from
+//                       tensor memory and V MN-major straight from its stage.
+//                       S_{j+1} is issued before P_{j-1} V_{j-1}, so that the
+//                       softmax gets it first.  The two write disjoint tensor
+//                       memory and every reuse is guarded by a barrier.  A K stage is free when its S is
 //                       done, a V stage and a P buffer when their P V is
 //                       (tcgen05.commit)
 //   softmax (warps 0-3) first move the CTA's Q rows from shared to tensor
@@ -270,9 +270,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == 4 || warp == 7) {
         // ================================================ MMA issue
         // Warp 4: S_0, then S_{j+1} once the softmax has read S_j out of
-        // tensor memory and K_{j+1} has landed.  Warp 7: P_j V_j once the
-        // softmax has written P_j and V_j has landed.  Each whole warp waits
-        // (suspending, so it takes no issue slots from the softmax warps);
+        // tensor memory and K_{j+1} has landed, and P_j V_j once the softmax
+        // has written P_j and V_j has landed (warp 7 idles here).  The whole
+        // warp waits (suspending, so it takes no issue slots from the softmax
+        // warps);
         // one elected lane, always lane 0, issues the MMAs and their commits
         // (a commit tracks the MMAs of its own thread).
         // descriptors: K is K-major, 8-token groups d * 16 bytes apart; V is
@@ -306,23 +307,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             __syncwarp();
         };
-        bool ok = true;
-        if (warp == 4) {
-            ok = ready(qready, 0, kfull, 0);
-            if (ok)
-                issue_s(0);
-            for (int j = 0; ok && j + 1 < ntiles; ++j) {
-                if (!(ok = ready(sfree, (uint32_t)(j & 1), kfull + 8u * ((j + 1) % kTcKStages),
-                                 (uint32_t)(((j + 1) / kTcKStages) & 1))))
-                    break;
-                issue_s(j + 1);
-            }
-        }
-        for (int j = 0; warp == 7 && ok && j < ntiles; ++j) {
+        auto issue_pv = [&](int j) -> bool {
             const int s = j & 1, vs = j % kTcVStages;
-            if (!(ok = ready(pready + 8u * s, (uint32_t)((j >> 1) & 1), vfull + 8u * vs,
-                             (uint32_t)((j / kTcVStages) & 1))))
-                break;
+            if (!ready(pready + 8u * s, (uint32_t)((j >> 1) & 1), vfull + 8u * vs,
+                       (uint32_t)((j / kTcVStages) & 1)))
+                return false;
             ptx::tc_fence_after();
             const int nbox = tc_boxes(j, ctx);
             const uint64_t vd = ptx::umma_desc_sw128(vstage(vs), 1024, tc_group_bytes(D));
@@ -335,6 +324,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 ptx::umma_commit(pfree + 8u * s);
             }
             __syncwarp();
+            return true;
+        };
+        // One issuing warp, in the order the softmax needs the results: once
+        // the softmax has read S_j, first S_{j+1}, then P_{j-1} V_{j-1} (its
+        // P was written before S_j was read).  The tensor pipe runs them in
+        // that order, so S_{j+1} does not queue behind a P V that only the
+        // softmax of tile j + 1 (its P buffer) or a rescale waits for.
+        bool ok = true;
+        if (warp == 4) {
+            ok = ready(qready, 0, kfull, 0);
+            if (ok)
+                issue_s(0);
+            for (int j = 0; ok && j < ntiles; ++j) {
+                if (j + 1 < ntiles) {
+                    if (!(ok = ready(sfree, (uint32_t)(j & 1),
+                                     kfull + 8u * ((j + 1) % kTcKStages),
+                                     (uint32_t)(((j + 1) / kTcKStages) & 1))))
+                        break;
+                    issue_s(j + 1);
+                }
+                if (j >= 1 && !(ok = issue_pv(j - 1)))
+                    break;
+            }
+            if (ok)
+                ok = issue_pv(ntiles - 1);
         }
         if (!ok && lane == 0) {
             report(p.dev_status, PA_DEV_WAIT_TIMEOUT);
@@ -384,17 +398,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         for (int j = 0; ok && j < ntiles; ++j) {
             const int s = j & 1;
-            // S_j, and P buffer s free (P_{j-2} V_{j-2} done, long since in
-            // the usual case): one non-blocking test of both; only when it
-            // fails, the abort check and the bounded waits
-            const uint32_t pph = (uint32_t)(((j - 2) >> 1) & 1);
-            if (!__all_sync(kFull, ptx::mbar_test_wait(sfull, (uint32_t)(j & 1)) &&
-                                       (j < 2 || ptx::mbar_test_wait(pfree + 8u * s, pph)))) {
+            // S_j: one non-blocking test; only when it fails, the abort check
+            // and the bounded wait
+            if (!__all_sync(kFull, ptx::mbar_test_wait(sfull, (uint32_t)(j & 1)))) {
                 if (__any_sync(kFull, *abort_flag != 0) ||
                     !__all_sync(kFull, ptx::mbar_wait_bounded(sfull, (uint32_t)(j & 1),
-                                                              kWaitLimitNs)) ||
-                    (j >= 2 && !__all_sync(kFull, ptx::mbar_wait_bounded(pfree + 8u * s, pph,
-                                                                         kWaitLimitNs)))) {
+                                                              kWaitLimitNs))) {
                     ok = false;
                     break;
                 }
@@ -500,6 +509,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 l4[k & 3] += (e0 + e1) + (e2 + e3);
             }
             l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            if (j >= 2) {
+                // P buffer s is free once P_{j-2} V_{j-2} is done (long since,
+                // in the usual case: one non-blocking test)
+                const uint32_t pph = (uint32_t)(((j - 2) >> 1) & 1);
+                if (!__all_sync(kFull, ptx::mbar_test_wait(pfree + 8u * s, pph)) &&
+                    !__all_sync(kFull, ptx::mbar_wait_bounded(pfree + 8u * s, pph, kWaitLimitNs))) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+            }
             ptx::tmem_st16(p_tm + lane_tm + (uint32_t)(s * 32), w0);
             ptx::tmem_st16(p_tm + lane_tm + (uint32_t)(s * 32 + 16), w1);
             if (tstart + kTcTile > ctx && ((ctx - tstart) & 15) != 0) {
