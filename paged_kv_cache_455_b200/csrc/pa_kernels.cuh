@@ -1851,8 +1851,11 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
             // so the stage never completes and the bounded waits run out
             const bool withhold = (int)blockIdx.x == p.withhold_cta && k == 1;
             const int h0 = d.h * hpc;
+            // (the first tile's query rows are read by the consumer warps
+            // themselves, straight after their wait)
+            const bool qcopy = newseg && k != 0;
             if (kv && lane == 0) {
-                int tx = newseg ? geo.q_bytes : 0;
+                int tx = qcopy ? geo.q_bytes : 0;
                 bool bad = false;
 #pragma unroll
                 for (int bx = 0; bx < 4; ++bx) {
@@ -1892,7 +1895,7 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
                                      bar, policy);
                 }
             }
-            if (q && newseg && !withhold && lane == 0 && geo.q_bytes > 0) {
+            if (q && qcopy && !withhold && lane == 0 && geo.q_bytes > 0) {
                 const T *qsrc = static_cast<const T *>(p.q) + ((int64_t)d.b * Hq + (int64_t)h0 * G) * D;
                 ptx::bulk_g2s(stage + (uint32_t)geo.q_off, qsrc, (uint32_t)geo.q_bytes, bar);
             }
@@ -2238,10 +2241,23 @@ __global__ void __launch_bounds__(KV8 ? kThreads8 : kThreads, 1)
                 math.begin(static_cast<const uint8_t *>(p.q) +
                                ((int64_t)d.b * Hq + (int64_t)(d.hg * hpc + hl) * G) * D * 2,
                            lane, p.scale_log2);
-            else if constexpr (MMA)
-                math.begin(qslot, lane);
-            else
-                math.begin(qslot, lane, p.scale_log2);
+            else {
+                if (q == 0) {
+                    // the range's first stage carries no query rows: this
+                    // warp copies its head's rows into the slot
+                    const uint4 *src = reinterpret_cast<const uint4 *>(
+                        static_cast<const T *>(p.q) +
+                        ((int64_t)d.b * Hq + (int64_t)(d.hg * hpc + hl) * G) * D);
+                    uint4 *dst = reinterpret_cast<uint4 *>(const_cast<uint8_t *>(qslot));
+                    for (int u = lane; u < geo.q_head_bytes / 16; u += 32)
+                        dst[u] = __ldg(src + u);
+                    __syncwarp();
+                }
+                if constexpr (MMA)
+                    math.begin(qslot, lane);
+                else
+                    math.begin(qslot, lane, p.scale_log2);
+            }
         }
         if (d.bad)
             seg_bad = true;
